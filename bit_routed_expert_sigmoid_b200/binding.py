@@ -1,0 +1,142 @@
+"""ctypes binding of libflint_moe.so (include/flint_moe.h): argument marshalling only.
+
+Every function here forwards to the C entry point of the same name. Pointers are plain integers
+(device addresses, e.g. torch's tensor.data_ptr(), or host addresses for *_host arguments);
+streams are cudaStream_t handles as integers (torch.cuda.Stream.cuda_stream). A non-OK status
+raises FlintError. Importing this module fails loudly when the library has not been built: there
+is no other implementation to fall back to.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libflint_moe.so")
+
+FLINT_OK = 0
+FLINT_ERR_INVALID_ARG = 1
+FLINT_ERR_UNSUPPORTED = 2
+FLINT_ERR_CUDA = 3
+FLINT_ERR_WORKSPACE = 4
+FLINT_ERR_DEVICE_CHECK = 5
+FLINT_ERR_TIMEOUT = 6
+
+FLINT_W_INT4_G128_FWHT128 = 0
+FLINT_W_NVFP4 = 1
+FLINT_FLAG_DEBUG_CHECKS = 0x1
+
+FLINT_BUF_LOGITS = 0
+FLINT_BUF_XQ = 1
+FLINT_BUF_YS = 2
+
+EXPORTS = (
+    "flint_moe_workspace_size", "flint_moe_create", "flint_moe_forward", "flint_moe_forward_host",
+    "flint_moe_routing", "flint_moe_intermediate", "flint_moe_error_word", "flint_moe_destroy",
+    "flint_moe_status_string",
+)
+
+
+class FlintError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {flint_moe_status_string(status)} (status {status})")
+
+
+class flint_moe_cfg(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("n_experts", ctypes.c_int), ("top_k", ctypes.c_int),
+                ("inter", ctypes.c_int), ("inter_shared", ctypes.c_int), ("fmt", ctypes.c_int),
+                ("t_max", ctypes.c_int), ("routed_scale", ctypes.c_float), ("norm_floor", ctypes.c_float),
+                ("flags", ctypes.c_uint)]
+
+
+class flint_moe_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("router_w", "gu_codes", "gu_scales", "gu_tscale", "dn_codes",
+                                                "dn_scales", "dn_tscale", "sh_gu", "sh_dn")]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m bit_routed_expert_sigmoid_b200.build` "
+                          "(the Flint MoE layer has no implementation other than its CUDA kernels)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, S, V = ctypes.POINTER, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+    sig = {
+        "flint_moe_workspace_size": (S, [P(flint_moe_cfg)]),
+        "flint_moe_create": (I, [P(flint_moe_cfg), P(flint_moe_weights), V, S, P(V)]),
+        "flint_moe_forward": (I, [V, V, I, V, V]),
+        "flint_moe_forward_host": (I, [V, V, I, V, V]),
+        "flint_moe_routing": (I, [V, V, V, V, V, V]),
+        "flint_moe_intermediate": (I, [V, I, V, S, V]),
+        "flint_moe_error_word": (I, [V, P(ctypes.c_uint)]),
+        "flint_moe_destroy": (I, [V]),
+        "flint_moe_status_string": (ctypes.c_char_p, [I]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def _check(status: int, where: str) -> None:
+    if status != FLINT_OK:
+        raise FlintError(status, where)
+
+
+def flint_moe_status_string(status: int) -> str:
+    return _lib.flint_moe_status_string(int(status)).decode()
+
+
+def flint_moe_workspace_size(cfg: flint_moe_cfg) -> int:
+    return int(_lib.flint_moe_workspace_size(ctypes.byref(cfg)))
+
+
+def flint_moe_create(cfg: flint_moe_cfg, weights: flint_moe_weights, workspace: int, workspace_bytes: int) -> int:
+    h = ctypes.c_void_p()
+    _check(_lib.flint_moe_create(ctypes.byref(cfg), ctypes.byref(weights), ctypes.c_void_p(workspace),
+                                 ctypes.c_size_t(workspace_bytes), ctypes.byref(h)), "flint_moe_create")
+    return h.value
+
+
+def flint_moe_forward(h: int, x: int, T: int, y: int, stream: int = 0) -> None:
+    _check(_lib.flint_moe_forward(ctypes.c_void_p(h), ctypes.c_void_p(x), int(T), ctypes.c_void_p(y),
+                                  ctypes.c_void_p(stream)), "flint_moe_forward")
+
+
+def flint_moe_forward_host(h: int, x_host: int, T: int, y_host: int, stream: int = 0) -> None:
+    _check(_lib.flint_moe_forward_host(ctypes.c_void_p(h), ctypes.c_void_p(x_host), int(T), ctypes.c_void_p(y_host),
+                                       ctypes.c_void_p(stream)), "flint_moe_forward_host")
+
+
+def flint_moe_routing(h: int, ids: int = 0, w: int = 0, offsets: int = 0, perm: int = 0, stream: int = 0) -> None:
+    _check(_lib.flint_moe_routing(ctypes.c_void_p(h), ctypes.c_void_p(ids), ctypes.c_void_p(w),
+                                  ctypes.c_void_p(offsets), ctypes.c_void_p(perm), ctypes.c_void_p(stream)),
+           "flint_moe_routing")
+
+
+def flint_moe_intermediate(h: int, which: int, dst: int, nbytes: int, stream: int = 0) -> None:
+    _check(_lib.flint_moe_intermediate(ctypes.c_void_p(h), int(which), ctypes.c_void_p(dst), ctypes.c_size_t(nbytes),
+                                       ctypes.c_void_p(stream)), "flint_moe_intermediate")
+
+
+def flint_moe_error_word(h: int) -> int:
+    out = ctypes.c_uint(0)
+    _check(_lib.flint_moe_error_word(ctypes.c_void_p(h), ctypes.byref(out)), "flint_moe_error_word")
+    return int(out.value)
+
+
+def flint_moe_destroy(h: int) -> None:
+    _check(_lib.flint_moe_destroy(ctypes.c_void_p(h)), "flint_moe_destroy")
+
+
+def raw_status(name: str, *args) -> int:
+    """Calls an entry point and returns its status code without raising (for argument-check tests)."""
+    return int(getattr(_lib, name)(*args))
+
+
+def library_handle():
+    return _lib

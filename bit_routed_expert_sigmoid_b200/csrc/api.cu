@@ -1,0 +1,280 @@
+// Host side of the Flint MoE C ABI: argument checks, workspace plan and the launch sequence.
+// The library allocates no device memory: weights, activations and workspace belong to the caller.
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "../../include/flint_moe.h"
+#include "kernels.cuh"
+
+using namespace flint;
+
+struct flint_moe_ctx {
+  flint_moe_cfg cfg;
+  flint_moe_weights w;
+  char* ws;
+  size_t ws_bytes;
+  // workspace carve-up
+  float* logits;
+  int* ids;
+  float* wts;
+  int* counts;
+  int* offsets;
+  int* perm;
+  int* inv;
+  int* active;
+  int* n_active;
+  unsigned* err;
+  __half* xq;
+  float* h32;
+  uint16_t* hs_hi;
+  uint16_t* hs_lo;
+  float* o;
+  float* ys;
+  uint16_t* x_stage;
+  uint16_t* y_stage;
+  int last_T;
+};
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+flint_status check_cfg(const flint_moe_cfg* c) {
+  if (!c) return FLINT_ERR_INVALID_ARG;
+  if (c->t_max < 1 || c->t_max > 16384) return FLINT_ERR_INVALID_ARG;
+  if (c->top_k < 1 || c->top_k > kMaxTopK) return FLINT_ERR_INVALID_ARG;
+  if (c->n_experts < c->top_k || c->n_experts <= 0) return FLINT_ERR_INVALID_ARG;
+  if (c->fmt != FLINT_W_INT4_G128_FWHT128 && c->fmt != FLINT_W_NVFP4) return FLINT_ERR_INVALID_ARG;
+  if (!(c->norm_floor > 0.f) || !(c->routed_scale == c->routed_scale)) return FLINT_ERR_INVALID_ARG;
+  if (c->hidden != kH || c->inter != kI || c->inter_shared != kIs) return FLINT_ERR_UNSUPPORTED;
+  if (c->n_experts % 32 != 0 || c->n_experts > kMaxE) return FLINT_ERR_UNSUPPORTED;
+  return FLINT_OK;
+}
+
+// Lays the workspace out; with base == nullptr only the size is computed.
+size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
+  const size_t T = c.t_max, E = c.n_experts, K = c.top_k, P = T * K;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return p;
+  };
+  char* p_logits = take(T * E * 4);
+  char* p_ids = take(P * 4);
+  char* p_wts = take(P * 4);
+  char* p_counts = take(E * 4);
+  char* p_offsets = take((E + 1) * 4);
+  char* p_perm = take(P * 4);
+  char* p_inv = take(P * 4);
+  char* p_active = take(E * 4);
+  char* p_nact = take(16);
+  char* p_err = take(16);
+  char* p_xq = take(T * kH * 2);
+  char* p_h32 = take(P * kI * 4);
+  char* p_hs_hi = take(T * kIs * 2);
+  char* p_hs_lo = take(T * kIs * 2);
+  char* p_o = take(P * kH * 4);
+  char* p_ys = take(T * kH * 4);
+  char* p_xs = take(T * kH * 2);
+  char* p_ys2 = take(T * kH * 2);
+  if (h) {
+    h->logits = reinterpret_cast<float*>(p_logits);
+    h->ids = reinterpret_cast<int*>(p_ids);
+    h->wts = reinterpret_cast<float*>(p_wts);
+    h->counts = reinterpret_cast<int*>(p_counts);
+    h->offsets = reinterpret_cast<int*>(p_offsets);
+    h->perm = reinterpret_cast<int*>(p_perm);
+    h->inv = reinterpret_cast<int*>(p_inv);
+    h->active = reinterpret_cast<int*>(p_active);
+    h->n_active = reinterpret_cast<int*>(p_nact);
+    h->err = reinterpret_cast<unsigned*>(p_err);
+    h->xq = reinterpret_cast<__half*>(p_xq);
+    h->h32 = reinterpret_cast<float*>(p_h32);
+    h->hs_hi = reinterpret_cast<uint16_t*>(p_hs_hi);
+    h->hs_lo = reinterpret_cast<uint16_t*>(p_hs_lo);
+    h->o = reinterpret_cast<float*>(p_o);
+    h->ys = reinterpret_cast<float*>(p_ys);
+    h->x_stage = reinterpret_cast<uint16_t*>(p_xs);
+    h->y_stage = reinterpret_cast<uint16_t*>(p_ys2);
+  }
+  return off;
+}
+
+#define FLINT_TRY(expr)                        \
+  do {                                         \
+    cudaError_t _e = (expr);                   \
+    if (_e != cudaSuccess) return FLINT_ERR_CUDA; \
+  } while (0)
+
+flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y, cudaStream_t s) {
+  const flint_moe_cfg& c = h->cfg;
+  const int E = c.n_experts, K = c.top_k;
+  const int fmt = c.fmt == FLINT_W_INT4_G128_FWHT128 ? kInt4 : kNvfp4;
+  FLINT_TRY(launch_router_logits(x, static_cast<const uint16_t*>(h->w.router_w), T, E, h->logits, s));
+  FLINT_TRY(launch_topk(h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, s));
+  FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, h->active, h->n_active, c.flags,
+                           h->err, s));
+  FLINT_TRY(launch_xq(x, T, fmt == kInt4 ? 1 : 0, h->xq, s));
+
+  GemvShared sh{};
+  sh.w_gu = static_cast<const uint8_t*>(h->w.sh_gu);
+  sh.w_dn = static_cast<const uint8_t*>(h->w.sh_dn);
+  sh.x = x;
+  sh.T = T;
+  sh.hs_hi = h->hs_hi;
+  sh.hs_lo = h->hs_lo;
+  sh.ys = h->ys;
+  FLINT_TRY(launch_gu_shared(sh, s));
+
+  const int groups = (T * K < E) ? T * K : E;
+  GemvRouted r{};
+  r.active = h->active;
+  r.n_active = h->n_active;
+  r.offsets = h->offsets;
+  r.perm = h->perm;
+  r.top_k = K;
+  r.xq = h->xq;
+  r.h_out = h->h32;
+  r.h_in = h->h32;
+  r.o_out = h->o;
+  r.codes = static_cast<const uint8_t*>(h->w.gu_codes);
+  r.scales = h->w.gu_scales;
+  r.tscale = h->w.gu_tscale;
+  FLINT_TRY(launch_gu_routed(r, fmt, groups, s));
+  r.codes = static_cast<const uint8_t*>(h->w.dn_codes);
+  r.scales = h->w.dn_scales;
+  r.tscale = h->w.dn_tscale;
+  FLINT_TRY(launch_dn_routed(r, fmt, groups, s));
+  FLINT_TRY(launch_dn_shared(sh, s));
+  FLINT_TRY(launch_combine(h->o, h->ys, h->wts, h->inv, T, K, c.routed_scale, y, s));
+  return FLINT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t flint_moe_workspace_size(const flint_moe_cfg* cfg) {
+  if (check_cfg(cfg) != FLINT_OK) return 0;
+  return plan(nullptr, *cfg, nullptr);
+}
+
+flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights* weights, void* workspace,
+                              size_t workspace_bytes, flint_moe_t* out) {
+  if (!out) return FLINT_ERR_INVALID_ARG;
+  *out = nullptr;
+  flint_status st = check_cfg(cfg);
+  if (st != FLINT_OK) return st;
+  if (!weights) return FLINT_ERR_INVALID_ARG;
+  const flint_moe_weights& w = *weights;
+  if (!aligned16(w.router_w) || !aligned16(w.gu_codes) || !aligned16(w.gu_scales) || !aligned16(w.dn_codes) ||
+      !aligned16(w.dn_scales) || !aligned16(w.sh_gu) || !aligned16(w.sh_dn))
+    return FLINT_ERR_INVALID_ARG;
+  if (cfg->fmt == FLINT_W_NVFP4 && (!w.gu_tscale || !w.dn_tscale)) return FLINT_ERR_INVALID_ARG;
+  if ((w.gu_tscale && (reinterpret_cast<uintptr_t>(w.gu_tscale) & 7u)) ||
+      (w.dn_tscale && (reinterpret_cast<uintptr_t>(w.dn_tscale) & 3u)))
+    return FLINT_ERR_INVALID_ARG;
+  const size_t need = plan(nullptr, *cfg, nullptr);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || workspace_bytes < need)
+    return FLINT_ERR_WORKSPACE;
+  flint_moe_ctx* h = new (std::nothrow) flint_moe_ctx();
+  if (!h) return FLINT_ERR_INVALID_ARG;
+  h->cfg = *cfg;
+  h->w = w;
+  h->ws = static_cast<char*>(workspace);
+  h->ws_bytes = workspace_bytes;
+  plan(h, *cfg, h->ws);
+  h->last_T = 0;
+  if (cudaMemset(h->err, 0, 16) != cudaSuccess) {
+    delete h;
+    return FLINT_ERR_CUDA;
+  }
+  *out = h;
+  return FLINT_OK;
+}
+
+flint_status flint_moe_forward(flint_moe_t h, const void* x, int T, void* y, void* stream) {
+  if (!h) return FLINT_ERR_INVALID_ARG;
+  if (T < 0 || T > h->cfg.t_max) return FLINT_ERR_INVALID_ARG;
+  if (T == 0) return FLINT_OK;
+  if (!aligned16(x) || !aligned16(y) || x == y) return FLINT_ERR_INVALID_ARG;
+  flint_status st = run_forward(h, static_cast<const uint16_t*>(x), T, static_cast<uint16_t*>(y),
+                                static_cast<cudaStream_t>(stream));
+  if (st == FLINT_OK) h->last_T = T;
+  return st;
+}
+
+flint_status flint_moe_forward_host(flint_moe_t h, const void* x_host, int T, void* y_host, void* stream) {
+  if (!h) return FLINT_ERR_INVALID_ARG;
+  if (T < 0 || T > h->cfg.t_max) return FLINT_ERR_INVALID_ARG;
+  if (T == 0) return FLINT_OK;
+  if (!x_host || !y_host) return FLINT_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(T) * kH * 2;
+  FLINT_TRY(cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, s));
+  flint_status st = run_forward(h, h->x_stage, T, h->y_stage, s);
+  if (st != FLINT_OK) return st;
+  h->last_T = T;
+  FLINT_TRY(cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, s));
+  return FLINT_OK;
+}
+
+flint_status flint_moe_routing(flint_moe_t h, int* ids, float* w, int* offsets, int* perm, void* stream) {
+  if (!h) return FLINT_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t P = static_cast<size_t>(h->last_T) * h->cfg.top_k;
+  if (ids && P) FLINT_TRY(cudaMemcpyAsync(ids, h->ids, P * 4, cudaMemcpyDeviceToDevice, s));
+  if (w && P) FLINT_TRY(cudaMemcpyAsync(w, h->wts, P * 4, cudaMemcpyDeviceToDevice, s));
+  if (offsets) FLINT_TRY(cudaMemcpyAsync(offsets, h->offsets, (h->cfg.n_experts + 1) * 4, cudaMemcpyDeviceToDevice, s));
+  if (perm && P) FLINT_TRY(cudaMemcpyAsync(perm, h->perm, P * 4, cudaMemcpyDeviceToDevice, s));
+  return FLINT_OK;
+}
+
+flint_status flint_moe_intermediate(flint_moe_t h, int which, void* dst, size_t bytes, void* stream) {
+  if (!h || !dst) return FLINT_ERR_INVALID_ARG;
+  const size_t T = h->last_T;
+  const void* src = nullptr;
+  size_t have = 0;
+  switch (which) {
+    case FLINT_BUF_LOGITS: src = h->logits; have = T * h->cfg.n_experts * 4; break;
+    case FLINT_BUF_XQ: src = h->xq; have = T * kH * 2; break;
+    case FLINT_BUF_YS: src = h->ys; have = T * kH * 4; break;
+    default: return FLINT_ERR_INVALID_ARG;
+  }
+  if (bytes > have) return FLINT_ERR_INVALID_ARG;
+  if (bytes) FLINT_TRY(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+  return FLINT_OK;
+}
+
+flint_status flint_moe_error_word(flint_moe_t h, unsigned* out) {
+  if (!h || !out) return FLINT_ERR_INVALID_ARG;
+  FLINT_TRY(cudaMemcpy(out, h->err, sizeof(unsigned), cudaMemcpyDeviceToHost));
+  FLINT_TRY(cudaMemset(h->err, 0, sizeof(unsigned)));
+  return FLINT_OK;
+}
+
+flint_status flint_moe_destroy(flint_moe_t h) {
+  delete h;
+  return FLINT_OK;
+}
+
+const char* flint_moe_status_string(flint_status s) {
+  switch (s) {
+    case FLINT_OK: return "ok";
+    case FLINT_ERR_INVALID_ARG: return "invalid argument";
+    case FLINT_ERR_UNSUPPORTED: return "unsupported shape or format";
+    case FLINT_ERR_CUDA: return "CUDA error";
+    case FLINT_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case FLINT_ERR_DEVICE_CHECK: return "device-side check failed";
+    case FLINT_ERR_TIMEOUT: return "bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,117 @@
+"""PyTorch plumbing around the C ABI: device buffers for one layer's weights and workspace.
+
+PyTorch only allocates device memory and provides streams here; every step of the forward runs in
+the library's CUDA kernels (binding.flint_moe_forward).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+H, I, IS = 2048, 512, 1024
+
+
+def _to_device(a, device):
+    if a is None:
+        return None
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).to(device)
+
+
+class FlintMoELayer:
+    """One Flint MoE layer resident on a CUDA device.
+
+    L is a dict of host arrays in the C-ABI storage layout (see synthetic.make_layer). The weights
+    are copied to the device once; the handle borrows them and the workspace."""
+
+    def __init__(self, L: dict, t_max: int, *, top_k: int = 6, device="cuda", flags: int = 0,
+                 routed_scale: float = 1.0, norm_floor: float = 2.0 ** -14):
+        self.device = torch.device(device)
+        self.E = int(L["E"])
+        self.top_k = top_k
+        self.t_max = t_max
+        fmt = B.FLINT_W_INT4_G128_FWHT128 if L["fmt"] == "int4" else B.FLINT_W_NVFP4
+        self.cfg = B.flint_moe_cfg(hidden=L["H"], n_experts=self.E, top_k=top_k, inter=L["I"],
+                                   inter_shared=L["Is"], fmt=fmt, t_max=t_max, routed_scale=routed_scale,
+                                   norm_floor=norm_floor, flags=flags)
+        self.tensors = {k: _to_device(L.get(k), self.device)
+                        for k in ("router_w", "gu_codes", "gu_scales", "gu_tscale", "dn_codes", "dn_scales",
+                                  "dn_tscale", "sh_gu", "sh_dn")}
+        ptr = {k: (v.data_ptr() if v is not None else None) for k, v in self.tensors.items()}
+        self.weights = B.flint_moe_weights(**ptr)
+        self.ws_bytes = B.flint_moe_workspace_size(self.cfg)
+        if self.ws_bytes == 0:
+            raise ValueError("configuration rejected by flint_moe_workspace_size")
+        self.workspace = torch.empty(self.ws_bytes + 256, dtype=torch.uint8, device=self.device)
+        base = self.workspace.data_ptr()
+        self.ws_ptr = (base + 255) // 256 * 256
+        self.handle = B.flint_moe_create(self.cfg, self.weights, self.ws_ptr, self.ws_bytes)
+
+    def weight_bytes(self) -> int:
+        return sum(v.numel() * v.element_size() for v in self.tensors.values() if v is not None)
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """x: [T][H] bf16 (or int16 bit patterns) on the device. Returns y [T][H] bf16."""
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty((T, H), dtype=torch.bfloat16, device=self.device)
+        s = (stream or torch.cuda.current_stream(self.device)).cuda_stream
+        B.flint_moe_forward(self.handle, x.data_ptr(), T, y.data_ptr(), s)
+        return y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None) -> None:
+        """x_host, y_host: [T][H] 16-bit host tensors (pinned for asynchronous copies)."""
+        s = (stream or torch.cuda.current_stream(self.device)).cuda_stream
+        B.flint_moe_forward_host(self.handle, x_host.data_ptr(), x_host.shape[0], y_host.data_ptr(), s)
+
+    def routing(self, T: int) -> dict:
+        K = self.top_k
+        out = {"ids": torch.empty((T, K), dtype=torch.int32, device=self.device),
+               "w": torch.empty((T, K), dtype=torch.float32, device=self.device),
+               "offsets": torch.empty((self.E + 1,), dtype=torch.int32, device=self.device),
+               "perm": torch.empty((T * K,), dtype=torch.int32, device=self.device)}
+        s = torch.cuda.current_stream(self.device).cuda_stream
+        B.flint_moe_routing(self.handle, out["ids"].data_ptr(), out["w"].data_ptr(), out["offsets"].data_ptr(),
+                            out["perm"].data_ptr(), s)
+        return out
+
+    def intermediate(self, which: int, T: int) -> torch.Tensor:
+        if which == B.FLINT_BUF_LOGITS:
+            t = torch.empty((T, self.E), dtype=torch.float32, device=self.device)
+        elif which == B.FLINT_BUF_XQ:
+            t = torch.empty((T, H), dtype=torch.float16, device=self.device)
+        elif which == B.FLINT_BUF_YS:
+            t = torch.empty((T, H), dtype=torch.float32, device=self.device)
+        else:
+            raise ValueError(which)
+        s = torch.cuda.current_stream(self.device).cuda_stream
+        B.flint_moe_intermediate(self.handle, which, t.data_ptr(), t.numel() * t.element_size(), s)
+        return t
+
+    def error_word(self) -> int:
+        return B.flint_moe_error_word(self.handle)
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            B.flint_moe_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def x_to_device(x_bits: np.ndarray, device="cuda") -> torch.Tensor:
+    """bf16 bit patterns [T][H] (uint16) -> device bf16 tensor."""
+    return torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def y_to_host_bits(y: torch.Tensor) -> np.ndarray:
+    return y.view(torch.int16).cpu().numpy().view(np.uint16)

@@ -1,0 +1,152 @@
+/*
+ * flint_moe.h - C ABI of a B200 (sm_100a) forward pass of one Flint mixture-of-experts layer.
+ *
+ * The layer (Aijuus/flint-w4exp, model summary; midagedev/bloomery issue #632, description;
+ * WaveCut/Flint-UD-Q4_K_XL-NInfer-v3 README, "What is inside"):
+ *
+ *   logits[t,e] = sum_j W_r[e,j] x[t,j]                       fp32 accumulation of exact bf16 products
+ *   s = sigmoid(logits); pick the top_k experts by score (no correction bias; ties to the lower id);
+ *   list the slots by ascending expert id; w_k = s_k / max(sum_k s_k, norm_floor)
+ *   routed expert e:  h = silu(Wg_e x') * (Wu_e x');  o = Wd_e h'
+ *   shared expert:    hs = silu(Sg x) * (Su x);       ys = Sd hs
+ *   y[t] = bf16( routed_scale * sum_k w_k o_k + ys )  (fixed slot order, one final rounding)
+ *
+ * For the int4 format x' and h' are x and h rotated per 128-segment by the normalised Sylvester
+ * Hadamard matrix Hn = H_128/sqrt(128) (the codes store W * blockdiag(Hn), Aijuus/flint-w4exp,
+ * weights row). For NVFP4, x' = x and h' = h (kekzle/Flint-NVFP4, W4A16).
+ *
+ * Conventions shared by every entry point:
+ *  - Every pointer argument that names layer data is a DEVICE pointer owned by the caller; the
+ *    library only borrows it and never allocates, frees or copies it. It must stay valid while
+ *    the handle uses it. Host pointers are named *_host.
+ *  - Device pointers must be 16-byte aligned; a misaligned or NULL pointer is rejected with
+ *    FLINT_ERR_INVALID_ARG before anything is launched.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Work is enqueued
+ *    asynchronously; no call synchronises the stream unless it says so.
+ *  - A handle is not re-entrant: its workspace holds one forward at a time, so calls on one
+ *    handle from several streams must be ordered by the caller.
+ *  - bf16 tensors are passed as raw 16-bit patterns (uint16_t or __nv_bfloat16 storage).
+ */
+#ifndef FLINT_MOE_H
+#define FLINT_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum flint_status {
+  FLINT_OK = 0,
+  FLINT_ERR_INVALID_ARG = 1,   /* NULL/misaligned pointer, T out of range, bad cfg value */
+  FLINT_ERR_UNSUPPORTED = 2,   /* a shape or format this build has no kernels for */
+  FLINT_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed */
+  FLINT_ERR_WORKSPACE = 4,     /* workspace NULL, misaligned or smaller than flint_moe_workspace_size */
+  FLINT_ERR_DEVICE_CHECK = 5,  /* a device-side check set the handle's error word */
+  FLINT_ERR_TIMEOUT = 6        /* a bounded device-side wait gave up */
+} flint_status;
+
+typedef enum flint_wformat {
+  /* int4 two's-complement codes, two per byte along K (low nibble = even K), one bf16 scale per
+   * 128 of K, stored against the per-128 Hadamard rotation (Aijuus/flint-w4exp, weights row). */
+  FLINT_W_INT4_G128_FWHT128 = 0,
+  /* NVFP4: E2M1 codes two per byte (low nibble = even column), one E4M3 (fn) scale per 16
+   * columns, one F32 tensor scale per Linear (kekzle/Flint-NVFP4, "What is in the files"). */
+  FLINT_W_NVFP4 = 1
+} flint_wformat;
+
+/* cfg.flags */
+#define FLINT_FLAG_DEBUG_CHECKS 0x1u  /* device-side range checks on ids / offsets; sets the error word */
+
+typedef struct flint_moe_cfg {
+  int hidden;         /* H: 2048 (the only width this build has kernels for) */
+  int n_experts;      /* E: a multiple of 32 in [32, 256] (Flint: 256) */
+  int top_k;          /* experts per token, 1..8 (Flint: 6) */
+  int inter;          /* I, routed SwiGLU width: 512 */
+  int inter_shared;   /* Is, shared-expert SwiGLU width: 1024 */
+  int fmt;            /* flint_wformat */
+  int t_max;          /* largest token count forward() will be given, 1..16384 */
+  float routed_scale; /* multiplies the routed sum (Flint: 1.0) */
+  float norm_floor;   /* floor of the selected-score sum (Flint: 2^-14) */
+  unsigned flags;     /* FLINT_FLAG_* */
+} flint_moe_cfg;
+
+/* Weight pointers (device, caller-owned, row-major [out][in]).
+ *   router_w   bf16 [E][H]
+ *   gu_codes   u8   [E][2I][H/2]   rows 0..I-1 are the gate projection, rows I..2I-1 the up projection
+ *   gu_scales  int4: bf16 [E][2I][H/128]; nvfp4: E4M3 [E][2I][H/16]
+ *   gu_tscale  f32  [E][2] (gate, up) tensor scales; required for nvfp4, optional (NULL = 1) for int4
+ *   dn_codes   u8   [E][H][I/2]
+ *   dn_scales  int4: bf16 [E][H][I/128]; nvfp4: E4M3 [E][H][I/16]
+ *   dn_tscale  f32  [E]; required for nvfp4, optional (NULL = 1) for int4
+ *   sh_gu      bf16 [2*Is][H]   gate rows then up rows
+ *   sh_dn      bf16 [H][Is]
+ * The int4 path multiplies codes by their bf16 scale in fp16, which is exact while
+ * 2^-14 <= |scale| <= 8188; out-of-range scales can be brought in range with a power of two folded
+ * into gu_tscale / dn_tscale (applied in fp32). */
+typedef struct flint_moe_weights {
+  const void* router_w;
+  const void* gu_codes;
+  const void* gu_scales;
+  const float* gu_tscale;
+  const void* dn_codes;
+  const void* dn_scales;
+  const float* dn_tscale;
+  const void* sh_gu;
+  const void* sh_dn;
+} flint_moe_weights;
+
+typedef struct flint_moe_ctx* flint_moe_t;
+
+/* Bytes of device workspace a handle with this cfg needs (0 if cfg is invalid). Depends on
+ * t_max, E, top_k and the widths only. */
+size_t flint_moe_workspace_size(const flint_moe_cfg* cfg);
+
+/* Validates cfg and the weight pointers, and records them with the caller's workspace (device,
+ * 256-byte aligned, at least flint_moe_workspace_size bytes, owned by the caller). Allocates no
+ * device memory; its only device work is one synchronous cudaMemset that clears the handle's
+ * 16-byte error word inside the workspace. On success *out receives a handle. */
+flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights* weights, void* workspace,
+                              size_t workspace_bytes, flint_moe_t* out);
+
+/* y = MoE(x) for T tokens: x bf16 [T][H] and y bf16 [T][H] are device pointers (distinct buffers).
+ * 0 <= T <= t_max (T = 0 is a no-op). Enqueues the kernels on `stream` and returns; the host never
+ * waits and nothing is copied back. T <= 8 takes the decode kernels, larger T the prefill ones. */
+flint_status flint_moe_forward(flint_moe_t h, const void* x, int T, void* y, void* stream);
+
+/* As flint_moe_forward, with x_host and y_host in host memory (pinned memory gives asynchronous
+ * copies): copies x into the workspace, runs the forward and copies y back, all on `stream`.
+ * The caller synchronises the stream before reading y_host. */
+flint_status flint_moe_forward_host(flint_moe_t h, const void* x_host, int T, void* y_host, void* stream);
+
+/* Device-to-device copies of the last forward's routing, enqueued on `stream` (any pointer may be
+ * NULL to skip it): ids int32 [T][top_k] and w f32 [T][top_k] in slot order (ascending expert id),
+ * offsets int32 [E+1] (exclusive prefix of per-expert counts), perm int32 [T*top_k] (position p
+ * holds t*top_k+k, ordered by expert then token). */
+flint_status flint_moe_routing(flint_moe_t h, int* ids, float* w, int* offsets, int* perm, void* stream);
+
+/* Intermediates of the last forward, for tests: device-to-device copy of `bytes` bytes. */
+enum {
+  FLINT_BUF_LOGITS = 0,   /* f32 [T][E] router logits */
+  FLINT_BUF_XQ = 1,       /* fp16 [T][H] the routed experts' input: rotated x (int4) or x (nvfp4),
+                             each 8-element block stored in the order 0,4,1,5,2,6,3,7 for int4 */
+  FLINT_BUF_YS = 2        /* f32 [T][H] shared-expert output */
+};
+flint_status flint_moe_intermediate(flint_moe_t h, int which, void* dst, size_t bytes, void* stream);
+
+/* Synchronously reads and clears the handle's device error word (set by device-side checks and
+ * bounded waits). *out = 0 when nothing was flagged. */
+flint_status flint_moe_error_word(flint_moe_t h, unsigned* out);
+
+/* Frees the host-side handle only; the caller still owns weights and workspace. NULL is a no-op. */
+flint_status flint_moe_destroy(flint_moe_t h);
+
+/* Static description of a status code. */
+const char* flint_moe_status_string(flint_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLINT_MOE_H */

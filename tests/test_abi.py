@@ -1,0 +1,94 @@
+"""The C-ABI library loads, exports every entry point include/flint_moe.h declares, and rejects bad
+arguments on the host before touching a device. No GPU needed."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_routed_expert_sigmoid_b200 import binding as B
+
+HEADER_DIR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(HEADER_DIR):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(HEADER_DIR, fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"\b(flint_\w+)\s*\(", src):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert "flint_moe_forward" in names and "flint_moe_create" in names
+    lib = B.library_handle()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(B.EXPORTS) <= set(names)
+
+
+def _cfg(**kw):
+    base = dict(hidden=2048, n_experts=256, top_k=6, inter=512, inter_shared=1024, fmt=0, t_max=64,
+                routed_scale=1.0, norm_floor=2.0 ** -14, flags=0)
+    base.update(kw)
+    return B.flint_moe_cfg(**base)
+
+
+def test_workspace_size_rules():
+    assert B.flint_moe_workspace_size(_cfg()) > 0
+    small, big = B.flint_moe_workspace_size(_cfg(t_max=8)), B.flint_moe_workspace_size(_cfg(t_max=2048))
+    assert 0 < small < big
+    for bad in (dict(hidden=4096), dict(inter=256), dict(n_experts=48), dict(n_experts=512), dict(top_k=0),
+                dict(top_k=9), dict(t_max=0), dict(fmt=7), dict(norm_floor=0.0), dict(n_experts=32, top_k=8)):
+        cfg = _cfg(**bad)
+        ok = bad == dict(n_experts=32, top_k=8)
+        assert (B.flint_moe_workspace_size(cfg) > 0) == ok, bad
+
+
+def test_create_rejects_bad_pointers_without_a_device():
+    cfg = _cfg()
+    w = B.flint_moe_weights(*([0x1000] * 9))
+    h = ctypes.c_void_p()
+    ws = B.flint_moe_workspace_size(cfg)
+    # null / misaligned weights
+    w0 = B.flint_moe_weights(*([0] * 9))
+    assert B.raw_status("flint_moe_create", ctypes.byref(cfg), ctypes.byref(w0), ctypes.c_void_p(0x100000),
+                        ctypes.c_size_t(ws), ctypes.byref(h)) == B.FLINT_ERR_INVALID_ARG
+    w1 = B.flint_moe_weights(*([0x1008] * 9))
+    assert B.raw_status("flint_moe_create", ctypes.byref(cfg), ctypes.byref(w1), ctypes.c_void_p(0x100000),
+                        ctypes.c_size_t(ws), ctypes.byref(h)) == B.FLINT_ERR_INVALID_ARG
+    # workspace too small / misaligned / missing
+    for ptr, size in ((0x100000, ws - 1), (0x100010, ws), (0, ws)):
+        assert B.raw_status("flint_moe_create", ctypes.byref(cfg), ctypes.byref(w), ctypes.c_void_p(ptr),
+                            ctypes.c_size_t(size), ctypes.byref(h)) == B.FLINT_ERR_WORKSPACE
+    # nvfp4 needs tensor scales
+    wn = B.flint_moe_weights(0x1000, 0x1000, 0x1000, None, 0x1000, 0x1000, None, 0x1000, 0x1000)
+    cfgn = _cfg(fmt=1)
+    assert B.raw_status("flint_moe_create", ctypes.byref(cfgn), ctypes.byref(wn), ctypes.c_void_p(0x100000),
+                        ctypes.c_size_t(B.flint_moe_workspace_size(cfgn)), ctypes.byref(h)) == B.FLINT_ERR_INVALID_ARG
+    # unsupported width
+    cfgu = _cfg(hidden=1024)
+    assert B.raw_status("flint_moe_create", ctypes.byref(cfgu), ctypes.byref(w), ctypes.c_void_p(0x100000),
+                        ctypes.c_size_t(ws), ctypes.byref(h)) == B.FLINT_ERR_UNSUPPORTED
+
+
+def test_calls_on_a_null_handle_fail_cleanly():
+    V = ctypes.c_void_p
+    assert B.raw_status("flint_moe_forward", V(0), V(0x1000), 1, V(0x2000), V(0)) == B.FLINT_ERR_INVALID_ARG
+    assert B.raw_status("flint_moe_forward_host", V(0), V(0x1000), 1, V(0x2000), V(0)) == B.FLINT_ERR_INVALID_ARG
+    assert B.raw_status("flint_moe_routing", V(0), V(0), V(0), V(0), V(0), V(0)) == B.FLINT_ERR_INVALID_ARG
+    assert B.raw_status("flint_moe_destroy", V(0)) == B.FLINT_OK
+    with pytest.raises(B.FlintError):
+        B.flint_moe_forward(0, 0x1000, 1, 0x2000)
+
+
+def test_status_strings():
+    for s in range(7):
+        assert B.flint_moe_status_string(s)
+    assert "unknown" in B.flint_moe_status_string(99)

@@ -1,0 +1,169 @@
+"""Parity of the CUDA layer (through the C ABI) against the fp64 oracle on seeded workloads."""
+
+import numpy as np
+import pytest
+
+from bit_routed_expert_sigmoid_b200 import synthetic as S
+from oracle import flint_moe_ref as R
+from tests import parity as PT
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # collected on CPU-only machines, skipped there
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+from bit_routed_expert_sigmoid_b200 import binding as B  # noqa: E402
+from bit_routed_expert_sigmoid_b200.layer import FlintMoELayer, x_to_device, y_to_host_bits  # noqa: E402
+
+_LAYERS = {}
+
+
+def layer(E, fmt, skew=False):
+    key = (E, fmt, skew)
+    if key not in _LAYERS:
+        _LAYERS[key] = S.make_layer(E, fmt, skew=skew)
+    return _LAYERS[key]
+
+
+def run(L, x_bits, top_k=6, t_max=None, flags=0):
+    T = x_bits.shape[0]
+    dev = FlintMoELayer(L, t_max=t_max or T, top_k=top_k, flags=flags)
+    xd = x_to_device(x_bits)
+    y = dev.forward(xd)
+    torch.cuda.synchronize()
+    return dev, xd, y
+
+
+def full_check(L, x_bits, top_k=6, keep=False):
+    T = x_bits.shape[0]
+    ref = R.moe_forward(L, x_bits, top_k=top_k, keep=keep)
+    dev, xd, y = run(L, x_bits, top_k=top_k)
+    PT.check_routing(dev.routing(T), ref, T, top_k)
+    st = PT.compare_y(y_to_host_bits(y), ref["y"])
+    assert st["finite"]
+    assert st["violations"] == 0, st
+    assert dev.error_word() == 0
+    return dev, xd, y, ref, st
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+def test_tiny_layer(fmt):
+    # E=32 routed experts, T=8 tokens
+    L = layer(32, fmt)
+    x = S.make_workload_x(8, 32)
+    full_check(L, x)
+
+
+@pytest.mark.parametrize("T", [1, 2, 4, 8])
+def test_decode_int4_full_layer(T):
+    L = layer(256, "int4")
+    full_check(L, S.make_workload_x(T, 256))
+
+
+@pytest.mark.parametrize("T", [1, 8])
+def test_decode_nvfp4_full_layer(T):
+    L = layer(256, "nvfp4")
+    full_check(L, S.make_workload_x(T, 256))
+
+
+@pytest.mark.parametrize("fmt,T", [("int4", 37), ("nvfp4", 37), ("int4", 300)])
+def test_ragged_token_counts(fmt, T):
+    L = layer(256, fmt)
+    full_check(L, S.make_workload_x(T, 256))
+
+
+def test_prefill_int4_full_size():
+    L = layer(256, "int4")
+    full_check(L, S.make_workload_x(2048, 256))
+
+
+def test_prefill_int4_skewed_loads():
+    L = layer(256, "int4", skew=True)
+    x = S.make_workload_x(2048, 256, skew=True)
+    dev, xd, y, ref, st = full_check(L, x)
+    counts = np.diff(ref["offsets"])
+    assert counts.max() > 300 and (counts == 0).any()          # skewed: hot and idle experts
+
+
+def test_prefill_nvfp4_full_size():
+    L = layer(256, "nvfp4")
+    full_check(L, S.make_workload_x(2048, 256))
+
+
+def test_top1_routing():
+    L = layer(32, "int4")
+    x = S.make_x(16)
+    ref = R.moe_forward(L, x, top_k=1)
+    keep = ref["gap"] >= 1e-4
+    dev, xd, y = run(L, x, top_k=1)
+    r = dev.routing(16)
+    np.testing.assert_array_equal(r["ids"].cpu().numpy()[keep], ref["ids"][keep])
+    np.testing.assert_array_equal(r["w"].cpu().numpy(), 1.0)
+    st = PT.compare_y(y_to_host_bits(y)[keep], ref["y"][keep])
+    assert st["violations"] == 0, st
+
+
+def test_all_tokens_on_six_experts():
+    # router column 0 strongly prefers experts 0..5, so each of them receives every token (several
+    # token chunks per expert) and the other experts receive none
+    L = dict(layer(256, "int4"))
+    rw = L["router_w"].copy()
+    rw[:, 0] = S.f32_to_bf16_bits(np.where(np.arange(256) < 6, 8.0, -8.0).astype(np.float32))
+    L["router_w"] = rw
+    x = S.make_x(64, skew=True)                                 # x[:, 0] = 1
+    dev, xd, y, ref, st = full_check(L, x)
+    np.testing.assert_array_equal(np.diff(ref["offsets"])[:6], 64)
+
+
+def test_intermediates_router_logits_and_rotation():
+    L = layer(256, "int4")
+    T = 8
+    x = S.make_workload_x(T, 256)
+    ref = R.moe_forward(L, x, keep=True)
+    dev, xd, y = run(L, x)
+    logits = dev.intermediate(B.FLINT_BUF_LOGITS, T).cpu().numpy()
+    np.testing.assert_allclose(logits, ref["logits"], rtol=0, atol=2e-5)
+    xq = dev.intermediate(B.FLINT_BUF_XQ, T).cpu().numpy().astype(np.float64)
+    xr = R.rotate_segments(R.bf16_to_f64(x))
+    np.testing.assert_allclose(PT.xq_natural_order(xq, True), xr, rtol=2 ** -11, atol=1e-6)
+    ys = dev.intermediate(B.FLINT_BUF_YS, T).cpu().numpy()
+    np.testing.assert_allclose(ys, ref["ys"], rtol=1e-4, atol=1e-4 * np.abs(ref["ys"]).max())
+
+
+def test_deterministic_across_runs():
+    L = layer(256, "int4")
+    x = S.make_workload_x(300, 256)
+    dev = FlintMoELayer(L, t_max=300)
+    xd = x_to_device(x)
+    a = dev.forward(xd).clone()
+    b = dev.forward(xd).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_forward_host_matches_device_forward():
+    L = layer(256, "int4")
+    T = 8
+    x = S.make_workload_x(T, 256)
+    dev = FlintMoELayer(L, t_max=T)
+    y_dev = dev.forward(x_to_device(x))
+    xh = torch.from_numpy(x.view(np.int16)).pin_memory()
+    yh = torch.empty((T, 2048), dtype=torch.int16).pin_memory()
+    dev.forward_host(xh, yh)
+    torch.cuda.synchronize()
+    assert torch.equal(yh, y_dev.view(torch.int16).cpu())
+
+
+def test_argument_errors_on_device():
+    L = layer(32, "int4")
+    dev = FlintMoELayer(L, t_max=8)
+    xd = x_to_device(S.make_x(8))
+    y = torch.empty((8, 2048), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(B.FlintError) as e:
+        B.flint_moe_forward(dev.handle, xd.data_ptr(), 9, y.data_ptr(), 0)
+    assert e.value.status == B.FLINT_ERR_INVALID_ARG
+    with pytest.raises(B.FlintError):
+        B.flint_moe_forward(dev.handle, xd.data_ptr() + 2, 4, y.data_ptr(), 0)
+    B.flint_moe_forward(dev.handle, xd.data_ptr(), 0, y.data_ptr(), 0)      # T = 0 is a no-op
+    torch.cuda.synchronize()
