@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Benchmark of the Flint MoE-layer forward on B200 (one JSON line on stdout from rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_int4] [--impl ours|reference]
+
+A step is one forward of the whole layer (router -> top-k -> permutation -> experts -> combine) over
+one batch of T synthetic tokens, inputs already resident in HBM. Between timed steps the L2 is
+flushed by writing a 256 MiB buffer (outside the timed events). Steps are timed on the device with
+CUDA events on the launching stream. With N > 1 (torchrun, one process per GPU) every rank runs its
+own replica on its own batch (the layer is token-parallel; no collective is needed) and the time is
+the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the reference arm of this repository: there is no
+reference implementation to install) on the host cores, on the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "MoE-layer tokens/s, HBM GB/s (% of 8 TB/s) at T=1..8; TFLOP/s % peak at T=2048"
+H, I, IS = 2048, 512, 1024
+HBM_NOMINAL_GBS = 8000.0
+BF16_DENSE_NOMINAL_TFLOPS = 2250.0
+FLUSH_BYTES = 256 << 20
+
+WORKLOADS = {
+    # name: (E, fmt, T, skew)
+    "decode_int4": (256, "int4", 8, False),
+    "prefill_int4": (256, "int4", 2048, False),
+    "prefill_int4_skew": (256, "int4", 2048, True),
+    "decode_nvfp4": (256, "nvfp4", 8, False),
+    "prefill_nvfp4": (256, "nvfp4", 2048, False),
+}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--workload", default="decode_int4", choices=sorted(WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-extras", action="store_true", help="skip the per-T decode and prefill side measurements")
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU-oracle baseline sample")
+    return p.parse_args()
+
+
+# --------------------------------------------------------------------------------------------- workload math
+
+def expert_bytes(fmt: str) -> int:
+    if fmt == "int4":
+        return 3 * H * I // 2 + (2 * I * (H // 128) + H * (I // 128)) * 2
+    return 3 * H * I // 2 + 2 * I * (H // 16) + H * (I // 16) + 3 * 4
+
+
+def algorithmic_bytes(E: int, fmt: str, T: int, n_active: int) -> int:
+    """Bytes one forward must move at least: the touched experts, the shared expert, the router, x and y."""
+    shared = (2 * IS * H + H * IS) * 2
+    router = E * H * 2
+    return n_active * expert_bytes(fmt) + shared + router + 2 * T * H * 2
+
+
+def grouped_gemm_flops(T: int, K: int = 6) -> int:
+    routed = 2 * T * K * (2 * I * H + H * I)
+    shared = 2 * T * (2 * IS * H + H * IS)
+    return routed + shared
+
+
+def stage_bytes(name: str, E: int, fmt: str, T: int, K: int, n_active: int) -> int:
+    """Algorithmic bytes of one kernel launch (weights it must stream plus its activations)."""
+    P = T * K
+    eb_gu = 2 * I * H // 2 + (2 * I * (H // 128) * 2 if fmt == "int4" else 2 * I * (H // 16) + 8)
+    eb_dn = H * I // 2 + (H * (I // 128) * 2 if fmt == "int4" else H * (I // 16) + 4)
+    return {
+        "router_logits": E * H * 2 + T * H * 2 + T * E * 4,
+        "gu_routed": n_active * eb_gu + T * H * 2 + P * I * 4,
+        "dn_routed": n_active * eb_dn + P * I * 4 + P * H * 4,
+        "gu_shared": 2 * IS * H * 2 + T * H * 2 + T * IS * 4,
+        "dn_shared": H * IS * 2 + T * IS * 4 + T * H * 4,
+        "combine": P * H * 4 + T * H * 4 + T * H * 2 + P * 8,
+    }.get(name, 0)
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch of `kernel` from the committed ncu summary, if it was taken on
+    the current kernel sources (source hash recorded beside the number); else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    cur = source_hash()
+    for line in open(path):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        f = dict(kv.split("=", 1) for kv in line.split())
+        if f.get("kernel") == kernel and f.get("workload") == workload and f.get("src") == cur:
+            return int(float(f["dram_bytes_per_launch"]))
+    return None
+
+
+def source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_routed_expert_sigmoid_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:12]
+
+
+# --------------------------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "50"], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons, power = [], None, set(), []
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+# --------------------------------------------------------------------------------------------- ours
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+
+    from bit_routed_expert_sigmoid_b200 import binding as B
+    from bit_routed_expert_sigmoid_b200 import synthetic as S
+    from bit_routed_expert_sigmoid_b200.layer import FlintMoELayer, x_to_device
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev_name = f"cuda:{local_rank}"
+    torch.cuda.set_device(dev_name)
+    E, fmt, T, skew = WORKLOADS[args.workload]
+    K_TOP = 6
+    L = S.make_layer(E, fmt, skew=skew)
+    t_max = max(T, 8)
+    layer = FlintMoELayer(L, t_max=max(t_max, 2048 if not args.no_extras else t_max), device=dev_name)
+    # each rank takes its own batch of token rows (weak scaling: T tokens per GPU)
+    redraws = S.redraw_table(E, skew=skew)
+    x_bits = S.make_x(T, skew=skew, redraws=redraws, first_row=0 if world == 1 else 0)
+    x = x_to_device(x_bits, dev_name)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev_name)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev_name)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed_steps(fn, K):
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        for i in range(K):
+            flush.zero_()
+            starts[i].record(stream)
+            fn()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+    fwd = lambda: layer.forward(x, y)  # noqa: E731
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd()
+    n_active = int((torch.diff(layer.routing(T)["offsets"]) > 0).sum().item())
+
+    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[0])
+                          if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local_rank)
+    clocks.start()
+    barrier()
+    wall0 = time.perf_counter()
+    step_ms = timed_steps(fwd, args.steps)
+    barrier()
+    wall1 = time.perf_counter()
+    total_ms = float(sum(step_ms))
+    if dist is not None:
+        tt = torch.tensor([total_ms], device=dev_name)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    value = world * T * args.steps / (total_ms / 1e3)
+
+    # per-kernel times of the same forward (instrumented pass)
+    n_st = B.flint_moe_stage_count(layer.handle, T)
+    names = [B.flint_moe_stage_name(layer.handle, T, i) for i in range(n_st)]
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)]
+    for e in evs:
+        e.record(stream)
+    torch.cuda.synchronize()
+    B.flint_moe_set_stage_events(layer.handle, [e.cuda_event for e in evs])
+    acc = np.zeros(n_st)
+    n_prof = min(args.steps, 200)
+    for _ in range(n_prof):
+        flush.zero_()
+        fwd()
+        torch.cuda.synchronize()
+        acc += [evs[i].elapsed_time(evs[i + 1]) for i in range(n_st)]
+    B.flint_moe_set_stage_events(layer.handle, None)
+    stage_ms = acc / n_prof
+    top = int(np.argmax(stage_ms))
+    peaks = measured_peaks()
+    st_bytes = stage_bytes(names[top], E, fmt, T, K_TOP, n_active)
+    achieved = st_bytes / (stage_ms[top] * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": names[top], "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": ncu_traffic(names[top], args.workload),
+                "algorithmic_bytes": st_bytes, "peak_source": peaks["source"] + " (burst copy)"}
+    stages = {n: round(float(t) * 1e3, 2) for n, t in zip(names, stage_ms)}
+
+    # end to end through the host-buffer entry point: H2D of x, forward, D2H of y
+    xh = torch.from_numpy(x_bits.view(np.int16)).pin_memory()
+    yh = torch.empty((T, H), dtype=torch.int16).pin_memory()
+    e2e_ms = timed_steps(lambda: layer.forward_host(xh, yh), min(args.steps, 500))
+    e2e_total = float(sum(e2e_ms))
+    if dist is not None:
+        tt = torch.tensor([e2e_total], device=dev_name)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_total = float(tt.item())
+    e2e = {"value": round(world * T * len(e2e_ms) / (e2e_total / 1e3), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
+           "ms_per_step": round(e2e_total / len(e2e_ms), 5)}
+
+    extras = {}
+    if not args.no_extras and args.workload == "decode_int4":
+        per_t = {}
+        for tt_ in (1, 2, 4, 8):
+            xt = x_to_device(S.make_x(tt_, redraws=redraws), dev_name)
+            yt = torch.empty((tt_, H), dtype=torch.bfloat16, device=dev_name)
+            f = lambda: layer.forward(xt, yt)  # noqa: E731
+            for _ in range(args.warmup):
+                f()
+            na = int((torch.diff(layer.routing(tt_)["offsets"]) > 0).sum().item())
+            ms = statistics.mean(timed_steps(f, min(args.steps, 1000)))
+            ab = algorithmic_bytes(E, fmt, tt_, na)
+            per_t[str(tt_)] = {"us": round(ms * 1e3, 2), "tokens_per_s": round(tt_ / (ms * 1e-3), 1),
+                               "distinct_experts": na, "algorithmic_MB": round(ab / 1e6, 3),
+                               "GB_per_s": round(ab / (ms * 1e-3) / 1e9, 1),
+                               "pct_of_8TBps": round(100 * ab / (ms * 1e-3) / 1e9 / HBM_NOMINAL_GBS, 2)}
+        extras["per_T"] = per_t
+    if not args.no_extras:
+        Tp = 2048
+        xp = x_to_device(S.make_x(Tp, redraws=redraws), dev_name)
+        yp = torch.empty((Tp, H), dtype=torch.bfloat16, device=dev_name)
+        f = lambda: layer.forward(xp, yp)  # noqa: E731
+        for _ in range(3):
+            f()
+        ms = statistics.mean(timed_steps(f, max(3, min(args.steps // 20, 50))))
+        fl = grouped_gemm_flops(Tp)
+        tf = fl / (ms * 1e-3) / 1e12
+        extras["prefill_T2048"] = {"us": round(ms * 1e3, 1), "tokens_per_s": round(Tp / (ms * 1e-3), 1),
+                                   "grouped_gemm_TFLOPs": round(tf, 2),
+                                   "pct_of_2250TF_dense_bf16": round(100 * tf / BF16_DENSE_NOMINAL_TFLOPS, 2),
+                                   "pct_of_measured_bf16": round(100 * tf / peaks["bf16_tflops"], 2)}
+    clk = clocks.stop()
+
+    result = None
+    if rank == 0:
+        ab = algorithmic_bytes(E, fmt, T, n_active)
+        cpu = cpu_baseline(args, L, x_bits, E) if world == 1 else None
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "w4a16: fp16 tensor-core MMA, fp32 accumulate",
+            "data": "synthetic (seeded; random-init weights of the Flint MoE layer shape)",
+            "config": {"workload": f"{args.workload}: E={E} top-6, H=2048, I=512, shared 1024, {fmt}, T={T} "
+                                   "tokens per GPU", "E": E, "T": T, "fmt": fmt, "distinct_experts": n_active,
+                       "l2": "flushed between timed steps (256 MiB write, outside the timed events)",
+                       "parallelism": f"replicas x{world} (token-parallel, no collective)"},
+            "hbm": {"algorithmic_bytes": ab, "GB_per_s": round(ab / (ms_per_step * 1e-3) / 1e9, 1),
+                    "pct_of_8TBps": round(100 * ab / (ms_per_step * 1e-3) / 1e9 / HBM_NOMINAL_GBS, 2),
+                    "pct_of_measured": round(100 * ab / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 2)},
+            "roofline": roofline, "stage_us": stages, "e2e": e2e,
+            "gpu_launches": n_st * args.steps, "clocks": clk, "cpu_baseline": cpu,
+            "wall_s_timed_region": round(wall1 - wall0, 4), **extras,
+        }
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    layer.close()
+    return result
+
+
+# --------------------------------------------------------------------------------------------- CPU oracle
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d["num_threads"] for d in threadpool_info() if d.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(args, L, x_bits, E) -> dict:
+    from oracle import flint_moe_ref as R
+    T = x_bits.shape[0]
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        R.moe_forward(L, x_bits)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= args.cpu_seconds or reps >= 1000:
+            break
+    return {"value": round(reps * T / el, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle forward of the same {T}-token batch, repeated {reps}x in {el:.1f} s"}
+
+
+def run_reference(args) -> dict:
+    from bit_routed_expert_sigmoid_b200 import synthetic as S
+    from oracle import flint_moe_ref as R
+    E, fmt, T, skew = WORKLOADS[args.workload]
+    L = S.make_layer(E, fmt, skew=skew)
+    # bounded sample: decode steps run whole; a prefill step runs the first 64 tokens of the batch
+    Ts = T if T <= 64 else 64
+    x_bits = S.make_x(Ts, skew=skew, redraws=S.redraw_table(E, skew=skew))
+    for _ in range(min(args.warmup, 1)):
+        R.moe_forward(L, x_bits)
+    steps = max(1, min(args.steps, 20 if Ts <= 8 else 5))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        R.moe_forward(L, x_bits)
+    el = time.perf_counter() - t0
+    value = steps * Ts / el
+    cores = blas_threads()
+    sample = f"fp64 oracle forward, {Ts} of the workload's {T} tokens per step, {steps} steps"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": 1,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": round(el / steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{args.workload}: E={E} top-6, H=2048, {fmt}, T={T}", "E": E, "T": T,
+                       "fmt": fmt},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    res = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

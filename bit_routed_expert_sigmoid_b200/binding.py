@@ -33,7 +33,7 @@ FLINT_BUF_YS = 2
 EXPORTS = (
     "flint_moe_workspace_size", "flint_moe_create", "flint_moe_forward", "flint_moe_forward_host",
     "flint_moe_routing", "flint_moe_intermediate", "flint_moe_error_word", "flint_moe_destroy",
-    "flint_moe_status_string",
+    "flint_moe_status_string", "flint_moe_set_stage_events", "flint_moe_stage_count", "flint_moe_stage_name",
 )
 
 
@@ -71,6 +71,9 @@ def _load():
         "flint_moe_error_word": (I, [V, P(ctypes.c_uint)]),
         "flint_moe_destroy": (I, [V]),
         "flint_moe_status_string": (ctypes.c_char_p, [I]),
+        "flint_moe_set_stage_events": (I, [V, P(V), I]),
+        "flint_moe_stage_count": (I, [V, I]),
+        "flint_moe_stage_name": (ctypes.c_char_p, [V, I, I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -131,6 +134,24 @@ def flint_moe_error_word(h: int) -> int:
 
 def flint_moe_destroy(h: int) -> None:
     _check(_lib.flint_moe_destroy(ctypes.c_void_p(h)), "flint_moe_destroy")
+
+
+def flint_moe_set_stage_events(h: int, events) -> None:
+    """events: sequence of cudaEvent_t handles (ints), or None to stop recording."""
+    if events is None:
+        _check(_lib.flint_moe_set_stage_events(ctypes.c_void_p(h), None, 0), "flint_moe_set_stage_events")
+        return
+    arr = (ctypes.c_void_p * len(events))(*events)
+    _check(_lib.flint_moe_set_stage_events(ctypes.c_void_p(h), arr, len(events)), "flint_moe_set_stage_events")
+
+
+def flint_moe_stage_count(h: int, T: int) -> int:
+    return int(_lib.flint_moe_stage_count(ctypes.c_void_p(h), int(T)))
+
+
+def flint_moe_stage_name(h: int, T: int, i: int) -> str:
+    r = _lib.flint_moe_stage_name(ctypes.c_void_p(h), int(T), int(i))
+    return r.decode() if r else ""
 
 
 def raw_status(name: str, *args) -> int:

@@ -34,6 +34,9 @@ struct flint_moe_ctx {
   uint16_t* x_stage;
   uint16_t* y_stage;
   int last_T;
+  // instrumentation (caller-owned cudaEvent_t handles)
+  cudaEvent_t events[32];
+  int n_events;
 };
 
 namespace {
@@ -106,6 +109,27 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
   return off;
 }
 
+const char* const kDecodeStages[] = {"router_logits", "topk", "permute", "xq", "gu_shared",
+                                     "gu_routed", "dn_routed", "dn_shared", "combine"};
+constexpr int kDecodeStageCount = sizeof(kDecodeStages) / sizeof(kDecodeStages[0]);
+
+int stage_count(const flint_moe_ctx*, int) { return kDecodeStageCount; }
+
+const char* stage_name(const flint_moe_ctx* h, int T, int i) {
+  return (i >= 0 && i < stage_count(h, T)) ? kDecodeStages[i] : nullptr;
+}
+
+// Records the next instrumentation event, if any.
+struct StageMarks {
+  flint_moe_ctx* h;
+  cudaStream_t s;
+  int next;
+  cudaError_t mark() {
+    if (h->n_events == 0 || next >= h->n_events) return cudaSuccess;
+    return cudaEventRecord(h->events[next++], s);
+  }
+};
+
 #define FLINT_TRY(expr)                        \
   do {                                         \
     cudaError_t _e = (expr);                   \
@@ -116,11 +140,17 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   const flint_moe_cfg& c = h->cfg;
   const int E = c.n_experts, K = c.top_k;
   const int fmt = c.fmt == FLINT_W_INT4_G128_FWHT128 ? kInt4 : kNvfp4;
+  StageMarks m{h, s, 0};
+  FLINT_TRY(m.mark());
   FLINT_TRY(launch_router_logits(x, static_cast<const uint16_t*>(h->w.router_w), T, E, h->logits, s));
+  FLINT_TRY(m.mark());
   FLINT_TRY(launch_topk(h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, s));
+  FLINT_TRY(m.mark());
   FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, h->active, h->n_active, c.flags,
                            h->err, s));
+  FLINT_TRY(m.mark());
   FLINT_TRY(launch_xq(x, T, fmt == kInt4 ? 1 : 0, h->xq, s));
+  FLINT_TRY(m.mark());
 
   GemvShared sh{};
   sh.w_gu = static_cast<const uint8_t*>(h->w.sh_gu);
@@ -131,6 +161,7 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   sh.hs_lo = h->hs_lo;
   sh.ys = h->ys;
   FLINT_TRY(launch_gu_shared(sh, s));
+  FLINT_TRY(m.mark());
 
   const int groups = (T * K < E) ? T * K : E;
   GemvRouted r{};
@@ -147,12 +178,16 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   r.scales = h->w.gu_scales;
   r.tscale = h->w.gu_tscale;
   FLINT_TRY(launch_gu_routed(r, fmt, groups, s));
+  FLINT_TRY(m.mark());
   r.codes = static_cast<const uint8_t*>(h->w.dn_codes);
   r.scales = h->w.dn_scales;
   r.tscale = h->w.dn_tscale;
   FLINT_TRY(launch_dn_routed(r, fmt, groups, s));
+  FLINT_TRY(m.mark());
   FLINT_TRY(launch_dn_shared(sh, s));
+  FLINT_TRY(m.mark());
   FLINT_TRY(launch_combine(h->o, h->ys, h->wts, h->inv, T, K, c.routed_scale, y, s));
+  FLINT_TRY(m.mark());
   return FLINT_OK;
 }
 
@@ -258,6 +293,25 @@ flint_status flint_moe_error_word(flint_moe_t h, unsigned* out) {
   FLINT_TRY(cudaMemset(h->err, 0, sizeof(unsigned)));
   return FLINT_OK;
 }
+
+flint_status flint_moe_set_stage_events(flint_moe_t h, void* const* events, int n) {
+  if (!h) return FLINT_ERR_INVALID_ARG;
+  if (!events) {
+    h->n_events = 0;
+    return FLINT_OK;
+  }
+  if (n < 1 || n > 32) return FLINT_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    if (!events[i]) return FLINT_ERR_INVALID_ARG;
+    h->events[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  h->n_events = n;
+  return FLINT_OK;
+}
+
+int flint_moe_stage_count(flint_moe_t h, int T) { return h ? stage_count(h, T) : 0; }
+
+const char* flint_moe_stage_name(flint_moe_t h, int T, int i) { return h ? stage_name(h, T, i) : nullptr; }
 
 flint_status flint_moe_destroy(flint_moe_t h) {
   delete h;

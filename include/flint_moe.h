@@ -139,6 +139,16 @@ flint_status flint_moe_intermediate(flint_moe_t h, int which, void* dst, size_t 
  * bounded waits). *out = 0 when nothing was flagged. */
 flint_status flint_moe_error_word(flint_moe_t h, unsigned* out);
 
+/* Instrumentation. With events != NULL every later forward records events[0] (a cudaEvent_t) on its
+ * stream before its first kernel and events[i+1] after its i-th kernel, so consecutive events time
+ * one kernel each; n must be at least flint_moe_stage_count(h, T) + 1 for the T used. The events are
+ * caller-owned. events == NULL turns recording off. */
+flint_status flint_moe_set_stage_events(flint_moe_t h, void* const* events, int n);
+
+/* Number of kernels forward(h, ., T, .) launches, and the name of the i-th (NULL if out of range). */
+int flint_moe_stage_count(flint_moe_t h, int T);
+const char* flint_moe_stage_name(flint_moe_t h, int T, int i);
+
 /* Frees the host-side handle only; the caller still owns weights and workspace. NULL is a no-op. */
 flint_status flint_moe_destroy(flint_moe_t h);
 
