@@ -34,6 +34,7 @@ EXPORTS = (
     "flint_moe_workspace_size", "flint_moe_create", "flint_moe_forward", "flint_moe_forward_host",
     "flint_moe_routing", "flint_moe_intermediate", "flint_moe_error_word", "flint_moe_destroy",
     "flint_moe_status_string", "flint_moe_set_stage_events", "flint_moe_stage_count", "flint_moe_stage_name",
+    "flint_moe_route_noalloc",
 )
 
 
@@ -74,6 +75,7 @@ def _load():
         "flint_moe_set_stage_events": (I, [V, P(V), I]),
         "flint_moe_stage_count": (I, [V, I]),
         "flint_moe_stage_name": (ctypes.c_char_p, [V, I, I]),
+        "flint_moe_route_noalloc": (I, [V, V, I, I, I, ctypes.c_float, V, V, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -152,6 +154,15 @@ def flint_moe_stage_count(h: int, T: int) -> int:
 def flint_moe_stage_name(h: int, T: int, i: int) -> str:
     r = _lib.flint_moe_stage_name(ctypes.c_void_p(h), int(T), int(i))
     return r.decode() if r else ""
+
+
+def flint_moe_route_noalloc(x: int, router_w: int, T: int, n_experts: int, top_k: int, norm_floor: float,
+                            ids: int, w: int, stream: int = 0) -> None:
+    """Routing (ids, w) for T <= 64 tokens using the library's fixed device scratch array instead of
+    a workspace: for callers that cannot allocate device memory."""
+    _check(_lib.flint_moe_route_noalloc(ctypes.c_void_p(x), ctypes.c_void_p(router_w), int(T), int(n_experts),
+                                        int(top_k), ctypes.c_float(norm_floor), ctypes.c_void_p(ids),
+                                        ctypes.c_void_p(w), ctypes.c_void_p(stream)), "flint_moe_route_noalloc")
 
 
 def raw_status(name: str, *args) -> int:
