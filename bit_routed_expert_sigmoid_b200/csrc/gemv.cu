@@ -7,149 +7,11 @@
 // The K order inside an MMA step is a permutation of the stored order; the activation buffers
 // are laid out with the same permutation, so every product pairs the right weight and activation.
 // Split-K partial sums are reduced through shared memory in a fixed warp order (deterministic).
+#include "frag.cuh"
 #include "kernels.cuh"
 
 namespace flint {
 
-namespace {
-
-// ---- A-fragment sources --------------------------------------------------------------------
-
-// One 128-wide K group of two rows for a thread: raw storage loaded with streaming loads.
-template <int FMT>
-struct RawA;
-
-template <>
-struct RawA<kInt4> {
-  uint4 r0, r1;  // 32 codes of row g, row g+8
-  __device__ __forceinline__ void load(const uint8_t* row0, const uint8_t* row1, int j, int t) {
-    r0 = ld_stream_v4(row0 + j * 64 + 16 * t);
-    r1 = ld_stream_v4(row1 + j * 64 + 16 * t);
-  }
-};
-
-template <>
-struct RawA<kNvfp4> {
-  uint4 r0, r1;
-  __device__ __forceinline__ void load(const uint8_t* row0, const uint8_t* row1, int j, int t) {
-    r0 = ld_stream_v4(row0 + j * 64 + 16 * t);
-    r1 = ld_stream_v4(row1 + j * 64 + 16 * t);
-  }
-};
-
-template <>
-struct RawA<kBf16> {
-  uint4 r0[4], r1[4];  // 32 bf16 of row g, row g+8
-  __device__ __forceinline__ void load(const uint8_t* row0, const uint8_t* row1, int j, int t) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      r0[q] = ld_stream_v4(row0 + (j * 128 + 32 * t) * 2 + 16 * q);
-      r1[q] = ld_stream_v4(row1 + (j * 128 + 32 * t) * 2 + 16 * q);
-    }
-  }
-};
-
-__device__ __forceinline__ uint32_t u4_word(const uint4& v, int q) {
-  return q == 0 ? v.x : (q == 1 ? v.y : (q == 2 ? v.z : v.w));
-}
-
-// B operand of one group for one thread: 32 stored activations (64 bytes) of token column g.
-struct RawB {
-  uint4 u[4];
-  __device__ __forceinline__ void load(const void* row, int j, int t, bool valid) {
-    if (valid) {
-      const uint8_t* p = static_cast<const uint8_t*>(row) + (j * 128 + 32 * t) * 2;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) u[q] = ld_nc_v4(p + 16 * q);
-    } else {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) u[q] = make_uint4(0, 0, 0, 0);
-    }
-  }
-  // step i uses stored elements 4i..4i+3
-  __device__ __forceinline__ uint32_t b0(int i) const { return (i & 1) ? u[i >> 1].z : u[i >> 1].x; }
-  __device__ __forceinline__ uint32_t b1(int i) const { return (i & 1) ? u[i >> 1].w : u[i >> 1].y; }
-};
-
-// Accumulates one 128-wide group of K into c (fp32) for rows g, g+8 and token columns 2t, 2t+1.
-// int4: the group scales sc0/sc1 (rows g, g+8) multiply the group's fp32 partial sums.
-// nvfp4: bs0/bs1 point at the rows' E4M3 block scales; codes x block scale are exact in fp16.
-template <int FMT, bool TWO_B>
-__device__ __forceinline__ void mma_group(float (&c)[4], const RawA<FMT>& A, const RawB& B, const RawB* B2, int j,
-                                          int t, float sc0, float sc1, const uint8_t* bs0, const uint8_t* bs1) {
-  if constexpr (FMT == kInt4) {
-    float part[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      uint32_t p0[4], p1[4];
-      int4x8_to_half2x4(u4_word(A.r0, w), p0);
-      int4x8_to_half2x4(u4_word(A.r1, w), p1);
-      {
-        const uint32_t a[4] = {p0[0], p1[0], p0[1], p1[1]};
-        mma_f16_16816(part, a, B.b0(2 * w), B.b1(2 * w));
-      }
-      {
-        const uint32_t a[4] = {p0[2], p1[2], p0[3], p1[3]};
-        mma_f16_16816(part, a, B.b0(2 * w + 1), B.b1(2 * w + 1));
-      }
-    }
-    c[0] = fmaf(sc0, part[0], c[0]);
-    c[1] = fmaf(sc0, part[1], c[1]);
-    c[2] = fmaf(sc1, part[2], c[2]);
-    c[3] = fmaf(sc1, part[3], c[3]);
-  } else if constexpr (FMT == kNvfp4) {
-    // the thread's 32 codes span two 16-column blocks: steps 0..3 and 4..7
-    const int blk = j * 8 + 2 * t;
-    uint32_t s0[2], s1[2];
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const uint32_t h0 = e4m3_to_half_bits(bs0[blk + q]);
-      const uint32_t h1 = e4m3_to_half_bits(bs1[blk + q]);
-      s0[q] = h0 | (h0 << 16);
-      s1[q] = h1 | (h1 << 16);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t w0 = u4_word(A.r0, i >> 1), w1 = u4_word(A.r1, i >> 1);
-      const int sh = (i & 1) * 16;
-      const uint32_t a0 = hmul2_u32(e2m1x2_to_half2(w0 >> sh), s0[i >> 2]);
-      const uint32_t a2 = hmul2_u32(e2m1x2_to_half2(w0 >> (sh + 8)), s0[i >> 2]);
-      const uint32_t a1 = hmul2_u32(e2m1x2_to_half2(w1 >> sh), s1[i >> 2]);
-      const uint32_t a3 = hmul2_u32(e2m1x2_to_half2(w1 >> (sh + 8)), s1[i >> 2]);
-      const uint32_t a[4] = {a0, a1, a2, a3};
-      mma_f16_16816(c, a, B.b0(i), B.b1(i));
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t a[4] = {u4_word(A.r0[i >> 1], (2 * i) & 3), u4_word(A.r1[i >> 1], (2 * i) & 3),
-                             u4_word(A.r0[i >> 1], (2 * i + 1) & 3), u4_word(A.r1[i >> 1], (2 * i + 1) & 3)};
-      mma_bf16_16816(c, a, B.b0(i), B.b1(i));
-      if constexpr (TWO_B) mma_bf16_16816(c, a, B2->b0(i), B2->b1(i));
-    }
-  }
-}
-
-// Fixed-order split-K reduction: warps ks = 0..KS-1 of row tile rt add their fragments in order.
-template <int KS>
-__device__ __forceinline__ bool reduce_splitk(float (&c)[4], float* red, int rt, int ks, int lane) {
-  float* mine = red + ((rt * KS + ks) * 32 + lane) * 4;
-  if (ks != 0) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) mine[q] = c[q];
-  }
-  __syncthreads();
-  if (ks != 0) return false;
-#pragma unroll
-  for (int w = 1; w < KS; ++w) {
-    const float* o = red + ((rt * KS + w) * 32 + lane) * 4;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) c[q] += o[q];
-  }
-  return true;
-}
-
-}  // namespace
 
 // ---------------------------------------------------------------------------------------------
 // Routed gate|up projection + SwiGLU. Grid (group slot, I/8): the CTA owns 8 gate rows and the 8
