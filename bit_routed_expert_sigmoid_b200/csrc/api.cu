@@ -1,5 +1,7 @@
 // Host side of the Flint MoE C ABI: argument checks, workspace plan and the launch sequence.
 // The library allocates no device memory: weights, activations and workspace belong to the caller.
+#include <cudaTypedefs.h>
+
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -24,9 +26,16 @@ struct flint_moe_ctx {
   int* inv;
   int* active;
   int* n_active;
+  int4* etab;
+  int* cnt;
   unsigned* err;
   __half* xq;
+  uint8_t* xq8;
+  float* xsc;
   float* h32;
+  __half* hq;
+  uint8_t* hq8;
+  float* hsc;
   uint16_t* hs_hi;
   uint16_t* hs_lo;
   float* o;
@@ -34,6 +43,8 @@ struct flint_moe_ctx {
   uint16_t* x_stage;
   uint16_t* y_stage;
   int last_T;
+  int n_sm;
+  CUtensorMap tm_gu, tm_sh_gu;  // tensor maps of the decode kernels' weight copies
   // instrumentation (caller-owned cudaEvent_t handles)
   cudaEvent_t events[32];
   int n_events;
@@ -59,6 +70,33 @@ flint_status check_cfg(const flint_moe_cfg* c) {
   return FLINT_OK;
 }
 
+// cuTensorMapEncodeTiled, from the driver through the runtime (no link-time driver dependency).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// 2-D map of `rows` rows of `row_bytes` bytes viewed as 32-bit words; box of box_words x box_rows.
+bool encode_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes, uint32_t box_words,
+                 uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {row_bytes / 4, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_words, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Lays the workspace out; with base == nullptr only the size is computed.
 size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
   const size_t T = c.t_max, E = c.n_experts, K = c.top_k, P = T * K;
@@ -77,9 +115,16 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
   char* p_inv = take(P * 4);
   char* p_active = take(E * 4);
   char* p_nact = take(16);
+  char* p_etab = take(kMaxActive * 2 * 16);
+  char* p_cnt = take(kCntInts * 4);
   char* p_err = take(16);
   char* p_xq = take(T * kH * 2);
+  char* p_xq8 = take(T * kH * 2);
+  char* p_xsc = take(T * (kH / kGroup) * 4);
   char* p_h32 = take(P * kI * 4);
+  char* p_hq = take(P * kI * 2);
+  char* p_hq8 = take(P * kI * 2);
+  char* p_hsc = take(P * (kI / kGroup) * 4);
   char* p_hs_hi = take(T * kIs * 2);
   char* p_hs_lo = take(T * kIs * 2);
   char* p_o = take(P * kH * 4);
@@ -96,9 +141,16 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
     h->inv = reinterpret_cast<int*>(p_inv);
     h->active = reinterpret_cast<int*>(p_active);
     h->n_active = reinterpret_cast<int*>(p_nact);
+    h->etab = reinterpret_cast<int4*>(p_etab);
+    h->cnt = reinterpret_cast<int*>(p_cnt);
     h->err = reinterpret_cast<unsigned*>(p_err);
     h->xq = reinterpret_cast<__half*>(p_xq);
     h->h32 = reinterpret_cast<float*>(p_h32);
+    h->hq = reinterpret_cast<__half*>(p_hq);
+    h->xq8 = reinterpret_cast<uint8_t*>(p_xq8);
+    h->xsc = reinterpret_cast<float*>(p_xsc);
+    h->hq8 = reinterpret_cast<uint8_t*>(p_hq8);
+    h->hsc = reinterpret_cast<float*>(p_hsc);
     h->hs_hi = reinterpret_cast<uint16_t*>(p_hs_hi);
     h->hs_lo = reinterpret_cast<uint16_t*>(p_hs_lo);
     h->o = reinterpret_cast<float*>(p_o);
@@ -109,14 +161,19 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
   return off;
 }
 
-const char* const kDecodeStages[] = {"router_logits", "topk", "permute", "xq", "gu_shared",
-                                     "gu_routed", "dn_routed", "dn_shared", "combine"};
-constexpr int kDecodeStageCount = sizeof(kDecodeStages) / sizeof(kDecodeStages[0]);
+// T <= kDecodeMaxT: three kernels chained by programmatic dependent launch; larger T: one kernel per step.
+const char* const kDecodeStages[] = {"route", "gate_up", "down"};
+const char* const kGemvStages[] = {"router_logits", "topk", "permute", "xq", "gu_shared",
+                                   "gu_routed", "dn_routed", "dn_shared", "combine"};
 
-int stage_count(const flint_moe_ctx*, int) { return kDecodeStageCount; }
+int stage_count(const flint_moe_ctx*, int T) {
+  return T <= kDecodeMaxT ? static_cast<int>(sizeof(kDecodeStages) / sizeof(kDecodeStages[0]))
+                          : static_cast<int>(sizeof(kGemvStages) / sizeof(kGemvStages[0]));
+}
 
 const char* stage_name(const flint_moe_ctx* h, int T, int i) {
-  return (i >= 0 && i < stage_count(h, T)) ? kDecodeStages[i] : nullptr;
+  if (i < 0 || i >= stage_count(h, T)) return nullptr;
+  return T <= kDecodeMaxT ? kDecodeStages[i] : kGemvStages[i];
 }
 
 // Records the next instrumentation event, if any.
@@ -142,6 +199,58 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   const int fmt = c.fmt == FLINT_W_INT4_G128_FWHT128 ? kInt4 : kNvfp4;
   StageMarks m{h, s, 0};
   FLINT_TRY(m.mark());
+  if (T <= kDecodeMaxT) {
+    DecodeParams d{};
+    d.tm_gu = h->tm_gu;
+    d.tm_sh_gu = h->tm_sh_gu;
+    d.fmt = fmt;
+    d.T = T;
+    d.E = E;
+    d.K = K;
+    d.floor_ = c.norm_floor;
+    d.routed_scale = c.routed_scale;
+    d.x = x;
+    d.wr = static_cast<const uint16_t*>(h->w.router_w);
+    d.gu_codes = static_cast<const uint8_t*>(h->w.gu_codes);
+    d.gu_scales = static_cast<const uint8_t*>(h->w.gu_scales);
+    d.gu_ts = h->w.gu_tscale;
+    d.dn_codes = static_cast<const uint8_t*>(h->w.dn_codes);
+    d.dn_scales = static_cast<const uint8_t*>(h->w.dn_scales);
+    d.dn_ts = h->w.dn_tscale;
+    d.sh_gu = static_cast<const uint8_t*>(h->w.sh_gu);
+    d.sh_dn = static_cast<const uint8_t*>(h->w.sh_dn);
+    d.y = y;
+    d.logits = h->logits;
+    d.ids = h->ids;
+    d.wts = h->wts;
+    d.counts = h->counts;
+    d.offsets = h->offsets;
+    d.perm = h->perm;
+    d.inv = h->inv;
+    d.active = h->active;
+    d.n_active = h->n_active;
+    d.etab = h->etab;
+    d.xq = h->xq;
+    d.h32 = h->h32;
+    d.hq = h->hq;
+    d.xq8 = h->xq8;
+    d.xsc = h->xsc;
+    d.hq8 = h->hq8;
+    d.hsc = h->hsc;
+    d.hs_hi = h->hs_hi;
+    d.hs_lo = h->hs_lo;
+    d.o = h->o;
+    d.ys = h->ys;
+    d.err = h->err;
+    d.cnt = h->cnt;
+    // with instrumentation events, one is recorded between consecutive kernels (which serialises them)
+    cudaEvent_t e1 = m.next < h->n_events ? h->events[m.next] : nullptr;
+    cudaEvent_t e2 = m.next + 1 < h->n_events ? h->events[m.next + 1] : nullptr;
+    m.next += (e1 ? 1 : 0) + (e2 ? 1 : 0);
+    FLINT_TRY(launch_decode(d, h->n_sm, s, e1, e2));
+    FLINT_TRY(m.mark());
+    return FLINT_OK;
+  }
   FLINT_TRY(launch_router_logits(x, static_cast<const uint16_t*>(h->w.router_w), T, E, h->logits, s));
   FLINT_TRY(m.mark());
   FLINT_TRY(launch_topk(h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, s));
@@ -226,7 +335,12 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
   h->ws_bytes = workspace_bytes;
   plan(h, *cfg, h->ws);
   h->last_T = 0;
-  if (cudaMemset(h->err, 0, 16) != cudaSuccess) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaMemset(h->err, 0, 16) != cudaSuccess || cudaMemset(h->cnt, 0, kCntInts * 4) != cudaSuccess ||
+      !encode_rows(&h->tm_gu, w.gu_codes, static_cast<uint64_t>(cfg->n_experts) * 2 * kI, kH / 2, 64, 8) ||
+      !encode_rows(&h->tm_sh_gu, w.sh_gu, 2 * kIs, kH * 2, 256, 2)) {
     delete h;
     return FLINT_ERR_CUDA;
   }

@@ -2,6 +2,8 @@
 // device code).
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace flint {
@@ -30,6 +32,64 @@ struct GemvShared {
   uint16_t* hs_lo;
   float* ys;                  // [T][H]
 };
+
+// ---- decode path (T <= kDecodeMaxT): three kernels chained by programmatic dependent launch ----
+constexpr int kDecodeMaxT = 8;
+constexpr int kMaxActive = 64;                 // active experts of a decode forward (T * top_k <= 64)
+// Counters of the decode kernels (ints in the workspace, zero between forwards; each is reset by
+// the last arriver that reads it).
+enum : int {
+  kCntRoute = 0,                               // route CTAs finished
+  kCntSeg = 32,                                // [kMaxActive][4] gate|up tiles finished per 128-segment of h
+  kCntBlk = kCntSeg + 4 * kMaxActive,          // [H/64] down tiles finished per 64-row block of y
+  kCntInts = kCntBlk + kH / 64
+};
+
+struct DecodeParams {
+  CUtensorMap tm_gu;              // gate|up codes as 32-bit words [E*2I][H/8], box 64 words x 8 rows
+  CUtensorMap tm_sh_gu;           // shared gate|up rows as 32-bit words [2Is][H/2], box 256 words x 2 rows
+  int fmt, T, E, K;
+  float floor_, routed_scale;
+  const uint16_t* x;              // [T][H] bf16
+  const uint16_t* wr;             // [E][H] bf16
+  const uint8_t* gu_codes;
+  const uint8_t* gu_scales;
+  const float* gu_ts;
+  const uint8_t* dn_codes;
+  const uint8_t* dn_scales;
+  const float* dn_ts;
+  const uint8_t* sh_gu;
+  const uint8_t* sh_dn;
+  uint16_t* y;                    // [T][H] bf16
+  float* logits;                  // [T][E]
+  int* ids;                       // [T][K]
+  float* wts;                     // [T][K]
+  int* counts;                    // [E]
+  int* offsets;                   // [E+1]
+  int* perm;                      // [P]
+  int* inv;                       // [T][K]
+  int* active;                    // [E]
+  int* n_active;
+  int4* etab;                     // [kMaxActive][2]: {e, offset, count, tokens (4 bits each)}, {ts_g, ts_u, ts_d, 0}
+  __half* xq;                     // [T][H] fp16 activation operand of gate|up (NVFP4; int4: kept for inspection)
+  uint8_t* xq8;                   // int4: [T][2][H] 16-bit fixed-point limbs (high s8, low u8) of Hn x
+  float* xsc;                     // int4: [T][H/128] value of one unit of the limbs' 16-bit integer, / 16
+  float* h32;                     // [P][I] SwiGLU output
+  __half* hq;                     // NVFP4: [P][I] fp16 activation operand of down
+  uint8_t* hq8;                   // int4: [P][2][I] limbs of Hn h
+  float* hsc;                     // int4: [P][I/128] unit of hq8, / 16
+  uint16_t* hs_hi;                // [T][Is] shared-expert SwiGLU output, bf16 pair
+  uint16_t* hs_lo;
+  float* o;                       // [P][H] routed down outputs
+  float* ys;                      // [T][H] shared-expert output
+  unsigned* err;
+  int* cnt;                       // [kCntInts]
+};
+
+// Launches the three decode kernels on `s`; with `events` (n_events >= 2) an event is recorded
+// after the first and second kernel (which serialises them; for instrumentation only).
+cudaError_t launch_decode(const DecodeParams& p, int n_sm, cudaStream_t s, cudaEvent_t ev_after_route,
+                          cudaEvent_t ev_after_gate_up);
 
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* wr, int T, int E, float* logits, cudaStream_t s);
 cudaError_t launch_topk(const float* logits, int T, int E, int K, float floor_, int* ids, float* wts, unsigned flags,

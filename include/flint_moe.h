@@ -105,14 +105,17 @@ size_t flint_moe_workspace_size(const flint_moe_cfg* cfg);
 
 /* Validates cfg and the weight pointers, and records them with the caller's workspace (device,
  * 256-byte aligned, at least flint_moe_workspace_size bytes, owned by the caller). Allocates no
- * device memory; its only device work is one synchronous cudaMemset that clears the handle's
- * 16-byte error word inside the workspace. On success *out receives a handle. */
+ * device memory; its only device work is two synchronous cudaMemsets that clear the handle's
+ * 16-byte error word and its arrival counters inside the workspace. On success *out receives a
+ * handle. */
 flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights* weights, void* workspace,
                               size_t workspace_bytes, flint_moe_t* out);
 
 /* y = MoE(x) for T tokens: x bf16 [T][H] and y bf16 [T][H] are device pointers (distinct buffers).
  * 0 <= T <= t_max (T = 0 is a no-op). Enqueues the kernels on `stream` and returns; the host never
- * waits and nothing is copied back. T <= 8 takes the decode kernels, larger T the prefill ones. */
+ * waits and nothing is copied back. T <= 8 takes the decode path: three kernels (route, gate|up,
+ * down + combine) chained by programmatic dependent launch, so each one starts streaming weights
+ * before its predecessor ends; larger T takes one kernel per step. */
 flint_status flint_moe_forward(flint_moe_t h, const void* x, int T, void* y, void* stream);
 
 /* As flint_moe_forward, with x_host and y_host in host memory (pinned memory gives asynchronous
@@ -142,7 +145,9 @@ flint_status flint_moe_error_word(flint_moe_t h, unsigned* out);
 /* Instrumentation. With events != NULL every later forward records events[0] (a cudaEvent_t) on its
  * stream before its first kernel and events[i+1] after its i-th kernel, so consecutive events time
  * one kernel each; n must be at least flint_moe_stage_count(h, T) + 1 for the T used. The events are
- * caller-owned. events == NULL turns recording off. */
+ * caller-owned. events == NULL turns recording off. On the decode path an event between two
+ * kernels removes their overlap, so per-kernel times then add up to more than an uninstrumented
+ * forward. */
 flint_status flint_moe_set_stage_events(flint_moe_t h, void* const* events, int n);
 
 /* Number of kernels forward(h, ., T, .) launches, and the name of the i-th (NULL if out of range). */
