@@ -85,7 +85,16 @@ def stage_bytes(name: str, E: int, fmt: str, T: int, K: int, n_active: int) -> i
     P = T * K
     eb_gu = 2 * I * H // 2 + (2 * I * (H // 128) * 2 if fmt == "int4" else 2 * I * (H // 16) + 8)
     eb_dn = H * I // 2 + (H * (I // 128) * 2 if fmt == "int4" else H * (I // 16) + 4)
+    sc_x = T * (H // 128) * 4 if fmt == "int4" else 0          # units of the 16-bit activation limbs
+    sc_h = P * (I // 128) * 4 if fmt == "int4" else 0
     return {
+        # decode path (T <= 8): three kernels
+        "route": E * H * 2 + T * H * 2 + T * E * 4 + T * H * 2 * (2 if fmt == "int4" else 1) + sc_x,
+        "gate_up": n_active * eb_gu + 2 * IS * H * 2 + T * H * 2 + T * H * 2 + sc_x + P * I * 4 + P * I * 2 + sc_h
+                   + 2 * T * IS * 2,
+        "down": n_active * eb_dn + H * IS * 2 + P * I * 2 + sc_h + 2 * T * IS * 2 + P * H * 4 * 2 + T * H * 4 * 2
+                + T * H * 2,
+        # larger T: one kernel per step
         "router_logits": E * H * 2 + T * H * 2 + T * E * 4,
         "gu_routed": n_active * eb_gu + T * H * 2 + P * I * 4,
         "dn_routed": n_active * eb_dn + P * I * 4 + P * H * 4,
@@ -153,6 +162,14 @@ class ClockSampler:
                                          stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return
+        # nvidia-smi's start-up can hold driver locks for a while: wait for its first sample (up to 10 s)
+        # so that it does not stall the launches of the timed region
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < 10.0 and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
 
     def stop(self) -> dict:
         if self.proc is None:
@@ -330,7 +347,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         result = {
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "w4a16: fp16 tensor-core MMA, fp32 accumulate",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": ("w4a16: int4 codes as exact int8 on the integer tensor cores against 16-bit fixed-point "
+                      "activations (int32 sums), fp32 accumulate" if fmt == "int4" and T <= 8 else
+                      "w4a16: fp16 tensor-core MMA, fp32 accumulate"),
             "data": "synthetic (seeded; random-init weights of the Flint MoE layer shape)",
             "config": {"workload": f"{args.workload}: E={E} top-6, H=2048, I=512, shared 1024, {fmt}, T={T} "
                                    "tokens per GPU", "E": E, "T": T, "fmt": fmt, "distinct_experts": n_active,

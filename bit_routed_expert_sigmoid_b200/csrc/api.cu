@@ -44,7 +44,7 @@ struct flint_moe_ctx {
   uint16_t* y_stage;
   int last_T;
   int n_sm;
-  CUtensorMap tm_gu, tm_sh_gu;  // tensor maps of the decode kernels' weight copies
+  CUtensorMap tm_gu, tm_sh_gu, tm_sh_dn;  // tensor maps of the decode kernels' weight copies
   // instrumentation (caller-owned cudaEvent_t handles)
   cudaEvent_t events[32];
   int n_events;
@@ -203,6 +203,7 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
     DecodeParams d{};
     d.tm_gu = h->tm_gu;
     d.tm_sh_gu = h->tm_sh_gu;
+    d.tm_sh_dn = h->tm_sh_dn;
     d.fmt = fmt;
     d.T = T;
     d.E = E;
@@ -340,7 +341,8 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
       cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       cudaMemset(h->err, 0, 16) != cudaSuccess || cudaMemset(h->cnt, 0, kCntInts * 4) != cudaSuccess ||
       !encode_rows(&h->tm_gu, w.gu_codes, static_cast<uint64_t>(cfg->n_experts) * 2 * kI, kH / 2, 64, 8) ||
-      !encode_rows(&h->tm_sh_gu, w.sh_gu, 2 * kIs, kH * 2, 256, 2)) {
+      !encode_rows(&h->tm_sh_gu, w.sh_gu, 2 * kIs, kH * 2, 256, 2) ||
+      !encode_rows(&h->tm_sh_dn, w.sh_dn, kH, kIs * 2, 128, 8)) {
     delete h;
     return FLINT_ERR_CUDA;
   }

@@ -47,6 +47,11 @@ namespace {
 constexpr uint64_t kWaitNs = FLINT_WAIT_NS;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
+// Asks L2 to fetch [ptr, ptr + bytes) from HBM (a hint; no completion to wait for).
+__device__ __forceinline__ void prefetch_l2(const void* ptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
@@ -58,17 +63,30 @@ __device__ __forceinline__ int atom_add_acq_rel(int* ctr, int v) {
   return old;
 }
 
-// Warp-collective arrival on a counter: the warp barrier orders every lane's earlier global writes
-// before lane 0's release, and lane 0's acquire before every lane's later reads. True in every lane
-// for the arrival that brings the counter to `target`.
-__device__ __forceinline__ bool warp_arrive_last(int* ctr, int target) {
-  __syncwarp();
-  int last = 0;
-  if ((threadIdx.x & 31) == 0) last = atom_add_acq_rel(ctr, 1) == target - 1;
-  last = __shfl_sync(kFull, last, 0);
-  __syncwarp();
-  return last != 0;
-}
+// A warp's arrival on a counter whose result is examined later: the warp barrier orders every
+// lane's earlier global writes before lane 0's release; the returned value is only waited for when
+// settle() reads it (typically one tile later), so the atomic's latency overlaps the next tile.
+// settle() returns the counter index if this arrival brought the counter to `target` (the warp is
+// the last arriver, and lane 0's acquire precedes every lane's later reads), else -1.
+struct PendingArrival {
+  int key = -1;                             // counter index, -1 when nothing is pending
+  int target = 0;
+  int old = 0;                              // lane 0: value before the add
+  __device__ __forceinline__ void arrive(int* cnt, int k, int tgt) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) old = atom_add_acq_rel(cnt + k, 1);
+    key = k;
+    target = tgt;
+  }
+  __device__ __forceinline__ int settle() {
+    if (key < 0) return -1;
+    const int o = __shfl_sync(kFull, old, 0);
+    const int k = key;
+    key = -1;
+    __syncwarp();
+    return o == target - 1 ? k : -1;
+  }
+};
 
 // 2-D tensor copy global -> this CTA's shared memory (one box of `map` at word x, row y), completing
 // its bytes on `bar`. x * 4 bytes is a multiple of 16 at every call.
@@ -147,20 +165,6 @@ __device__ __forceinline__ void int4_group(float (&acc)[4], const uint4& ra, con
 #pragma unroll
   for (int q = 0; q < 4; ++q)
     acc[q] = fmaf(static_cast<float>((dh[0][q] + dh[1][q]) * 256 + dl[0][q] + dl[1][q]), f[q], acc[q]);
-}
-
-// Limbs of token row `row` (hi row at row, lo row at row + width) for group j: the thread's 32 bytes.
-__device__ __forceinline__ void load_limbs(uint4 (&bh)[2], uint4 (&bl)[2], const uint8_t* row, int width, int j, int t,
-                                           bool valid) {
-  if (valid) {
-    const uint8_t* ph = row + j * 128 + 32 * t;
-    bh[0] = ld_nc_v4(ph);
-    bh[1] = ld_nc_v4(ph + 16);
-    bl[0] = ld_nc_v4(ph + width);
-    bl[1] = ld_nc_v4(ph + width + 16);
-  } else {
-    bh[0] = bh[1] = bl[0] = bl[1] = make_uint4(0, 0, 0, 0);
-  }
 }
 
 // One 128-wide K group of a 16-row NVFP4 tile into two fp32 accumulator sets (steps alternate).
@@ -278,18 +282,34 @@ __device__ __forceinline__ float key_float(unsigned k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
+// Routing of a forward in one CTA's shared memory. Every projection CTA derives it from the logits
+// (top-k and tables are a few microseconds of work for T <= 8): a CTA never waits for another.
+struct RouteSmem {
+  int ids[kMaxActive];                      // [T][K] selected experts, slots by ascending id
+  float w[kMaxActive];                      // [T][K] routing weights
+  int inv[kMaxActive];                      // [T][K] permuted position of each (token, slot)
+  int cnt[kMaxE];                           // table scratch: counts, then offsets
+  unsigned mask[kMaxE];                     // table scratch: token bit masks
+  int4 etab[kMaxActive][2];                 // active experts: {e, offset, count, tokens}, {ts_g, ts_u, ts_d, 0}
+  int na;                                   // number of active experts
+};
+
 // Top-k of one token (one warp): K rounds of a warp argmax on the fp32 logits. The router is
 // unbiased and sigmoid increasing, so the largest logits are the largest scores; ties go to the
 // lower id. The slots are listed by ascending expert id and w_k = s_k / max(sum of the chosen s,
 // floor), the sum taken in slot order (midagedev/bloomery issue #632, host-policy comment).
-__device__ void topk_token(const DecodeParams& p, int tok, int* s_ids) {
+__device__ __forceinline__ void topk_token(const DecodeParams& p, int tok, RouteSmem& rs, bool publish) {
   const int lane = threadIdx.x & 31;
   const int E = p.E, K = p.K, per = E >> 5;
+  const float floor_ = p.floor_;
+  const float* logits = p.logits;
+  int* g_ids = p.ids;
+  float* g_wts = p.wts;
   // element j of lane l is expert l + 32j; key 0 marks an element that is absent or taken (every
   // finite logit has a key above 0)
   unsigned key[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) key[j] = (j < per) ? float_key(__ldcg(p.logits + tok * E + lane + 32 * j)) : 0u;
+  for (int j = 0; j < 8; ++j) key[j] = (j < per) ? float_key(__ldcg(logits + tok * E + lane + 32 * j)) : 0u;
   int my_id = 0;
   float my_l = 0.f;
   for (int k = 0; k < K; ++k) {
@@ -320,21 +340,38 @@ __device__ void topk_token(const DecodeParams& p, int tok, int* s_ids) {
   }
   float sum = 0.f;
   for (int r = 0; r < K; ++r) sum += __shfl_sync(kFull, s_r, r);
-  const float denom = fmaxf(sum, p.floor_);
+  const float denom = fmaxf(sum, floor_);
   if (lane < K) {
-    p.ids[tok * K + rank] = my_id;
-    p.wts[tok * K + rank] = s / denom;
-    s_ids[tok * K + rank] = my_id;
+    rs.ids[tok * K + rank] = my_id;
+    rs.w[tok * K + rank] = s / denom;
+    if (publish) {
+      g_ids[tok * K + rank] = my_id;
+      g_wts[tok * K + rank] = s / denom;
+    }
   }
 }
 
-// Routing tables from the selected ids (one warp): counts, offsets (E+1), the experts with tokens
-// (ascending), the expert table for the projection kernels, and the expert-major permutation
-// (pairs of one expert by ascending token): perm[p] = t*K+k, inv[t*K+k] = p. Ranks come from bit
-// masks and scans, so the result does not depend on the order atomics run in.
-__device__ void build_tables(const DecodeParams& p, const int* s_ids, int* scr_cnt, unsigned* scr_mask) {
+// Routing tables from the selected ids (one warp): the experts with tokens (ascending) and their
+// table, and the expert-major permutation (pairs of one expert by ascending token): position p
+// holds t*K+k, inv[t*K+k] = p. Ranks come from bit masks and scans, so the result does not depend
+// on the order atomics run in. With `publish` the tables also go to global memory (counts,
+// offsets (E+1), perm, inv, active experts, their table) for inspection.
+__device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& rs, bool publish) {
+  int* scr_cnt = rs.cnt;
+  unsigned* scr_mask = rs.mask;
+  const int* s_ids = rs.ids;
   const int lane = threadIdx.x & 31;
   const int T = p.T, E = p.E, K = p.K, P = T * K;
+  // parameters in registers: the table stores below could otherwise force them to be reloaded
+  const float* gu_ts = p.gu_ts;
+  const float* dn_ts = p.dn_ts;
+  int* g_counts = p.counts;
+  int* g_offsets = p.offsets;
+  int* g_active = p.active;
+  int4* g_etab = p.etab;
+  int* g_n_active = p.n_active;
+  int* g_perm = p.perm;
+  int* g_inv = p.inv;
   for (int e = lane; e < kMaxE; e += 32) {
     scr_cnt[e] = 0;
     scr_mask[e] = 0u;
@@ -344,13 +381,15 @@ __device__ void build_tables(const DecodeParams& p, const int* s_ids, int* scr_c
   if (lane < P) { atomicAdd(&scr_cnt[id0], 1); atomicOr(&scr_mask[id0], 1u << (lane / K)); }
   if (lane + 32 < P) { atomicAdd(&scr_cnt[id1], 1); atomicOr(&scr_mask[id1], 1u << ((lane + 32) / K)); }
   __syncwarp();
-  int cnt[8], s = 0, a = 0;                        // lane holds experts 8*lane .. 8*lane+7
-#pragma unroll
+  // lane holds experts 8*lane .. 8*lane+7 (loops kept rolled: this code runs once per CTA, where
+  // instruction fetches dominate)
+  int s = 0, a = 0;
+#pragma unroll 1
   for (int j = 0; j < 8; ++j) {
     const int e = 8 * lane + j;
-    cnt[j] = (e < E) ? scr_cnt[e] : 0;
-    s += cnt[j];
-    a += cnt[j] > 0;
+    const int c = e < E ? scr_cnt[e] : 0;
+    s += c;
+    a += c > 0;
   }
   int si = s, ai = a;
 #pragma unroll
@@ -360,33 +399,45 @@ __device__ void build_tables(const DecodeParams& p, const int* s_ids, int* scr_c
   }
   int off = si - s, slot = ai - a;
   __syncwarp();
-#pragma unroll
+#pragma unroll 1
   for (int j = 0; j < 8; ++j) {
     const int e = 8 * lane + j;
-    if (e < E) {
-      p.counts[e] = cnt[j];
-      p.offsets[e] = off;
-      scr_cnt[e] = off;
-      if (cnt[j] > 0) {
-        const unsigned m = scr_mask[e];
-        unsigned toks = 0;
-        int n = 0;
-        for (int tt = 0; tt < T; ++tt)
-          if ((m >> tt) & 1u) toks |= static_cast<unsigned>(tt) << (4 * n++);
-        const float tsg = p.gu_ts ? p.gu_ts[2 * e] : 1.f;
-        const float tsu = p.gu_ts ? p.gu_ts[2 * e + 1] : 1.f;
-        const float tsd = p.dn_ts ? p.dn_ts[e] : 1.f;
-        p.active[slot] = e;
-        p.etab[2 * slot] = make_int4(e, off, cnt[j], static_cast<int>(toks));
-        p.etab[2 * slot + 1] = make_int4(__float_as_int(tsg), __float_as_int(tsu), __float_as_int(tsd), 0);
-        ++slot;
-      }
-      off += cnt[j];
+    if (e >= E) break;
+    const int c = scr_cnt[e];
+    if (publish) {
+      g_counts[e] = c;
+      g_offsets[e] = off;
     }
+    scr_cnt[e] = off;
+    if (c > 0) {
+      const unsigned m = scr_mask[e];
+      unsigned toks = 0;
+      int n = 0;
+#pragma unroll 1
+      for (int tt = 0; tt < T; ++tt)
+        if ((m >> tt) & 1u) toks |= static_cast<unsigned>(tt) << (4 * n++);
+      const float tsg = gu_ts ? __ldg(gu_ts + 2 * e) : 1.f;
+      const float tsu = gu_ts ? __ldg(gu_ts + 2 * e + 1) : 1.f;
+      const float tsd = dn_ts ? __ldg(dn_ts + e) : 1.f;
+      const int4 t0 = make_int4(e, off, c, static_cast<int>(toks));
+      const int4 t1 = make_int4(__float_as_int(tsg), __float_as_int(tsu), __float_as_int(tsd), 0);
+      rs.etab[slot][0] = t0;
+      rs.etab[slot][1] = t1;
+      if (publish) {
+        g_active[slot] = e;
+        g_etab[2 * slot] = t0;
+        g_etab[2 * slot + 1] = t1;
+      }
+      ++slot;
+    }
+    off += c;
   }
   if (lane == 31) {
-    p.offsets[E] = si;
-    *p.n_active = ai;
+    rs.na = ai;
+    if (publish) {
+      g_offsets[E] = si;
+      *g_n_active = ai;
+    }
   }
   __syncwarp();
 #pragma unroll
@@ -395,19 +446,28 @@ __device__ void build_tables(const DecodeParams& p, const int* s_ids, int* scr_c
     if (q < P) {
       const int id = h ? id1 : id0, tt = q / K;
       const int pos = scr_cnt[id] + __popc(scr_mask[id] & ((1u << tt) - 1u));
-      p.perm[pos] = q;
-      p.inv[q] = pos;
+      rs.inv[q] = pos;
+      if (publish) {
+        g_perm[pos] = q;
+        g_inv[q] = pos;
+      }
     }
   }
+}
+
+// A group of `nw` warps (group-relative warp index gw; named barrier `bar` over the group's
+// threads): top-k of every token (a token per warp), then the tables (the group's first warp).
+__device__ __noinline__ void route_group(const DecodeParams& p, RouteSmem& rs, bool publish, int gw, int nw,
+                                            int bar) {
+  for (int tok = gw; tok < p.T; tok += nw) topk_token(p, tok, rs, publish);
+  named_bar_sync(bar, nw * 32);
+  if (gw == 0) build_tables(p, rs, publish);
+  named_bar_sync(bar, nw * 32);
 }
 
 __global__ void __launch_bounds__(kRouteWarps * 32) decode_route_kernel(const __grid_constant__ DecodeParams p) {
   pdl_trigger();                                   // the gate|up kernel may start its shared-expert tiles
   __shared__ __align__(128) uint16_t xs[kDecodeMaxT * kH];
-  __shared__ int scr_cnt[kMaxE];
-  __shared__ unsigned scr_mask[kMaxE];
-  __shared__ int s_ids[kMaxActive];
-  __shared__ int s_last;
   __shared__ uint64_t xbar;
   const int warp = threadIdx.x >> 5;
   const int gw = blockIdx.x * kRouteWarps + warp, nw = gridDim.x * kRouteWarps;
@@ -426,30 +486,36 @@ __global__ void __launch_bounds__(kRouteWarps * 32) decode_route_kernel(const __
     route_row(p, e, w, xs);
   }
   for (int sg = gw; sg < p.T * (kH / kGroup); sg += nw) xq_segment(p, sg / (kH / kGroup), sg % (kH / kGroup), xs);
-  __syncthreads();                                 // the CTA's writes precede thread 0's release
-  if (threadIdx.x == 0) s_last = atom_add_acq_rel(p.cnt + kCntRoute, 1) == static_cast<int>(gridDim.x) - 1;
-  __syncthreads();                                 // thread 0's acquire precedes the CTA's reads
-  if (!s_last) return;
-  if (warp < p.T) topk_token(p, warp, s_ids);
-  __syncthreads();
-  if (warp == 0) build_tables(p, s_ids, scr_cnt, scr_mask);
-  if (threadIdx.x == 0) p.cnt[kCntRoute] = 0;
 }
 
 // ================================================================================ weight pipelines
 
-constexpr int kPW = 8;                      // warps per CTA, each with its own pipeline
 constexpr int kShGuTiles = kIs / 2;         // shared gate|up tiles: 2 hs columns each
-constexpr int kShDnTiles = kH / 4;          // shared down tiles: 4 ys rows each
+constexpr int kShDnTiles = kH / 8;          // shared down tiles: 8 ys rows each, in 4 stages
 constexpr int kGuTilesPerExpert = kI / 8;   // 64 routed gate|up tiles: 8 h columns each
 constexpr int kDnTilesPerExpert = kH / 32;  // 64 routed down tiles: 32 o rows each
 
 
-constexpr int kDnStage = 4096 + 512;        // codes (16 rows x 256 B, or 2 bf16 rows x 2 KB) + scales
-constexpr int kDnDepth = 4;                 // leaves ~80 KB of the SM's L1 for the activation rows
-struct DnWarp {                             // 18,560 bytes
-  alignas(128) uint8_t stage[kDnDepth][kDnStage];
-  uint64_t full[kDnDepth];
+constexpr int kDnStage = 4096 + 512;        // codes (16 rows x 256 B, or 8 bf16 rows x 512 B) + scales
+// int4 runs 16 warps with 2-stage rings (at most 128 registers), NVFP4 8 warps with 4 stages; about
+// 128 KB per SM in flight, and the rest of the SM's 256 KB holds L1 lines of the activation rows.
+template <int FMT>
+struct DnGeom {
+  static constexpr int kWarps = FMT == kInt4 ? 16 : 8;
+  static constexpr int kDepth = FMT == kInt4 ? 2 : 4;
+};
+template <int FMT>
+struct DnWarp {
+  alignas(128) uint8_t stage[DnGeom<FMT>::kDepth][kDnStage];
+  uint64_t full[DnGeom<FMT>::kDepth];
+};
+template <int FMT>
+struct DnShared {
+  DnWarp<FMT> w[DnGeom<FMT>::kWarps];
+  RouteSmem rs;
+  alignas(128) uint8_t hq[kMaxActive][2 * kI];        // down operand of every position: int4 limbs (hi, lo), NVFP4 fp16
+  float hsc[kMaxActive][kI / kGroup];                 // int4: unit / 16 of each segment of hq
+  uint64_t hqbar;                                     // completion of the operand copy
 };
 
 // Bounded wait for a stage (the barrier is the warp's own).
@@ -470,13 +536,13 @@ struct ExpertInfo {
 // an entry is then fetched by shuffles instead of a round trip to L2 per tile.
 struct WarpTable {
   int4 a[2], b[2];
-  __device__ __forceinline__ void load(const DecodeParams& p, int na) {
+  __device__ __forceinline__ void load(const RouteSmem& rs) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int gi = lane + 32 * h;
-      a[h] = gi < na ? __ldcg(p.etab + 2 * gi) : make_int4(0, 0, 0, 0);
-      b[h] = gi < na ? __ldcg(p.etab + 2 * gi + 1) : make_int4(0, 0, 0, 0);
+      a[h] = gi < rs.na ? rs.etab[gi][0] : make_int4(0, 0, 0, 0);
+      b[h] = gi < rs.na ? rs.etab[gi][1] : make_int4(0, 0, 0, 0);
     }
   }
   // entry of active slot gi (warp-uniform)
@@ -499,8 +565,8 @@ __device__ __forceinline__ int token_of(const DecodeParams& p, const ExpertInfo&
   return min(static_cast<int>((ex.toks >> (4 * col)) & 0xFu), p.T - 1);
 }
 
-__device__ __forceinline__ int active_count(const DecodeParams& p) {
-  return min(max(__ldcg(p.n_active), 0), min(kMaxActive, p.T * p.K));
+__device__ __forceinline__ int active_count(const DecodeParams& p, const RouteSmem& rs) {
+  return min(max(rs.na, 0), min(kMaxActive, p.T * p.K));
 }
 
 // ============================================================================================ gate|up
@@ -510,12 +576,12 @@ __device__ __forceinline__ int active_count(const DecodeParams& p) {
 // shared expert) and of the routed operand (int4: limbs, NVFP4: fp16), rows padded by 64 bytes so
 // that the 8-lane phases of the fragment loads of different tokens hit different banks.
 // Warps per CTA and stages per warp ring: int4 (at most 128 registers) runs 16 warps with 2 stages,
-// NVFP4 (more registers per thread) 8 warps with 4; either way about 128 KB per SM in flight. A ring
-// holds at most one tile's 4 stages, which keeps the scale double buffer safe.
+// NVFP4 (more registers per thread) 8 warps with 3; about 128 / 96 KB per SM in flight. A ring holds
+// at most one tile's 4 stages, which keeps the scale double buffer safe.
 template <int FMT>
 struct GuGeom {
   static constexpr int kWarps = FMT == kInt4 ? 16 : 8;
-  static constexpr int kDepth = FMT == kInt4 ? 2 : 4;
+  static constexpr int kDepth = FMT == kInt4 ? 2 : 3;
 };
 constexpr int kGuStage = 4096;
 constexpr int kTokPitch = 2 * kH + 64;      // bytes per token row of x or of the routed operand
@@ -533,10 +599,16 @@ struct GuShared {
   alignas(128) uint8_t xs[kDecodeMaxT][kTokPitch];    // x, bf16
   alignas(128) uint8_t xq[kDecodeMaxT][kTokPitch];    // int4: hi limbs, lo limbs; NVFP4: fp16 x
   float xsc[kDecodeMaxT][kH / kGroup];                // int4: unit / 16 of each segment of xq
+  RouteSmem rs;
   uint64_t xbar;                                      // completion of the x copies
   uint64_t xqbar;                                     // completion of the operand copies
-  int xq_issued;                                      // a warp has requested the operand
+  uint64_t route_ready;                               // the routing warps have filled rs
 };
+
+// Warps kRouteWarp0.. of a gate|up CTA derive the routing (they hold no shared-expert tile: tile
+// b + ncta * w is one only for w < 512 / ncta <= 4); the others wait for it on an mbarrier only when
+// they reach a routed tile, so their shared-expert tiles never stall.
+constexpr int kRouteWarp0 = 4;
 
 // Warp-collective: stage s (K groups 4q..4q+3, q = s mod 4) of tile `tile`, as few large copies (the
 // copy engine's cost is per copy more than per byte). Shared tile st: one tensor box with Sg rows
@@ -634,31 +706,45 @@ __global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
   auto tile_of = [&](int k) { return static_cast<int>(blockIdx.x) + ncta * (warp + kWarps * k); };
   int na = -1;                                     // active experts; known after the grid dependency
   WarpTable tab;
+  // Once per warp, the first time a routed tile is needed (or at the end). The routing warps wait
+  // for the route kernel and derive the routing from its logits (CTA 0 also publishes the tables);
+  // the first of them requests the operand rows and signals route_ready.
   auto routing = [&]() {
     if (na < 0) {
-      pdl_wait();                                  // the route kernel has finished and is visible
-      pdl_trigger();                               // the down kernel may start its prologue
-      na = active_count(p);
-      tab.load(p, na);
-      // the first warp of the CTA here requests the operand rows the route kernel wrote
-      int mine = 0;
-      if (lane == 0) mine = atomicCAS(&sm.xq_issued, 0, 1) == 0;
-      mine = __shfl_sync(kFull, mine, 0);
-      if (mine) {
-        constexpr int kRow = 2 * kH;               // int4: hi + lo limbs; NVFP4: fp16
-        const uint8_t* src = FMT == kInt4 ? p.xq8 : reinterpret_cast<const uint8_t*>(p.xq);
-        if (lane == 0) mbar_arrive_expect_tx(&sm.xqbar, p.T * kRow + (FMT == kInt4 ? p.T * (kH / kGroup) * 4 : 0));
-        __syncwarp();
-        if (lane < p.T) bulk_g2s(sm.xq[lane], src + static_cast<size_t>(lane) * kRow, kRow, &sm.xqbar);
-        if (FMT == kInt4 && lane == 31) bulk_g2s(&sm.xsc[0][0], p.xsc, p.T * (kH / kGroup) * 4, &sm.xqbar);
+      if (warp >= kRouteWarp0) {
+        pdl_wait();                                // the route kernel has finished and is visible
+        route_group(p, sm.rs, blockIdx.x == 0, warp - kRouteWarp0, kWarps - kRouteWarp0, 1);
+        // the down kernel reads CTA 0's published tables: they are visible before any trigger
+        if (blockIdx.x == 0) __threadfence();
+        pdl_trigger();
+        if (warp == kRouteWarp0) {
+          constexpr int kRow = 2 * kH;             // int4: hi + lo limbs; NVFP4: fp16
+          const uint8_t* src = FMT == kInt4 ? p.xq8 : reinterpret_cast<const uint8_t*>(p.xq);
+          if (lane == 0) mbar_arrive_expect_tx(&sm.xqbar, p.T * kRow + (FMT == kInt4 ? p.T * (kH / kGroup) * 4 : 0));
+          __syncwarp();
+          if (lane < p.T) bulk_g2s(sm.xq[lane], src + static_cast<size_t>(lane) * kRow, kRow, &sm.xqbar);
+          if (FMT == kInt4 && lane == 31) bulk_g2s(&sm.xsc[0][0], p.xsc, p.T * (kH / kGroup) * 4, &sm.xqbar);
+          if (lane == 0) mbar_arrive(&sm.route_ready);
+        }
+      } else {
+        pdl_wait();
+        wait_stage(p, &sm.route_ready, 0);
+        pdl_trigger();
       }
+      na = active_count(p, sm.rs);
+      tab.load(sm.rs);
     }
   };
-  auto valid = [&](int k) {
+  auto valid = [&](int k) {                        // blocks until the routing is known if needed
     const int tl = tile_of(k);
     if (tl < kShGuTiles) return true;
     routing();
     return tl < kShGuTiles + kGuTilesPerExpert * na;
+  };
+  auto can_issue = [&](int k) {                    // as valid, but a shared-tile warp does not wait
+    if (na < 0 && warp < kRouteWarp0 && tile_of(k) >= kShGuTiles && !mbar_test_wait(&sm.route_ready, 0))
+      return false;
+    return valid(k);
   };
   auto info = [&](int tl) {
     ExpertInfo ex{};
@@ -666,6 +752,10 @@ __global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
     return ex;
   };
 
+  // The shared expert's down weights need no routing either: into L2 now, in 32 KB chunks over the
+  // CTAs, for the down kernel.
+  if (threadIdx.x == 0)
+    for (int c = blockIdx.x; c < kH * kIs * 2 / 32768; c += gridDim.x) prefetch_l2(p.sh_dn + c * 32768, 32768);
   // Shared-expert stages need no routing: request them first, then stage x and build the routed
   // operand while the route kernel runs.
   int s_issue = 0;
@@ -675,7 +765,7 @@ __global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
     if (lane == 0) {
       mbar_init(&sm.xbar, 1);
       mbar_init(&sm.xqbar, 1);
-      sm.xq_issued = 0;
+      mbar_init(&sm.route_ready, 1);
       fence_mbar_init();
       mbar_arrive_expect_tx(&sm.xbar, p.T * kH * 2);
     }
@@ -686,6 +776,14 @@ __global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
   wait_stage(p, &sm.xbar, 0);
   bool have_xq = false;
 
+  // the previous routed tile's segment arrival; the last arriver of a segment rotates it
+  PendingArrival seg_arr;
+  auto finish_last = [&](int key) {
+    if (key < 0) return;
+    const int gi = (key - kCntSeg) / 4, seg = (key - kCntSeg) % 4;
+    finish_segment(p, tab.get(p, gi), seg);
+    if (lane == 0) p.cnt[key] = 0;
+  };
   float acc[2][4];
   ExpertInfo ex{};
   bool bvalid = false;
@@ -694,7 +792,7 @@ __global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
   for (int s = 0;; ++s) {
     const int k = s >> 2, q = s & 3, tl = tile_of(k);
     if (q == 0 && !valid(k)) break;
-    for (; s_issue < s + kDepth && valid(s_issue >> 2); ++s_issue)      // keep the ring full
+    for (; s_issue < s + kDepth && can_issue(s_issue >> 2); ++s_issue)  // keep the ring full
       gu_issue(p, ws, s_issue, tile_of(s_issue >> 2), info(tile_of(s_issue >> 2)));
     if (q == 0) {
 #pragma unroll
@@ -784,30 +882,30 @@ __global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
           p.h32[static_cast<size_t>(ex.off + col) * kI + 8 * i8 + g] = silu(c[qq] * ex.tsg) * (c[2 + qq] * ex.tsu);
       }
       const int seg = i8 / (kGroup / 8);
-      if (warp_arrive_last(p.cnt + kCntSeg + 4 * gi + seg, kGroup / 8)) {
-        finish_segment(p, ex, seg);
-        if (lane == 0) p.cnt[kCntSeg + 4 * gi + seg] = 0;
-      }
+      finish_last(seg_arr.settle());
+      seg_arr.arrive(p.cnt, kCntSeg + 4 * gi + seg, kGroup / 8);
     }
   }
   routing();                                       // every warp passes the grid dependency before it ends
+  finish_last(seg_arr.settle());
   if (!have_xq) wait_stage(p, &sm.xqbar, 0);       // no bulk copy may still write this CTA's memory
 }
 
 // ============================================================================================ down
 
-// Warp-collective: stage q = s mod 2 of tile `tile`, one contiguous copy of its rows. Shared tile sd:
-// Sd rows 4sd + 2q, +1 (2 KB each, all of K). Routed tile (gi, b): 16 rows 32b + 16q .. +16 of the
-// expert's down rows, all of K (256 B each), and their scales.
-__device__ void dn_issue(const DecodeParams& p, DnWarp& ws, int s, int tile, const ExpertInfo& ex) {
+// Warp-collective: stage q of tile `tile` (slot s mod depth). Shared tile sd: one tensor box with
+// Sd rows 8sd .. +8, K quarter q (512 B each). Routed tile (gi, b): 16 rows 32b + 16q .. +16 of the
+// expert's down rows, all of K (256 B each, contiguous), and their scales.
+template <int FMT>
+__device__ void dn_issue(const DecodeParams& p, DnWarp<FMT>& ws, int s, int q, int tile, const ExpertInfo& ex) {
   const int lane = threadIdx.x & 31;
-  const int slot = s % kDnDepth, q = s & 1;
+  const int slot = s % DnGeom<FMT>::kDepth;
   uint8_t* st = ws.stage[slot];
   uint64_t* bar = &ws.full[slot];
   if (tile < kShDnTiles) {
     if (lane == 0) {
       mbar_arrive_expect_tx(bar, 4096);
-      bulk_g2s(st, p.sh_dn + static_cast<size_t>(4 * tile + 2 * q) * (kIs * 2), 4096, bar);
+      tma_load_2d(st, &p.tm_sh_dn, q * 128, 8 * tile, bar);
     }
     return;
   }
@@ -830,27 +928,19 @@ __device__ __forceinline__ void prefetch_range(const void* base, size_t bytes) {
   for (size_t o = static_cast<size_t>(threadIdx.x & 31) * 128; o < bytes; o += 32 * 128) prefetch_l1(b + o);
 }
 
-// Warp: L1 prefetch of the activation rows down tile `tile` reads (gate|up outputs; call after the
-// grid dependency): hs of every token for a shared tile, the expert's rows of the down operand for
-// a routed one (its positions are consecutive).
-__device__ void dn_prefetch(const DecodeParams& p, int tile, const ExpertInfo& ex) {
+// Warp: L1 prefetch of the activation rows a shared down tile reads (hs of every token; call after
+// the grid dependency). Routed tiles read their operand from shared memory.
+__device__ void dn_prefetch(const DecodeParams& p, int tile, const ExpertInfo&) {
   if (tile < kShDnTiles) {
     prefetch_range(p.hs_hi, static_cast<size_t>(p.T) * kIs * 2);
     prefetch_range(p.hs_lo, static_cast<size_t>(p.T) * kIs * 2);
-    return;
-  }
-  if (p.fmt == kInt4) {
-    prefetch_range(p.hq8 + static_cast<size_t>(ex.off) * (2 * kI), static_cast<size_t>(ex.n) * (2 * kI));
-    prefetch_range(p.hsc + static_cast<size_t>(ex.off) * (kI / kGroup), static_cast<size_t>(ex.n) * (kI / kGroup) * 4);
-  } else {
-    prefetch_range(p.hq + static_cast<size_t>(ex.off) * kI, static_cast<size_t>(ex.n) * kI * 2);
   }
 }
 
 // y rows nb*64 .. +64 of every token (one warp), slots in slot order. The (position, weight) of
 // every pair is fetched once (lane q holds pairs q and q + 32); lane l then owns rows 4(l mod 16)
-// .. +4 of token t0 + l/16 and of token t0 + 2 + l/16, whose o rows it loads together.
-__device__ void combine_block(const DecodeParams& p, int nb) {
+// .. +4 of token t0 + l/16, two tokens per round.
+__device__ void combine_block(const DecodeParams& p, const RouteSmem& rs, int nb) {
   const int lane = threadIdx.x & 31;
   const int n = nb * 64 + 4 * (lane & 15), K = p.K, P = p.T * K;
   int pos[2];
@@ -858,86 +948,120 @@ __device__ void combine_block(const DecodeParams& p, int nb) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int q = lane + 32 * h;
-    pos[h] = q < P ? min(max(__ldcg(p.inv + q), 0), P - 1) : 0;
-    wt[h] = q < P ? __ldcg(p.wts + q) : 0.f;
+    pos[h] = q < P ? min(max(rs.inv[q], 0), P - 1) : 0;
+    wt[h] = q < P ? rs.w[q] : 0.f;
   }
-  for (int t0 = 0; t0 < p.T; t0 += 4) {
-    float4 ov[2][kMaxTopK], yv[2];
-    float w[2][kMaxTopK];
+#pragma unroll 1
+  for (int t0 = 0; t0 < p.T; t0 += 2) {
+    const int tok = t0 + (lane >> 4);
+    const bool tv = tok < p.T;
+    const float4 yv = tv ? __ldcg(reinterpret_cast<const float4*>(p.ys + tok * kH + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 ov[kMaxTopK];
+    float w[kMaxTopK];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int tok = t0 + 2 * u + (lane >> 4);
-      const bool tv = tok < p.T;
-      yv[u] = tv ? __ldcg(reinterpret_cast<const float4*>(p.ys + tok * kH + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int k = 0; k < kMaxTopK; ++k) {
-        if (k < K) {
-          const int q = min(tok, p.T - 1) * K + k;       // per lane: read both halves of the table
-          const int p0 = __shfl_sync(kFull, pos[0], q & 31), p1 = __shfl_sync(kFull, pos[1], q & 31);
-          const float w0 = __shfl_sync(kFull, wt[0], q & 31), w1 = __shfl_sync(kFull, wt[1], q & 31);
-          w[u][k] = q < 32 ? w0 : w1;
-          ov[u][k] = tv ? __ldcg(reinterpret_cast<const float4*>(p.o + static_cast<size_t>(q < 32 ? p0 : p1) * kH + n))
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+    for (int k = 0; k < kMaxTopK; ++k) {
+      if (k < K) {
+        const int q = min(tok, p.T - 1) * K + k;         // per lane: read both halves of the table
+        const int p0 = __shfl_sync(kFull, pos[0], q & 31), p1 = __shfl_sync(kFull, pos[1], q & 31);
+        const float w0 = __shfl_sync(kFull, wt[0], q & 31), w1 = __shfl_sync(kFull, wt[1], q & 31);
+        w[k] = q < 32 ? w0 : w1;
+        ov[k] = tv ? __ldcg(reinterpret_cast<const float4*>(p.o + static_cast<size_t>(q < 32 ? p0 : p1) * kH + n))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
+    if (tv) {
+      float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int tok = t0 + 2 * u + (lane >> 4);
-      if (tok < p.T) {
-        float a[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int k = 0; k < kMaxTopK; ++k)
-          if (k < K) {
-            a[0] = fmaf(w[u][k], ov[u][k].x, a[0]);
-            a[1] = fmaf(w[u][k], ov[u][k].y, a[1]);
-            a[2] = fmaf(w[u][k], ov[u][k].z, a[2]);
-            a[3] = fmaf(w[u][k], ov[u][k].w, a[3]);
-          }
-        uint2 out;
-        out.x = pack_bf162(fmaf(p.routed_scale, a[0], yv[u].x), fmaf(p.routed_scale, a[1], yv[u].y));
-        out.y = pack_bf162(fmaf(p.routed_scale, a[2], yv[u].z), fmaf(p.routed_scale, a[3], yv[u].w));
-        *reinterpret_cast<uint2*>(p.y + tok * kH + n) = out;
-      }
+      for (int k = 0; k < kMaxTopK; ++k)
+        if (k < K) {
+          a[0] = fmaf(w[k], ov[k].x, a[0]);
+          a[1] = fmaf(w[k], ov[k].y, a[1]);
+          a[2] = fmaf(w[k], ov[k].z, a[2]);
+          a[3] = fmaf(w[k], ov[k].w, a[3]);
+        }
+      uint2 out;
+      out.x = pack_bf162(fmaf(p.routed_scale, a[0], yv.x), fmaf(p.routed_scale, a[1], yv.y));
+      out.y = pack_bf162(fmaf(p.routed_scale, a[2], yv.z), fmaf(p.routed_scale, a[3], yv.w));
+      *reinterpret_cast<uint2*>(p.y + tok * kH + n) = out;
     }
   }
 }
 
 template <int FMT>
-__global__ void __launch_bounds__(kPW * 32, 1) decode_down_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(DnGeom<FMT>::kWarps * 32, 1)
+    decode_down_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int kWarps = DnGeom<FMT>::kWarps, kDepth = DnGeom<FMT>::kDepth;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  DnWarp& ws = reinterpret_cast<DnWarp*>(smem_raw)[warp];
+  DnShared<FMT>& sm = *reinterpret_cast<DnShared<FMT>*>(smem_raw);
+  DnWarp<FMT>& ws = sm.w[warp];
   if (lane == 0) {
 #pragma unroll
-    for (int i = 0; i < kDnDepth; ++i) mbar_init(&ws.full[i], 1);
+    for (int i = 0; i < kDepth; ++i) mbar_init(&ws.full[i], 1);
+    if (warp == 0) mbar_init(&sm.hqbar, 1);
     fence_mbar_init();
   }
   __syncwarp();
-  // This kernel starts only after every gate|up warp has passed its own grid dependency, so the
-  // routing tables are complete; the gate|up outputs are read only after pdl_wait below.
-  const int na = active_count(p);
+  // This kernel starts only after every gate|up warp has triggered, and gate|up CTA 0 triggers only
+  // after publishing the routing tables (fenced): they are read here while gate|up still runs. The
+  // gate|up outputs are read only after pdl_wait below.
+  if (warp == 0) {
+    const int nact = min(max(__ldcg(p.n_active), 0), min(kMaxActive, p.T * p.K));
+    for (int gi = lane; gi < nact; gi += 32) {
+      sm.rs.etab[gi][0] = __ldcg(p.etab + 2 * gi);
+      sm.rs.etab[gi][1] = __ldcg(p.etab + 2 * gi + 1);
+    }
+    for (int q = lane; q < p.T * p.K; q += 32) {
+      sm.rs.inv[q] = __ldcg(p.inv + q);
+      sm.rs.w[q] = __ldcg(p.wts + q);
+    }
+    if (lane == 0) sm.rs.na = nact;
+  }
+  __syncthreads();
+  const int na = active_count(p, sm.rs);
   WarpTable tab;
-  tab.load(p, na);
+  tab.load(sm.rs);
   const int n_tiles = kShDnTiles + kDnTilesPerExpert * na;
   const int ncta = gridDim.x;
-  auto tile_of = [&](int k) { return static_cast<int>(blockIdx.x) + ncta * (warp + kPW * k); };
+  auto tile_of = [&](int k) { return static_cast<int>(blockIdx.x) + ncta * (warp + kWarps * k); };
   auto info = [&](int tl) {
     ExpertInfo ex{};
     if (tl >= kShDnTiles) ex = tab.get(p, (tl - kShDnTiles) / kDnTilesPerExpert);
     return ex;
   };
+  // Stage s of this warp -> (tile ordinal k, stage q in the tile): a shared tile has 4 stages and can
+  // only be a warp's first tile (ncta * kWarps > kShDnTiles), routed tiles have 2.
+  const int first_len = tile_of(0) < kShDnTiles ? 4 : 2;
+  auto stage_k = [&](int s) { return s < first_len ? 0 : 1 + (s - first_len) / 2; };
+  auto stage_q = [&](int s) { return s < first_len ? s : (s - first_len) % 2; };
+  auto issue = [&](int s) {
+    const int tl = tile_of(stage_k(s));
+    dn_issue<FMT>(p, ws, s, stage_q(s), tl, info(tl));
+  };
   int s_issue = 0;
-  for (; s_issue < kDnDepth && tile_of(s_issue >> 1) < n_tiles; ++s_issue)
-    dn_issue(p, ws, s_issue, tile_of(s_issue >> 1), info(tile_of(s_issue >> 1)));
+  for (; s_issue < kDepth && tile_of(stage_k(s_issue)) < n_tiles; ++s_issue) issue(s_issue);
   pdl_wait();                                      // h and hs of the gate|up kernel
+  if (warp == 0 && lane == 0) {                    // the down operand of every position, one copy
+    const int P = p.T * p.K;
+    mbar_arrive_expect_tx(&sm.hqbar, P * 2 * kI + (FMT == kInt4 ? P * (kI / kGroup) * 4 : 0));
+    bulk_g2s(&sm.hq[0][0], FMT == kInt4 ? p.hq8 : reinterpret_cast<const uint8_t*>(p.hq), P * 2 * kI, &sm.hqbar);
+    if (FMT == kInt4) bulk_g2s(&sm.hsc[0][0], p.hsc, P * (kI / kGroup) * 4, &sm.hqbar);
+  }
+  bool have_hq = false;
   if (tile_of(0) < n_tiles) dn_prefetch(p, tile_of(0), info(tile_of(0)));
 
+  // the previous tile's block arrival; the last arriver of a 64-row block combines it
+  PendingArrival blk_arr;
+  auto combine_last = [&](int key) {
+    if (key < 0) return;
+    combine_block(p, sm.rs, key - kCntBlk);
+    if (lane == 0) p.cnt[key] = 0;
+  };
   float acc[2][2][4];                              // [16-row half][accumulator set][fragment]
   ExpertInfo ex{};
   const int target = 2 * na + kShDnTiles / (kH / 64);
   for (int s = 0;; ++s) {
-    const int k = s >> 1, q = s & 1, tl = tile_of(k);
+    const int k = stage_k(s), q = stage_q(s), tl = tile_of(k);
     if (tl >= n_tiles) break;
     if (q == 0) {
 #pragma unroll
@@ -947,73 +1071,80 @@ __global__ void __launch_bounds__(kPW * 32, 1) decode_down_kernel(const __grid_c
       if (tl >= kShDnTiles) ex = info(tl);
       if (tile_of(k + 1) < n_tiles) dn_prefetch(p, tile_of(k + 1), info(tile_of(k + 1)));
     }
-    const int slot = s % kDnDepth;
-    wait_stage(p, &ws.full[slot], (s / kDnDepth) & 1);
+    const int slot = s % kDepth;
+    wait_stage(p, &ws.full[slot], (s / kDepth) & 1);
     const uint8_t* st = ws.stage[slot];
     if (tl < kShDnTiles) {
-      // rows 4tl + 2q + g (g = 0, 1) of Sd, all of K; hs as a bf16 pair (hi + lo)
+      // rows 8tl + g (g < 8) of Sd, K quarter q (groups 2q, 2q+1); hs as a bf16 pair (hi + lo)
       const bool bv = g < p.T;
       const size_t r = static_cast<size_t>(bv ? g : 0) * kIs;
 #pragma unroll
-      for (int j = 0; j < kIs / kGroup; ++j) {
+      for (int jj = 0; jj < 2; ++jj) {
         RawA<kBf16> A;
-        load_a_bf16_rows(A, st, kIs * 2, 2, g, j, t);
+        load_a_bf16_rows(A, st, 512, 8, g, jj, t);
         RawB Bh, Bl;
-        Bh.load(p.hs_hi + r, j, t, bv);
-        Bl.load(p.hs_lo + r, j, t, bv);
-        bf16_group(acc[q], A, Bh, &Bl);
+        Bh.load(p.hs_hi + r, 2 * q + jj, t, bv);
+        Bl.load(p.hs_lo + r, 2 * q + jj, t, bv);
+        bf16_group(acc[0], A, Bh, &Bl);
       }
     } else {
       // 16 rows (half q of the 32-row tile), all of K = 4 groups
+      if (!have_hq) {
+        wait_stage(p, &sm.hqbar, 0);
+        have_hq = true;
+      }
       const bool bv = g < ex.n;
-      const size_t prow = static_cast<size_t>(ex.off + (bv ? g : 0));
+      const uint8_t* hrow = sm.hq[ex.off + (bv ? g : 0)];
       const uint8_t* sc = st + 4096;
       if constexpr (FMT == kInt4) {
         const uint16_t* s16 = reinterpret_cast<const uint16_t*>(sc);
         const bool v0 = 2 * t < ex.n, v1 = 2 * t + 1 < ex.n;
-        const float* x0p = p.hsc + static_cast<size_t>(ex.off + (v0 ? 2 * t : 0)) * (kI / kGroup);
-        const float* x1p = p.hsc + static_cast<size_t>(ex.off + (v1 ? 2 * t + 1 : 0)) * (kI / kGroup);
+        const float* x0p = sm.hsc[ex.off + (v0 ? 2 * t : 0)];
+        const float* x1p = sm.hsc[ex.off + (v1 ? 2 * t + 1 : 0)];
 #pragma unroll
         for (int j = 0; j < kI / kGroup; ++j) {
           const uint4 ra = *reinterpret_cast<const uint4*>(st + g * 256 + j * 64 + 16 * t);
           const uint4 rb = *reinterpret_cast<const uint4*>(st + (g + 8) * 256 + j * 64 + 16 * t);
           uint4 bh[2], bl[2];
-          load_limbs(bh, bl, p.hq8 + prow * (2 * kI), kI, j, t, bv);
+          if (bv) {
+            const uint8_t* ph = hrow + j * 128 + 32 * t;
+            bh[0] = *reinterpret_cast<const uint4*>(ph);
+            bh[1] = *reinterpret_cast<const uint4*>(ph + 16);
+            bl[0] = *reinterpret_cast<const uint4*>(ph + kI);
+            bl[1] = *reinterpret_cast<const uint4*>(ph + kI + 16);
+          } else {
+            bh[0] = bh[1] = bl[0] = bl[1] = make_uint4(0, 0, 0, 0);
+          }
           const float s0 = bf16_bits_to_f32(s16[g * 4 + j]), s1 = bf16_bits_to_f32(s16[(g + 8) * 4 + j]);
-          const float x0 = v0 ? __ldg(x0p + j) : 0.f, x1 = v1 ? __ldg(x1p + j) : 0.f;
+          const float x0 = v0 ? x0p[j] : 0.f, x1 = v1 ? x1p[j] : 0.f;
           const float f[4] = {s0 * x0, s0 * x1, s1 * x0, s1 * x1};
           int4_group(acc[q][0], ra, rb, bh, bl, f);
         }
       } else {
-        const __half* hrow = p.hq + prow * kI;
 #pragma unroll
         for (int j = 0; j < kI / kGroup; ++j) {
           const uint4 ra = *reinterpret_cast<const uint4*>(st + g * 256 + j * 64 + 16 * t);
           const uint4 rb = *reinterpret_cast<const uint4*>(st + (g + 8) * 256 + j * 64 + 16 * t);
           RawB B;
-          B.load(hrow, j, t, bv);
+          load_b_smem(B, hrow, j, t, bv);
           nvfp4_group(acc[q], ra, rb, B, sc + g * 32, sc + (g + 8) * 32, j, t);
         }
       }
     }
     __syncwarp();                                  // every lane's reads of the slot precede its refill
-    if (tile_of(s_issue >> 1) < n_tiles) {          // s_issue == s + kDnDepth: refill this slot
-      dn_issue(p, ws, s_issue, tile_of(s_issue >> 1), info(tile_of(s_issue >> 1)));
+    if (tile_of(stage_k(s_issue)) < n_tiles) {     // s_issue == s + kDepth: refill this slot
+      issue(s_issue);
       ++s_issue;
     }
-    if (q != 1) continue;
+    if (q != (tl < kShDnTiles ? 3 : 1)) continue;
     // ---- tile epilogue
     int nb;
     if (tl < kShDnTiles) {
-      const int n0 = 4 * tl;
-      if (g < 2) {
+      const int n0 = 8 * tl;
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {
-            const int tok = 2 * t + qq;
-            if (tok < p.T) p.ys[tok * kH + n0 + 2 * h + g] = acc[h][0][qq] + acc[h][1][qq];
-          }
+      for (int qq = 0; qq < 2; ++qq) {
+        const int tok = 2 * t + qq;
+        if (tok < p.T) p.ys[tok * kH + n0 + g] = acc[0][0][qq] + acc[0][1][qq];
       }
       nb = n0 / 64;
     } else {
@@ -1029,11 +1160,11 @@ __global__ void __launch_bounds__(kPW * 32, 1) decode_down_kernel(const __grid_c
         }
       nb = b / 2;
     }
-    if (warp_arrive_last(p.cnt + kCntBlk + nb, target)) {
-      combine_block(p, nb);
-      if (lane == 0) p.cnt[kCntBlk + nb] = 0;
-    }
+    combine_last(blk_arr.settle());
+    blk_arr.arrive(p.cnt, kCntBlk + nb, target);
   }
+  combine_last(blk_arr.settle());
+  if (!have_hq) wait_stage(p, &sm.hqbar, 0);       // no bulk copy may still write this CTA's memory
 }
 
 template <typename Kern>
@@ -1066,15 +1197,16 @@ cudaError_t allow_smem(Kern kernel, size_t bytes) {
 cudaError_t launch_decode(const DecodeParams& p, int n_sm, cudaStream_t s, cudaEvent_t ev_after_route,
                           cudaEvent_t ev_after_gate_up) {
   constexpr size_t kGuSmem4 = sizeof(GuShared<kInt4>), kGuSmemF = sizeof(GuShared<kNvfp4>);
-  constexpr size_t kDnSmem = sizeof(DnWarp) * kPW;
-  static_assert(kGuSmem4 <= 227 * 1024 && kGuSmemF <= 227 * 1024 && kDnSmem <= 227 * 1024, "shared memory per CTA");
+  constexpr size_t kDnSmem4 = sizeof(DnShared<kInt4>), kDnSmemF = sizeof(DnShared<kNvfp4>);
+  static_assert(kGuSmem4 <= 227 * 1024 && kGuSmemF <= 227 * 1024 && kDnSmem4 <= 227 * 1024 && kDnSmemF <= 227 * 1024,
+                "shared memory per CTA");
   static bool smem_set = false;                    // per process; the attribute is per function
   if (!smem_set) {
     cudaError_t e;
     if ((e = allow_smem(decode_gate_up_kernel<kInt4>, kGuSmem4)) != cudaSuccess) return e;
     if ((e = allow_smem(decode_gate_up_kernel<kNvfp4>, kGuSmemF)) != cudaSuccess) return e;
-    if ((e = allow_smem(decode_down_kernel<kInt4>, kDnSmem)) != cudaSuccess) return e;
-    if ((e = allow_smem(decode_down_kernel<kNvfp4>, kDnSmem)) != cudaSuccess) return e;
+    if ((e = allow_smem(decode_down_kernel<kInt4>, kDnSmem4)) != cudaSuccess) return e;
+    if ((e = allow_smem(decode_down_kernel<kNvfp4>, kDnSmemF)) != cudaSuccess) return e;
     if ((e = allow_smem(decode_route_kernel, 0)) != cudaSuccess) return e;
     smem_set = true;
   }
@@ -1086,8 +1218,8 @@ cudaError_t launch_decode(const DecodeParams& p, int n_sm, cudaStream_t s, cudaE
                      : launch_ex(decode_gate_up_kernel<kNvfp4>, n_sm, GuGeom<kNvfp4>::kWarps * 32, kGuSmemF, true, s, p);
   if (e != cudaSuccess) return e;
   if (ev_after_gate_up && (e = cudaEventRecord(ev_after_gate_up, s)) != cudaSuccess) return e;
-  return p.fmt == kInt4 ? launch_ex(decode_down_kernel<kInt4>, n_sm, kPW * 32, kDnSmem, true, s, p)
-                        : launch_ex(decode_down_kernel<kNvfp4>, n_sm, kPW * 32, kDnSmem, true, s, p);
+  return p.fmt == kInt4 ? launch_ex(decode_down_kernel<kInt4>, n_sm, DnGeom<kInt4>::kWarps * 32, kDnSmem4, true, s, p)
+                        : launch_ex(decode_down_kernel<kNvfp4>, n_sm, DnGeom<kNvfp4>::kWarps * 32, kDnSmemF, true, s, p);
 }
 
 }  // namespace flint

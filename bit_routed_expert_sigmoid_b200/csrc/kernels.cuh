@@ -48,6 +48,7 @@ enum : int {
 struct DecodeParams {
   CUtensorMap tm_gu;              // gate|up codes as 32-bit words [E*2I][H/8], box 64 words x 8 rows
   CUtensorMap tm_sh_gu;           // shared gate|up rows as 32-bit words [2Is][H/2], box 256 words x 2 rows
+  CUtensorMap tm_sh_dn;           // shared down rows as 32-bit words [H][Is/2], box 128 words x 8 rows
   int fmt, T, E, K;
   float floor_, routed_scale;
   const uint16_t* x;              // [T][H] bf16
