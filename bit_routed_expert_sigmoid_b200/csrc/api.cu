@@ -30,6 +30,7 @@ struct flint_moe_ctx {
   int* cnt;
   unsigned* err;
   __half* xq;
+  __half* xg;
   uint8_t* xq8;
   float* xsc;
   float* h32;
@@ -45,6 +46,11 @@ struct flint_moe_ctx {
   int last_T;
   int n_sm;
   CUtensorMap tm_gu, tm_sh_gu, tm_sh_dn;  // tensor maps of the decode kernels' weight copies
+  CUtensorMap tm_pf_gu, tm_pf_dn;          // prefill: routed codes, 16-word x 128-row boxes, 64-byte swizzle
+  CUtensorMap tm_pf_sh_gu, tm_pf_sh_dn;    // prefill: shared-expert weights, 64 x 128 bf16 boxes
+  CUtensorMap tm_pf_router;                // prefill: router rows [E][H], 64 x 128 bf16 boxes
+  CUtensorMap tm_pf_hs_hi, tm_pf_hs_lo;    // prefill: shared-expert hidden pair [t_max][Is]
+  CUtensorMap tm_pf_xg, tm_pf_hq;          // prefill: routed activation rows (fp16, 64 x 64 boxes)
   // instrumentation (caller-owned cudaEvent_t handles)
   cudaEvent_t events[32];
   int n_events;
@@ -97,6 +103,33 @@ bool encode_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_b
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over `rows` rows of `row_bytes` bytes with elements of `dtype` (`elem` bytes each); box of
+// box_inner elements x box_rows rows, with the given swizzle. Rows past `rows` read as zeros.
+bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, uint32_t elem, uint64_t rows,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {row_bytes / elem, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_bf16_tiles(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols * 2, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool encode_f16_rows64(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rows, cols * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool encode_code_tiles(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes) {
+  return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, rows, row_bytes, 16, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 // Lays the workspace out; with base == nullptr only the size is computed.
 size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
   const size_t T = c.t_max, E = c.n_experts, K = c.top_k, P = T * K;
@@ -119,6 +152,7 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
   char* p_cnt = take(kCntInts * 4);
   char* p_err = take(16);
   char* p_xq = take(T * kH * 2);
+  char* p_xg = take(P * kH * 2);
   char* p_xq8 = take(T * kH * 2);
   char* p_xsc = take(T * (kH / kGroup) * 4);
   char* p_h32 = take(P * kI * 4);
@@ -145,6 +179,7 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
     h->cnt = reinterpret_cast<int*>(p_cnt);
     h->err = reinterpret_cast<unsigned*>(p_err);
     h->xq = reinterpret_cast<__half*>(p_xq);
+    h->xg = reinterpret_cast<__half*>(p_xg);
     h->h32 = reinterpret_cast<float*>(p_h32);
     h->hq = reinterpret_cast<__half*>(p_hq);
     h->xq8 = reinterpret_cast<uint8_t*>(p_xq8);
@@ -252,49 +287,53 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
     FLINT_TRY(m.mark());
     return FLINT_OK;
   }
-  FLINT_TRY(launch_router_logits(x, static_cast<const uint16_t*>(h->w.router_w), T, E, h->logits, s));
+  PrefillParams pp{};
+  pp.T = T;
+  pp.top_k = K;
+  pp.E = E;
+  pp.logits = h->logits;
+  pp.active = h->active;
+  pp.n_active = h->n_active;
+  pp.offsets = h->offsets;
+  pp.perm = h->perm;
+  pp.hq = h->hq;
+  pp.o = h->o;
+  pp.hs_hi = h->hs_hi;
+  pp.hs_lo = h->hs_lo;
+  pp.ys = h->ys;
+  pp.err = h->err;
+  // B = x as given (map encoded per call: x changes, rows past T read as zeros)
+  if (!encode_bf16_tiles(&pp.tm_b, x, T, kH)) return FLINT_ERR_CUDA;
+  pp.tm_a = h->tm_pf_router;
+  FLINT_TRY(launch_prefill_shared(pp, kPhaseRouter, h->n_sm, s));
   FLINT_TRY(m.mark());
   FLINT_TRY(launch_topk(h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, s));
   FLINT_TRY(m.mark());
   FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, h->active, h->n_active, c.flags,
                            h->err, s));
   FLINT_TRY(m.mark());
-  FLINT_TRY(launch_xq(x, T, fmt == kInt4 ? 1 : 0, h->xq, s));
+  FLINT_TRY(launch_xg(x, T, K, h->inv, fmt == kInt4 ? 1 : 0, h->xg, s));
   FLINT_TRY(m.mark());
 
-  GemvShared sh{};
-  sh.w_gu = static_cast<const uint8_t*>(h->w.sh_gu);
-  sh.w_dn = static_cast<const uint8_t*>(h->w.sh_dn);
-  sh.x = x;
-  sh.T = T;
-  sh.hs_hi = h->hs_hi;
-  sh.hs_lo = h->hs_lo;
-  sh.ys = h->ys;
-  FLINT_TRY(launch_gu_shared(sh, s));
+  pp.tm_a = h->tm_pf_sh_gu;                        // shared gate|up: B = x
+  FLINT_TRY(launch_prefill_shared(pp, kPhaseGateUp, h->n_sm, s));
   FLINT_TRY(m.mark());
-
-  const int groups = (T * K < E) ? T * K : E;
-  GemvRouted r{};
-  r.active = h->active;
-  r.n_active = h->n_active;
-  r.offsets = h->offsets;
-  r.perm = h->perm;
-  r.top_k = K;
-  r.xq = h->xq;
-  r.h_out = h->h32;
-  r.h_in = h->h32;
-  r.o_out = h->o;
-  r.codes = static_cast<const uint8_t*>(h->w.gu_codes);
-  r.scales = h->w.gu_scales;
-  r.tscale = h->w.gu_tscale;
-  FLINT_TRY(launch_gu_routed(r, fmt, groups, s));
+  pp.tm_codes = h->tm_pf_gu;
+  pp.tm_act = h->tm_pf_xg;
+  pp.scales = h->w.gu_scales;
+  pp.tscale = h->w.gu_tscale;
+  FLINT_TRY(launch_prefill_routed(pp, fmt, kPhaseGateUp, h->n_sm, s));
   FLINT_TRY(m.mark());
-  r.codes = static_cast<const uint8_t*>(h->w.dn_codes);
-  r.scales = h->w.dn_scales;
-  r.tscale = h->w.dn_tscale;
-  FLINT_TRY(launch_dn_routed(r, fmt, groups, s));
+  pp.tm_codes = h->tm_pf_dn;
+  pp.tm_act = h->tm_pf_hq;
+  pp.scales = h->w.dn_scales;
+  pp.tscale = h->w.dn_tscale;
+  FLINT_TRY(launch_prefill_routed(pp, fmt, kPhaseDown, h->n_sm, s));
   FLINT_TRY(m.mark());
-  FLINT_TRY(launch_dn_shared(sh, s));
+  pp.tm_a = h->tm_pf_sh_dn;
+  pp.tm_b = h->tm_pf_hs_hi;
+  pp.tm_b2 = h->tm_pf_hs_lo;
+  FLINT_TRY(launch_prefill_shared(pp, kPhaseDown, h->n_sm, s));
   FLINT_TRY(m.mark());
   FLINT_TRY(launch_combine(h->o, h->ys, h->wts, h->inv, T, K, c.routed_scale, y, s));
   FLINT_TRY(m.mark());
@@ -342,7 +381,16 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
       cudaMemset(h->err, 0, 16) != cudaSuccess || cudaMemset(h->cnt, 0, kCntInts * 4) != cudaSuccess ||
       !encode_rows(&h->tm_gu, w.gu_codes, static_cast<uint64_t>(cfg->n_experts) * 2 * kI, kH / 2, 64, 8) ||
       !encode_rows(&h->tm_sh_gu, w.sh_gu, 2 * kIs, kH * 2, 256, 2) ||
-      !encode_rows(&h->tm_sh_dn, w.sh_dn, kH, kIs * 2, 128, 8)) {
+      !encode_rows(&h->tm_sh_dn, w.sh_dn, kH, kIs * 2, 128, 8) ||
+      !encode_code_tiles(&h->tm_pf_gu, w.gu_codes, static_cast<uint64_t>(cfg->n_experts) * 2 * kI, kH / 2) ||
+      !encode_code_tiles(&h->tm_pf_dn, w.dn_codes, static_cast<uint64_t>(cfg->n_experts) * kH, kI / 2) ||
+      !encode_bf16_tiles(&h->tm_pf_sh_gu, w.sh_gu, 2 * kIs, kH) ||
+      !encode_bf16_tiles(&h->tm_pf_sh_dn, w.sh_dn, kH, kIs) ||
+      !encode_bf16_tiles(&h->tm_pf_router, w.router_w, cfg->n_experts, kH) ||
+      !encode_bf16_tiles(&h->tm_pf_hs_hi, h->hs_hi, cfg->t_max, kIs) ||
+      !encode_bf16_tiles(&h->tm_pf_hs_lo, h->hs_lo, cfg->t_max, kIs) ||
+      !encode_f16_rows64(&h->tm_pf_xg, h->xg, static_cast<uint64_t>(cfg->t_max) * cfg->top_k, kH) ||
+      !encode_f16_rows64(&h->tm_pf_hq, h->hq, static_cast<uint64_t>(cfg->t_max) * cfg->top_k, kI)) {
     delete h;
     return FLINT_ERR_CUDA;
   }
@@ -394,7 +442,15 @@ flint_status flint_moe_intermediate(flint_moe_t h, int which, void* dst, size_t 
   size_t have = 0;
   switch (which) {
     case FLINT_BUF_LOGITS: src = h->logits; have = T * h->cfg.n_experts * 4; break;
-    case FLINT_BUF_XQ: src = h->xq; have = T * kH * 2; break;
+    case FLINT_BUF_XQ:
+      if (T <= kDecodeMaxT) {
+        src = h->xq;
+        have = T * kH * 2;
+      } else {
+        src = h->xg;
+        have = T * h->cfg.top_k * kH * 2;
+      }
+      break;
     case FLINT_BUF_YS: src = h->ys; have = T * kH * 4; break;
     default: return FLINT_ERR_INVALID_ARG;
   }

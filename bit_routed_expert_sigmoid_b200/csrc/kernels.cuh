@@ -92,12 +92,40 @@ struct DecodeParams {
 cudaError_t launch_decode(const DecodeParams& p, int n_sm, cudaStream_t s, cudaEvent_t ev_after_route,
                           cudaEvent_t ev_after_gate_up);
 
+// ---- prefill path (T > kDecodeMaxT): tcgen05 grouped GEMMs ----
+enum PfPhase : int { kPhaseGateUp = 0, kPhaseDown = 1, kPhaseRouter = 2 };
+
+struct PrefillParams {
+  CUtensorMap tm_codes;           // routed: codes as 32-bit words [rows][K/8], box 16 words x 128 rows, 64-byte swizzle
+  CUtensorMap tm_act;             // routed: fp16 activation rows (xg or hq), box 64 x 64 rows, 128-byte swizzle
+  CUtensorMap tm_a;               // dense phases: bf16 weights (shared expert, router), box 64 x 128 rows, 128-byte swizzle
+  CUtensorMap tm_b;               // shared: bf16 activations (x, or hs_hi), box 64 x 128 rows, 128-byte swizzle
+  CUtensorMap tm_b2;              // shared down: hs_lo
+  int T, top_k, E;
+  float* logits;                  // router phase output [T][E]
+  const int* active;              // ascending experts with tokens
+  const int* n_active;
+  const int* offsets;             // [E+1]
+  const int* perm;                // [P]
+  const void* scales;             // int4 bf16 / nvfp4 e4m3, layout of the codes
+  const float* tscale;            // gate|up [E][2] or down [E]; may be null
+  __half* hq;                     // routed gate|up output [P][I]
+  float* o;                       // routed down output [P][H]
+  uint16_t* hs_hi;                // shared gate|up output [T][Is], bf16 pair
+  uint16_t* hs_lo;
+  float* ys;                      // shared down output [T][H]
+  unsigned* err;
+};
+
+cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, int n_sm, cudaStream_t s);
+cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, cudaStream_t s);
+
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* wr, int T, int E, float* logits, cudaStream_t s);
 cudaError_t launch_topk(const float* logits, int T, int E, int K, float floor_, int* ids, float* wts, unsigned flags,
                         unsigned* err, cudaStream_t s);
 cudaError_t launch_permute(const int* ids, int T, int K, int E, int* counts, int* offsets, int* perm, int* inv,
                            int* active, int* n_active, unsigned flags, unsigned* err, cudaStream_t s);
-cudaError_t launch_xq(const uint16_t* x, int T, int rotate, __half* xq, cudaStream_t s);
+cudaError_t launch_xg(const uint16_t* x, int T, int K, const int* inv, int rotate, __half* xg, cudaStream_t s);
 
 cudaError_t launch_gu_routed(const GemvRouted& a, int fmt, int groups, cudaStream_t s);
 cudaError_t launch_dn_routed(const GemvRouted& a, int fmt, int groups, cudaStream_t s);

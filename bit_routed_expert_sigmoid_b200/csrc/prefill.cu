@@ -1,0 +1,816 @@
+// Expert projections for large token counts (prefill): grouped GEMMs on the fifth-generation tensor
+// cores (tcgen05.mma, fp32 accumulators in tensor memory).
+//
+// Routed experts (pf_routed_kernel). The permuted rows of one expert are its tokens; a tile is
+// (expert, a chunk of up to 128 of those rows, a pair of 128-row weight blocks): for gate|up the
+// gate rows [128r, 128r+128) and the matching up rows, for down the output rows [256r, 256r+128)
+// and [256r+128, 256r+256). One persistent CTA per SM walks the tiles; its warps specialise:
+//   warp 0       TMA copies of the 4-bit codes, 128 K per stage, into a shared-memory ring
+//   warp 3       TMA copies of the chunk's activation rows (fp16, stored per permuted row so that
+//                an expert's rows are contiguous; 128-byte swizzled K-major) into a second ring
+//   warps 4-11   dequantisation: a thread owns one weight row of one block, turns its 128 codes of
+//                the stage into exact fp16 (int4: code x bf16 group scale; NVFP4: E2M1 x E4M3) and
+//                writes them to tensor memory with tcgen05.st, where the MMA reads its A operand.
+//                A in tensor memory costs no shared-memory bandwidth, which a 128 x 48 MMA with A
+//                in shared memory would exhaust.
+//   warps 1, 2   one MMA-issuing thread per block (an MMA instruction takes ~45 cycles to issue, so
+//                two issuers keep N = 48 tiles near the tensor-core rate); D[128 x N] per block
+//   warps 12-15  epilogue: gate|up -> h = silu(g) u, int4: rotated per 128-segment by the Hadamard
+//                butterfly, stored fp16 in the order of the down operand; down -> o in fp32.
+// Every dependency is an mbarrier: TMA transaction counts, cp.async arrivals, tcgen05.commit
+// arrivals and thread arrivals; every wait is bounded and sets a timeout bit on expiry.
+//
+// The shared expert (pf_shared_kernel) is a dense bf16 GEMM of the same shape of pipeline with the
+// weights and activations brought by TMA in the 128-byte swizzled layout and read by the MMA from
+// shared memory.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace flint {
+
+namespace {
+
+#ifndef FLINT_WAIT_NS
+#define FLINT_WAIT_NS 1000000000ull          // 1 s
+#endif
+constexpr uint64_t kPfWaitNs = FLINT_WAIT_NS;
+constexpr unsigned kAll = 0xFFFFFFFFu;
+
+constexpr int kPfN = 64;                     // tokens per tile (MMA N, padded to a multiple of 16)
+constexpr int kPfSK = 128;                   // K per pipeline stage
+constexpr int kPfDA = 6;                     // code ring depth
+constexpr int kPfDB = 6;                     // activation ring depth
+constexpr int kPfCodeStage = 2 * 128 * kPfSK / 2;    // 16 KB: two blocks of 128 rows x 64 bytes
+constexpr int kPfActChunk = kPfN * 128;              // 64 K of every row, 128-byte swizzled
+constexpr int kPfActStage = 2 * kPfActChunk;         // 16 KB
+constexpr int kSlabPitch = 132;              // floats per token row of the epilogue's transpose slab
+constexpr int kPfThreads = 512;
+
+// tensor-memory columns: two accumulator slots of (D0 | D1) x 64 columns, then two A stages of two
+// blocks x 64 columns (128 fp16 of K)
+constexpr uint32_t kColD1 = 64;
+constexpr uint32_t kColSlot = 128;
+constexpr uint32_t kColA = 256;
+
+// ---------------------------------------------------------------------------------------------
+// tcgen05 / TMA primitives
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// D[tmem d] (+)= A[tmem a] * B[smem desc]^T
+__device__ __forceinline__ void tc_mma_ta(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a), "l"(bdesc), "r"(idesc), "r"(acc));
+}
+
+// D[tmem d] (+)= A[smem desc] * B[smem desc]^T
+__device__ __forceinline__ void tc_mma_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc));
+}
+
+// 32 consecutive columns of the warp's 32 lanes (lane i of the warp = its own row)
+__device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) | (static_cast<uint64_t>(2) << 61);
+}
+
+// Instruction descriptor of kind::f16 with fp32 D, K-major A and B, M = 128.
+__device__ __forceinline__ uint32_t idesc_m128(int n, bool bf16) {
+  return (1u << 4) | (bf16 ? (1u << 7) | (1u << 10) : 0u) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Bounded wait: false if the CTA has given up (another wait expired) or this one expires.
+__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) {
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kPfWaitNs) {
+      atomicOr(err, kErrTimeout);
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+// Every lane waits (each acquires the barrier's phase itself); the verdict is warp-uniform.
+__device__ __forceinline__ bool pf_wait_all(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned* err) {
+  const bool ok = pf_wait(bar, parity, abort, err);
+  return __all_sync(kAll, ok) != 0;
+}
+
+// ---------------------------------------------------------------------------------------------
+// tile table of the routed kernels
+
+struct TileTab {
+  int n, total;
+  int start[kMaxE + 1];   // first tile of active expert i
+  int e[kMaxE];
+  int off[kMaxE];         // first permuted row
+  int cnt[kMaxE];         // permuted rows
+  int nch[kMaxE];         // chunks of kPfN rows
+};
+
+struct PfTile {
+  int e, row0, n, rp;     // expert, first permuted row of the chunk, rows in it (1..kPfN), block pair
+};
+
+// Warp 0: tiles of active expert i are rp-major over its chunks; experts in ascending order.
+__device__ void build_tiles(TileTab& tt, const PrefillParams& p, int rp_count) {
+  const int lane = threadIdx.x & 31;
+  const int n = min(*p.n_active, kMaxE);
+  int base = 0;
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    const int i = i0 + lane;
+    int tiles = 0;
+    if (i < n) {
+      const int e = p.active[i];
+      const int off = p.offsets[e];
+      const int c = max(p.offsets[e + 1] - off, 0);
+      const int nch = (c + kPfN - 1) / kPfN;
+      tt.e[i] = e;
+      tt.off[i] = off;
+      tt.cnt[i] = c;
+      tt.nch[i] = nch;
+      tiles = rp_count * nch;
+    }
+    int v = tiles;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int u = __shfl_up_sync(kAll, v, d);
+      if (lane >= d) v += u;
+    }
+    if (i < n) tt.start[i] = base + v - tiles;
+    base += __shfl_sync(kAll, v, 31);
+  }
+  if (lane == 0) {
+    tt.n = n;
+    tt.total = base;
+    tt.start[n] = base;
+  }
+}
+
+__device__ __forceinline__ PfTile tile_at(const TileTab& tt, int t) {
+  int lo = 0, hi = tt.n - 1;                 // last i with start[i] <= t (t < total)
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tt.start[mid] <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  const int local = t - tt.start[lo], nch = tt.nch[lo];
+  const int rp = local / nch, ch = local - rp * nch;
+  PfTile r;
+  r.e = tt.e[lo];
+  r.row0 = tt.off[lo] + ch * kPfN;
+  r.n = min(kPfN, tt.cnt[lo] - ch * kPfN);
+  r.rp = rp;
+  return r;
+}
+
+template <int PHASE>
+struct PfGeom;
+template <>
+struct PfGeom<kPhaseGateUp> {
+  static constexpr int K = kH, S = kH / kPfSK, RP = kI / 128;
+  // first weight row of block b of a tile
+  __device__ static int row(int e, int rp, int b) { return e * 2 * kI + b * kI + rp * 128; }
+};
+template <>
+struct PfGeom<kPhaseDown> {
+  static constexpr int K = kI, S = kI / kPfSK, RP = kH / 256;
+  __device__ static int row(int e, int rp, int b) { return e * kH + rp * 256 + b * 128; }
+};
+
+// shared-memory layout of the routed kernel (offsets from a 1024-byte aligned base)
+constexpr int kOffAct = 0;
+constexpr int kOffCode = kOffAct + kPfDB * kPfActStage;
+constexpr int kOffSlab = kOffCode + kPfDA * kPfCodeStage;
+constexpr int kOffTab = kOffSlab + 32 * kSlabPitch * 4;
+constexpr int kOffBar = (kOffTab + static_cast<int>(sizeof(TileTab)) + 7) / 8 * 8;
+
+struct PfBars {
+  uint64_t code_full[kPfDA], code_empty[kPfDA];
+  uint64_t act_full[kPfDB], act_empty[kPfDB];
+  uint64_t a_full[2][2], a_empty[2][2];       // [A stage in tensor memory][block]
+  uint64_t acc_full[2][2], acc_empty[2];       // [accumulator slot][block]
+  uint64_t done[2];
+  uint32_t tmem;
+  int abort;
+};
+constexpr int kPfSmem = kOffBar + static_cast<int>(sizeof(PfBars)) + 1024;   // + alignment slack
+static_assert(kPfSmem <= 227 * 1024, "shared memory per CTA");
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+}
+
+// silu with the fast exponential and division (relative error a few ulp of fp32)
+__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
+// int4 scale (bf16) -> fp16 pair; flags scales whose products with the codes fp16 cannot hold exactly
+__device__ __forceinline__ uint32_t scale_half2(uint32_t bf16_bits, bool& bad) {
+  const float s = bf16_bits_to_f32(static_cast<uint16_t>(bf16_bits));
+  const float a = fabsf(s);
+  bad |= (a > 8188.f) || (a != 0.f && a < 6.103515625e-05f);
+  return pack_half2(s, s);
+}
+
+// Turns the 128 codes of one row of one stage into 64 fp16 pairs in tensor memory.
+// int4: word w of the row gives columns 4w..4w+3 = pairs (n0,n4),(n1,n5),(n2,n6),(n3,n7) of its
+// eight codes (the order the activation operand is stored in). NVFP4: natural order.
+template <int FMT>
+__device__ __forceinline__ void dequant_stage(uint32_t taddr, const uint4 (&w)[4], uint32_t s_int4, uint2 s_fp4) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t v[32];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint4 wv = w[2 * half + q];
+      const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int col = 16 * q + 4 * k;            // column within this half
+        if constexpr (FMT == kInt4) {
+          uint32_t pr[4];
+          int4x8_to_half2x4(words[k], pr);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) v[col + j] = hmul2_u32(pr[j], s_int4);
+        } else {
+          // word index within the stage = 8 half + 4 q + k; 16-code block = that / 2
+          const int blk = (8 * half + 4 * q + k) >> 1;
+          const uint32_t sb = (blk < 4 ? (s_fp4.x >> (8 * blk)) : (s_fp4.y >> (8 * (blk - 4)))) & 0xFFu;
+          const uint32_t h = e4m3_to_half_bits(sb);
+          const uint32_t s2 = h | (h << 16);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) v[col + j] = hmul2_u32(e2m1x2_to_half2(words[k] >> (8 * j)), s2);
+        }
+      }
+    }
+    tc_st32(taddr + 32 * half, v);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// routed grouped GEMM
+
+template <int FMT, int PHASE>
+__global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_constant__ PrefillParams p) {
+  using G = PfGeom<PHASE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  TileTab& tt = *reinterpret_cast<TileTab*>(sm + kOffTab);
+  PfBars& bb = *reinterpret_cast<PfBars*>(sm + kOffBar);
+  float* slab = reinterpret_cast<float*>(sm + kOffSlab);
+  volatile int* abort = &bb.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kPfDA; ++i) {
+      mbar_init(&bb.code_full[i], 1);
+      mbar_init(&bb.code_empty[i], 8);
+    }
+    for (int i = 0; i < kPfDB; ++i) {
+      mbar_init(&bb.act_full[i], 1);
+      mbar_init(&bb.act_empty[i], 2);
+    }
+    for (int t = 0; t < 2; ++t)
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&bb.a_full[t][b], 4);
+        mbar_init(&bb.a_empty[t][b], 1);
+      }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bb.acc_full[a][0], 1);
+      mbar_init(&bb.acc_full[a][1], 1);
+      mbar_init(&bb.acc_empty[a], 4);
+    }
+    mbar_init(&bb.done[0], 1);
+    mbar_init(&bb.done[1], 1);
+    bb.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) build_tiles(tt, p, G::RP);
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&bb.tmem)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bb.tmem;
+  const int total = tt.total;
+
+  if (warp == 0) {
+    // ---- codes: two TMA boxes (128 rows x 64 bytes) per stage
+    int it = 0;
+    if (lane == 0) {
+      for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+        const PfTile tl = tile_at(tt, t);
+        const int r0 = G::row(tl.e, tl.rp, 0), r1 = G::row(tl.e, tl.rp, 1);
+        for (int s = 0; s < G::S; ++s, ++it) {
+          const int slot = it % kPfDA;
+          if (it >= kPfDA && !pf_wait(&bb.code_empty[slot], ((it / kPfDA) - 1) & 1, abort, p.err)) break;
+          uint8_t* st = sm + kOffCode + slot * kPfCodeStage;
+          mbar_arrive_expect_tx(&bb.code_full[slot], kPfCodeStage);
+          tma_2d(st, &p.tm_codes, s * (kPfSK / 8), r0, &bb.code_full[slot]);
+          tma_2d(st + kPfCodeStage / 2, &p.tm_codes, s * (kPfSK / 8), r1, &bb.code_full[slot]);
+        }
+      }
+      // no copy may still be in flight when the CTA exits
+      for (int j = max(it - kPfDA, 0); j < it; ++j) pf_wait(&bb.code_full[j % kPfDA], (j / kPfDA) & 1, abort, p.err);
+    }
+  } else if (warp == 3) {
+    // ---- activations: the chunk's rows are contiguous (permuted order), two TMA boxes of 64 rows x
+    // 64 fp16 (128-byte swizzled) per stage; rows past the chunk only feed unused accumulator columns
+    if (lane == 0) {
+      int it = 0;
+      for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+        const PfTile tl = tile_at(tt, t);
+        bool ok = true;
+        for (int s = 0; s < G::S; ++s, ++it) {
+          const int slot = it % kPfDB;
+          if (it >= kPfDB && !pf_wait(&bb.act_empty[slot], ((it / kPfDB) - 1) & 1, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = sm + kOffAct + slot * kPfActStage;
+          mbar_arrive_expect_tx(&bb.act_full[slot], kPfActStage);
+          tma_2d(st, &p.tm_act, s * kPfSK, tl.row0, &bb.act_full[slot]);
+          tma_2d(st + kPfActChunk, &p.tm_act, s * kPfSK + 64, tl.row0, &bb.act_full[slot]);
+        }
+        if (!ok) break;
+      }
+      for (int j = max(it - kPfDB, 0); j < it; ++j) pf_wait(&bb.act_full[j % kPfDB], (j / kPfDB) & 1, abort, p.err);
+    }
+  } else if (warp == 1 || warp == 2) {
+    // ---- MMA issue, one thread per block
+    const int b = warp - 1;
+    if (lane == 0) {
+      int it = 0, ti = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++ti) {
+        const PfTile tl = tile_at(tt, t);
+        const int npad = (tl.n + 15) & ~15;
+        const uint32_t idesc = idesc_m128(npad, false);
+        const int as = ti & 1;
+        const uint32_t d = tmem + as * kColSlot + b * kColD1;
+        if (ti >= 2 && !pf_wait(&bb.acc_empty[as], ((ti >> 1) - 1) & 1, abort, p.err)) break;
+        tc_fence_after();
+        for (int s = 0; s < G::S; ++s, ++it) {
+          const int ts = it & 1, bs = it % kPfDB;
+          if (!pf_wait(&bb.a_full[ts][b], (it >> 1) & 1, abort, p.err) ||
+              !pf_wait(&bb.act_full[bs], (it / kPfDB) & 1, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = tmem + kColA + ts * 128 + b * 64;
+          const uint32_t b0 = smem_u32(sm + kOffAct + bs * kPfActStage);
+#pragma unroll
+          for (int ks = 0; ks < kPfSK / 16; ++ks)
+            tc_mma_ta(d, a0 + ks * 8, sdesc_sw128(b0 + (ks >> 2) * kPfActChunk + (ks & 3) * 32), idesc,
+                      (s | ks) ? 1u : 0u);
+          tc_commit(&bb.a_empty[ts][b]);
+          tc_commit(&bb.act_empty[bs]);
+        }
+        if (ok) tc_commit(&bb.acc_full[as][b]);
+      }
+      tc_commit(&bb.done[b]);                       // every MMA of this thread has completed
+      pf_wait(&bb.done[b], 0, abort, p.err);
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ---- dequantisation into tensor memory
+    const int b = (warp - 4) >> 2, q = warp & 3;
+    const int r = 32 * q + lane;
+    const int swz = (lane >> 1) & 3;               // 64-byte swizzle of the code rows (row r at r*64)
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    // Scales are fetched ahead: int4 all of the row's group scales one tile ahead; NVFP4 the 16 E4M3
+    // block scales of a stage pair one pair ahead.
+    constexpr int kSc4 = FMT == kInt4 ? G::S / 2 : 1;
+    uint32_t sc_next[kSc4];
+    uint4 fp_next = make_uint4(0, 0, 0, 0);
+    auto load_int4 = [&](int row) {
+      const uint32_t* s32 = reinterpret_cast<const uint32_t*>(p.scales) + static_cast<size_t>(row) * (G::S / 2);
+#pragma unroll
+      for (int k = 0; k < kSc4; ++k) sc_next[k] = __ldg(s32 + k);
+    };
+    auto load_fp4 = [&](int row, int pair) {
+      fp_next = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.scales) +
+                                                     static_cast<size_t>(row) * (G::K / 16) + pair * 16));
+    };
+    int t = blockIdx.x;
+    int row = 0;
+    if (t < total) {
+      const PfTile tl = tile_at(tt, t);
+      row = G::row(tl.e, tl.rp, b) + r;
+      if constexpr (FMT == kInt4) load_int4(row);
+      else load_fp4(row, 0);
+    }
+    int it = 0;
+    bool bad = false;
+    while (t < total && !*abort) {
+      const int t_next = t + gridDim.x;
+      int row_next = -1;
+      if (t_next < total) {
+        const PfTile tn = tile_at(tt, t_next);
+        row_next = G::row(tn.e, tn.rp, b) + r;
+      }
+      uint32_t sc[kSc4];                         // consumed from sc[0], shifted down every 2 stages
+#pragma unroll
+      for (int k = 0; k < kSc4; ++k) sc[k] = sc_next[k];
+      if constexpr (FMT == kInt4) {
+        if (row_next >= 0) load_int4(row_next);
+      }
+      uint4 fp_cur = make_uint4(0, 0, 0, 0);
+      bool ok = true;
+      for (int s = 0; s < G::S; ++s, ++it) {
+        const int slot = it % kPfDA, ts = it & 1;
+        uint2 s_fp4 = make_uint2(0, 0);
+        if constexpr (FMT == kNvfp4) {
+          if ((s & 1) == 0) {
+            fp_cur = fp_next;
+            if (s + 2 < G::S) load_fp4(row, (s + 2) >> 1);
+            else if (row_next >= 0) load_fp4(row_next, 0);
+          }
+          s_fp4 = (s & 1) ? make_uint2(fp_cur.z, fp_cur.w) : make_uint2(fp_cur.x, fp_cur.y);
+        }
+        if (!pf_wait_all(&bb.code_full[slot], (it / kPfDA) & 1, abort, p.err)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* src = sm + kOffCode + slot * kPfCodeStage + b * (kPfCodeStage / 2) + r * (kPfSK / 2);
+        uint4 w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w[k] = *reinterpret_cast<const uint4*>(src + ((k ^ swz) << 4));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bb.code_empty[slot]);
+        uint32_t s_int4 = 0;
+        if constexpr (FMT == kInt4) {
+          s_int4 = scale_half2((sc[0] >> (16 * (s & 1))) & 0xFFFFu, bad);
+          if (s & 1) {
+#pragma unroll
+            for (int k = 0; k + 1 < kSc4; ++k) sc[k] = sc[k + 1];
+          }
+        }
+        if (it >= 2 && !pf_wait_all(&bb.a_empty[ts][b], ((it >> 1) - 1) & 1, abort, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        dequant_stage<FMT>(lane_base + kColA + ts * 128 + b * 64, w, s_int4, s_fp4);
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bb.a_full[ts][b]);
+      }
+      if (!ok) break;
+      t = t_next;
+      row = row_next;
+    }
+    if (bad) atomicOr(p.err, kErrRange);
+  } else if (warp >= 12) {
+    // ---- epilogue
+    const int q = warp & 3, r = 32 * q + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    int ti = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++ti) {
+      const PfTile tl = tile_at(tt, t);
+      const int as = ti & 1;
+      if (!pf_wait_all(&bb.acc_full[as][0], (ti >> 1) & 1, abort, p.err) ||
+          !pf_wait_all(&bb.acc_full[as][1], (ti >> 1) & 1, abort, p.err))
+        break;
+      tc_fence_after();
+      const uint32_t dbase = lane_base + as * kColSlot;
+      if constexpr (PHASE == kPhaseGateUp) {
+        float tsg = 1.f, tsu = 1.f;
+        if (p.tscale) {
+          tsg = p.tscale[2 * tl.e];
+          tsu = p.tscale[2 * tl.e + 1];
+        }
+        for (int j0 = 0; j0 < tl.n; j0 += 32) {
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            if (j0 + 16 * hf < tl.n) {
+              uint32_t g[16], u[16];
+              tc_ld16(dbase + j0 + 16 * hf, g);
+              tc_ld16(dbase + kColD1 + j0 + 16 * hf, u);
+              tc_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                const float gv = __uint_as_float(g[c]) * tsg, uv = __uint_as_float(u[c]) * tsu;
+                slab[(16 * hf + c) * kSlabPitch + r] = silu_fast(gv) * uv;
+              }
+            }
+          }
+          named_bar_sync(1, 128);
+          for (int jj = 8 * q; jj < 8 * q + 8; ++jj) {
+            if (j0 + jj >= tl.n) break;
+            const float4 hv = *reinterpret_cast<const float4*>(slab + jj * kSlabPitch + 4 * lane);
+            float v[4] = {hv.x, hv.y, hv.z, hv.w};
+            if constexpr (FMT == kInt4) fwht128_warp(v);
+            store_seg_half(p.hq + static_cast<size_t>(tl.row0 + j0 + jj) * kI + tl.rp * 128, v, FMT == kInt4);
+          }
+          named_bar_sync(1, 128);
+        }
+      } else {
+        const float ts = p.tscale ? p.tscale[tl.e] : 1.f;
+        for (int j0 = 0; j0 < tl.n; j0 += 16) {
+          uint32_t d0[16], d1[16];
+          tc_ld16(dbase + j0, d0);
+          tc_ld16(dbase + kColD1 + j0, d1);
+          tc_wait_ld();
+          float* orow = p.o + static_cast<size_t>(tl.row0 + j0) * kH + tl.rp * 256 + r;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            if (j0 + c < tl.n) {
+              orow[static_cast<size_t>(c) * kH] = __uint_as_float(d0[c]) * ts;
+              orow[static_cast<size_t>(c) * kH + 128] = __uint_as_float(d1[c]) * ts;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bb.acc_empty[as]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+}
+
+// ---------------------------------------------------------------------------------------------
+// shared expert: dense bf16 GEMM, operands by TMA
+
+constexpr int kShThreads = 256;
+constexpr uint32_t kShColD1 = 128;                   // D1 after the 128 columns of D0
+constexpr int kShBox = 128 * 128;                    // 128 rows x 64 bf16, 128-byte swizzled
+
+template <int PHASE>
+struct ShGeom;
+template <>
+struct ShGeom<kPhaseGateUp> {
+  static constexpr int S = kH / 64, RP = kIs / 128, NB = 1, D = 4;
+  __device__ static int row(int rp, int b) { return b * kIs + rp * 128; }
+};
+template <>
+struct ShGeom<kPhaseDown> {
+  static constexpr int S = kIs / 64, RP = kH / 256, NB = 2, D = 3;
+  __device__ static int row(int rp, int b) { return rp * 256 + b * 128; }
+};
+// router logits: A = router rows (experts rp*256 + b*128 ..), B = x; RP = ceil(E / 256) at run time
+template <>
+struct ShGeom<kPhaseRouter> {
+  static constexpr int S = kH / 64, RP = 0, NB = 1, D = 4;
+  __device__ static int row(int rp, int b) { return rp * 256 + b * 128; }
+};
+
+template <int PHASE>
+struct ShLayout {
+  using G = ShGeom<PHASE>;
+  static constexpr int kStage = (2 + G::NB) * kShBox;
+  static constexpr int kOffBar = G::D * kStage;
+};
+
+struct ShBars {
+  uint64_t full[4], empty[4];
+  uint64_t acc_full[2], acc_empty[2], fin[2];
+  uint32_t tmem;
+  int abort;
+};
+
+template <int PHASE>
+constexpr int sh_smem() {
+  return ShLayout<PHASE>::kOffBar + static_cast<int>(sizeof(ShBars)) + 1024;
+}
+static_assert(sh_smem<kPhaseGateUp>() <= 227 * 1024 && sh_smem<kPhaseDown>() <= 227 * 1024 &&
+                  sh_smem<kPhaseRouter>() <= 227 * 1024,
+              "shared memory per CTA");
+
+template <int PHASE>
+__global__ void __launch_bounds__(kShThreads, 1) pf_shared_kernel(const __grid_constant__ PrefillParams p) {
+  using G = ShGeom<PHASE>;
+  using L = ShLayout<PHASE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  ShBars& bb = *reinterpret_cast<ShBars*>(sm + L::kOffBar);
+  volatile int* abort = &bb.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = (p.T + 127) / 128;
+  const int total = (PHASE == kPhaseRouter ? (p.E + 255) / 256 : G::RP) * nch;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < G::D; ++i) {
+      mbar_init(&bb.full[i], 1);
+      mbar_init(&bb.empty[i], 2);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bb.acc_full[b], 1);
+      mbar_init(&bb.acc_empty[b], 1);
+      mbar_init(&bb.fin[b], 1);
+    }
+    bb.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(smem_u32(&bb.tmem)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bb.tmem;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+        const int rp = t / nch, c0 = (t - rp * nch) * 128;
+        for (int s = 0; s < G::S; ++s, ++it) {
+          const int slot = it % G::D;
+          if (it >= G::D && !pf_wait(&bb.empty[slot], ((it / G::D) - 1) & 1, abort, p.err)) break;
+          uint8_t* st = sm + slot * L::kStage;
+          mbar_arrive_expect_tx(&bb.full[slot], L::kStage);
+          tma_2d(st, &p.tm_a, s * 64, G::row(rp, 0), &bb.full[slot]);
+          tma_2d(st + kShBox, &p.tm_a, s * 64, G::row(rp, 1), &bb.full[slot]);
+          tma_2d(st + 2 * kShBox, &p.tm_b, s * 64, c0, &bb.full[slot]);
+          if constexpr (G::NB == 2) tma_2d(st + 3 * kShBox, &p.tm_b2, s * 64, c0, &bb.full[slot]);
+        }
+      }
+      for (int j = max(it - G::D, 0); j < it; ++j) pf_wait(&bb.full[j % G::D], (j / G::D) & 1, abort, p.err);
+    }
+  } else if (warp == 1 || warp == 2) {
+    const int b = warp - 1;
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      const uint32_t idesc = idesc_m128(128, true);
+      const uint32_t d = tmem + b * kShColD1;
+      for (int t = blockIdx.x, ti = 0; t < total && ok; t += gridDim.x, ++ti) {
+        if (ti > 0 && !pf_wait(&bb.acc_empty[b], (ti - 1) & 1, abort, p.err)) break;   // D drained
+        tc_fence_after();
+        for (int s = 0; s < G::S; ++s, ++it) {
+          const int slot = it % G::D;
+          if (!pf_wait(&bb.full[slot], (it / G::D) & 1, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_u32(sm + slot * L::kStage);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = sdesc_sw128(st + b * kShBox + ks * 32);
+            tc_mma_ss(d, ad, sdesc_sw128(st + 2 * kShBox + ks * 32), idesc, (s | ks) ? 1u : 0u);
+            if constexpr (G::NB == 2) tc_mma_ss(d, ad, sdesc_sw128(st + 3 * kShBox + ks * 32), idesc, 1u);
+          }
+          tc_commit(&bb.empty[slot]);
+        }
+        if (ok) tc_commit(&bb.acc_full[b]);
+      }
+      tc_commit(&bb.fin[b]);                        // every MMA of this thread has completed
+      pf_wait(&bb.fin[b], 0, abort, p.err);
+    }
+  } else if (warp >= 4) {
+    const int q = warp & 3, r = 32 * q + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    for (int t = blockIdx.x, ti = 0; t < total; t += gridDim.x, ++ti) {
+      const int rp = t / nch, c0 = (t - rp * nch) * 128;
+      const int n = min(128, p.T - c0);
+      if (!pf_wait_all(&bb.acc_full[0], ti & 1, abort, p.err) || !pf_wait_all(&bb.acc_full[1], ti & 1, abort, p.err))
+        break;
+      tc_fence_after();
+      for (int j0 = 0; j0 < n; j0 += 16) {
+        uint32_t d0[16], d1[16];
+        tc_ld16(lane_base + j0, d0);
+        tc_ld16(lane_base + kShColD1 + j0, d1);
+        tc_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          if (j0 + c >= n) break;
+          const size_t tok = static_cast<size_t>(c0 + j0 + c);
+          if constexpr (PHASE == kPhaseRouter) {
+            const int e0 = rp * 256 + r;
+            if (e0 < p.E) p.logits[tok * p.E + e0] = __uint_as_float(d0[c]);
+            if (e0 + 128 < p.E) p.logits[tok * p.E + e0 + 128] = __uint_as_float(d1[c]);
+          } else if constexpr (PHASE == kPhaseGateUp) {
+            const float hs = silu_fast(__uint_as_float(d0[c])) * __uint_as_float(d1[c]);
+            const uint16_t hi = f32_to_bf16_bits(hs);
+            const uint16_t lo = f32_to_bf16_bits(hs - bf16_bits_to_f32(hi));
+            p.hs_hi[tok * kIs + rp * 128 + r] = hi;
+            p.hs_lo[tok * kIs + rp * 128 + r] = lo;
+          } else {
+            p.ys[tok * kH + rp * 256 + r] = __uint_as_float(d0[c]);
+            p.ys[tok * kH + rp * 256 + 128 + r] = __uint_as_float(d1[c]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 128) {                     // D drained: the issuers may overwrite it
+        mbar_arrive(&bb.acc_empty[0]);
+        mbar_arrive(&bb.acc_empty[1]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem));
+}
+
+template <typename Kern>
+cudaError_t allow_smem(Kern kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, int n_sm, cudaStream_t s) {
+  static bool smem_set = false;
+  if (!smem_set) {
+    cudaError_t e;
+    if ((e = allow_smem(pf_routed_kernel<kInt4, kPhaseGateUp>, kPfSmem)) != cudaSuccess) return e;
+    if ((e = allow_smem(pf_routed_kernel<kInt4, kPhaseDown>, kPfSmem)) != cudaSuccess) return e;
+    if ((e = allow_smem(pf_routed_kernel<kNvfp4, kPhaseGateUp>, kPfSmem)) != cudaSuccess) return e;
+    if ((e = allow_smem(pf_routed_kernel<kNvfp4, kPhaseDown>, kPfSmem)) != cudaSuccess) return e;
+    smem_set = true;
+  }
+  if (fmt == kInt4) {
+    if (phase == kPhaseGateUp) pf_routed_kernel<kInt4, kPhaseGateUp><<<n_sm, kPfThreads, kPfSmem, s>>>(p);
+    else pf_routed_kernel<kInt4, kPhaseDown><<<n_sm, kPfThreads, kPfSmem, s>>>(p);
+  } else {
+    if (phase == kPhaseGateUp) pf_routed_kernel<kNvfp4, kPhaseGateUp><<<n_sm, kPfThreads, kPfSmem, s>>>(p);
+    else pf_routed_kernel<kNvfp4, kPhaseDown><<<n_sm, kPfThreads, kPfSmem, s>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, cudaStream_t s) {
+  static bool smem_set = false;
+  if (!smem_set) {
+    cudaError_t e;
+    if ((e = allow_smem(pf_shared_kernel<kPhaseGateUp>, sh_smem<kPhaseGateUp>())) != cudaSuccess) return e;
+    if ((e = allow_smem(pf_shared_kernel<kPhaseDown>, sh_smem<kPhaseDown>())) != cudaSuccess) return e;
+    if ((e = allow_smem(pf_shared_kernel<kPhaseRouter>, sh_smem<kPhaseRouter>())) != cudaSuccess) return e;
+    smem_set = true;
+  }
+  const int rp = phase == kPhaseGateUp ? ShGeom<kPhaseGateUp>::RP
+                 : phase == kPhaseDown ? ShGeom<kPhaseDown>::RP
+                                       : (p.E + 255) / 256;
+  const int tiles = rp * ((p.T + 127) / 128);
+  const int grid = tiles < n_sm ? tiles : n_sm;
+  if (phase == kPhaseGateUp) pf_shared_kernel<kPhaseGateUp><<<grid, kShThreads, sh_smem<kPhaseGateUp>(), s>>>(p);
+  else if (phase == kPhaseDown) pf_shared_kernel<kPhaseDown><<<grid, kShThreads, sh_smem<kPhaseDown>(), s>>>(p);
+  else pf_shared_kernel<kPhaseRouter><<<grid, kShThreads, sh_smem<kPhaseRouter>(), s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace flint

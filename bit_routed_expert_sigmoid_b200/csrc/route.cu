@@ -235,12 +235,13 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __rest
 }
 
 // ---------------------------------------------------------------------------------------------
-// Routed-expert activation operand: xq = fp16(Hn x) per 128-segment for the int4 format (the codes
-// store W*blockdiag(Hn): Aijuus/flint-w4exp, weights row) or fp16(x) for NVFP4. One warp per
-// (token, segment). For int4 every 8-block is stored in the order 0,4,1,5,2,6,3,7 to match the
-// fp16 pairs the int4 decoder produces.
-__global__ void __launch_bounds__(256) xq_kernel(const uint16_t* __restrict__ x, int T, int rotate,
-                                                 __half* __restrict__ xq) {
+// Routed-expert activation operand of the prefill path: fp16(Hn x) per 128-segment for the int4
+// format (the codes store W*blockdiag(Hn): Aijuus/flint-w4exp, weights row) or fp16(x) for NVFP4,
+// written once per slot of the token at its permuted row inv[t][k], so that the rows of one expert
+// are contiguous. One warp per (token, segment). For int4 every 8-block is stored in the order
+// 0,4,1,5,2,6,3,7 to match the fp16 pairs the int4 decoder produces.
+__global__ void __launch_bounds__(256) xg_kernel(const uint16_t* __restrict__ x, int T, int K,
+                                                 const int* __restrict__ inv, int rotate, __half* __restrict__ xg) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gw = blockIdx.x * 8 + warp;
   const int t = gw / (kH / kGroup), seg = gw % (kH / kGroup);
@@ -249,7 +250,10 @@ __global__ void __launch_bounds__(256) xq_kernel(const uint16_t* __restrict__ x,
   const uint2 raw = ld_nc_v2(src);
   float v[4] = {bf16lo_to_f32(raw.x), bf16hi_to_f32(raw.x), bf16lo_to_f32(raw.y), bf16hi_to_f32(raw.y)};
   if (rotate) fwht128_warp(v);
-  store_seg_half(xq + static_cast<size_t>(t) * kH + seg * kGroup, v, rotate != 0);
+  for (int k = 0; k < K; ++k) {
+    const int prow = inv[t * K + k];
+    store_seg_half(xg + static_cast<size_t>(prow) * kH + seg * kGroup, v, rotate != 0);
+  }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -274,9 +278,9 @@ cudaError_t launch_permute(const int* ids, int T, int K, int E, int* counts, int
   return cudaGetLastError();
 }
 
-cudaError_t launch_xq(const uint16_t* x, int T, int rotate, __half* xq, cudaStream_t s) {
+cudaError_t launch_xg(const uint16_t* x, int T, int K, const int* inv, int rotate, __half* xg, cudaStream_t s) {
   const int warps = T * (kH / kGroup);
-  xq_kernel<<<(warps + 7) / 8, 256, 0, s>>>(x, T, rotate, xq);
+  xg_kernel<<<(warps + 7) / 8, 256, 0, s>>>(x, T, K, inv, rotate, xg);
   return cudaGetLastError();
 }
 

@@ -132,8 +132,10 @@ flint_status flint_moe_routing(flint_moe_t h, int* ids, float* w, int* offsets, 
 /* Intermediates of the last forward, for tests: device-to-device copy of `bytes` bytes. */
 enum {
   FLINT_BUF_LOGITS = 0,   /* f32 [T][E] router logits */
-  FLINT_BUF_XQ = 1,       /* fp16 [T][H] the routed experts' input: rotated x (int4) or x (nvfp4),
-                             each 8-element block stored in the order 0,4,1,5,2,6,3,7 for int4 */
+  FLINT_BUF_XQ = 1,       /* fp16, the routed experts' input: rotated x (int4) or x (nvfp4), each
+                             8-element block stored in the order 0,4,1,5,2,6,3,7 for int4; [T][H]
+                             after a forward with T <= 8, [T*top_k][H] in permuted row order (row p
+                             holds token perm[p] / top_k) after a larger one */
   FLINT_BUF_YS = 2        /* f32 [T][H] shared-expert output */
 };
 flint_status flint_moe_intermediate(flint_moe_t h, int which, void* dst, size_t bytes, void* stream);
