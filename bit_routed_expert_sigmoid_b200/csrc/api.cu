@@ -292,12 +292,10 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   pp.top_k = K;
   pp.E = E;
   pp.logits = h->logits;
-  pp.active = h->active;
-  pp.n_active = h->n_active;
   pp.offsets = h->offsets;
   pp.perm = h->perm;
   pp.hq = h->hq;
-  pp.o = h->o;
+  pp.o = reinterpret_cast<__half*>(h->o);          // fp16 [P][H] view of the fp32 buffer
   pp.hs_hi = h->hs_hi;
   pp.hs_lo = h->hs_lo;
   pp.ys = h->ys;
@@ -309,7 +307,7 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   FLINT_TRY(m.mark());
   FLINT_TRY(launch_topk(h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, s));
   FLINT_TRY(m.mark());
-  FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, h->active, h->n_active, c.flags,
+  FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, c.flags,
                            h->err, s));
   FLINT_TRY(m.mark());
   FLINT_TRY(launch_xg(x, T, K, h->inv, fmt == kInt4 ? 1 : 0, h->xg, s));
@@ -335,7 +333,7 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   pp.tm_b2 = h->tm_pf_hs_lo;
   FLINT_TRY(launch_prefill_shared(pp, kPhaseDown, h->n_sm, s));
   FLINT_TRY(m.mark());
-  FLINT_TRY(launch_combine(h->o, h->ys, h->wts, h->inv, T, K, c.routed_scale, y, s));
+  FLINT_TRY(launch_prefill_combine(reinterpret_cast<const __half*>(h->o), h->ys, h->wts, h->inv, T, K, c.routed_scale, y, s));
   FLINT_TRY(m.mark());
   return FLINT_OK;
 }

@@ -16,7 +16,7 @@
 //   warps 1, 2   one MMA-issuing thread per block (an MMA instruction takes ~45 cycles to issue, so
 //                two issuers keep N = 48 tiles near the tensor-core rate); D[128 x N] per block
 //   warps 12-15  epilogue: gate|up -> h = silu(g) u, int4: rotated per 128-segment by the Hadamard
-//                butterfly, stored fp16 in the order of the down operand; down -> o in fp32.
+//                butterfly, stored fp16 in the order of the down operand; down -> o in fp16.
 // Every dependency is an mbarrier: TMA transaction counts, cp.async arrivals, tcgen05.commit
 // arrivals and thread arrivals; every wait is bounded and sets a timeout bit on expiry.
 //
@@ -149,7 +149,7 @@ __device__ __forceinline__ bool pf_wait_all(uint64_t* bar, uint32_t parity, vola
 
 struct TileTab {
   int n, total;
-  int start[kMaxE + 1];   // first tile of active expert i
+  int start[kMaxE + 1];   // first tile of expert i
   int e[kMaxE];
   int off[kMaxE];         // first permuted row
   int cnt[kMaxE];         // permuted rows
@@ -160,16 +160,17 @@ struct PfTile {
   int e, row0, n, rp;     // expert, first permuted row of the chunk, rows in it (1..kPfN), block pair
 };
 
-// Warp 0: tiles of active expert i are rp-major over its chunks; experts in ascending order.
+// Warp 0: tiles of expert e are rp-major over its chunks; experts in ascending order (an expert
+// without rows has none).
 __device__ void build_tiles(TileTab& tt, const PrefillParams& p, int rp_count) {
   const int lane = threadIdx.x & 31;
-  const int n = min(*p.n_active, kMaxE);
+  const int n = min(p.E, kMaxE);
   int base = 0;
   for (int i0 = 0; i0 < n; i0 += 32) {
     const int i = i0 + lane;
     int tiles = 0;
     if (i < n) {
-      const int e = p.active[i];
+      const int e = i;
       const int off = p.offsets[e];
       const int c = max(p.offsets[e + 1] - off, 0);
       const int nch = (c + kPfN - 1) / kPfN;
@@ -563,12 +564,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_c
           tc_ld16(dbase + j0, d0);
           tc_ld16(dbase + kColD1 + j0, d1);
           tc_wait_ld();
-          float* orow = p.o + static_cast<size_t>(tl.row0 + j0) * kH + tl.rp * 256 + r;
+          __half* orow = p.o + static_cast<size_t>(tl.row0 + j0) * kH + tl.rp * 256 + r;
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             if (j0 + c < tl.n) {
-              orow[static_cast<size_t>(c) * kH] = __uint_as_float(d0[c]) * ts;
-              orow[static_cast<size_t>(c) * kH + 128] = __uint_as_float(d1[c]) * ts;
+              orow[static_cast<size_t>(c) * kH] = __float2half_rn(__uint_as_float(d0[c]) * ts);
+              orow[static_cast<size_t>(c) * kH + 128] = __float2half_rn(__uint_as_float(d1[c]) * ts);
             }
           }
         }
@@ -766,6 +767,40 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shared_kernel(const __grid_c
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem));
 }
 
+// ---------------------------------------------------------------------------------------------
+// combine: y[t][n] = bf16(routed_scale * sum_k w[t][k] * o[inv[t][k]][n] + ys[t][n]), the slots
+// summed in slot order (ascending expert id) in fp32, one rounding at the end. One CTA per token,
+// 8 columns per thread.
+__global__ void __launch_bounds__(256) pf_combine_kernel(const __half* __restrict__ o, const float* __restrict__ ys,
+                                                         const float* __restrict__ w, const int* __restrict__ inv,
+                                                         int K, float routed_scale, uint16_t* __restrict__ y) {
+  const int t = blockIdx.x;
+  const int n = threadIdx.x * 8;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  for (int k = 0; k < K; ++k) {
+    const float wk = w[t * K + k];
+    const uint4 ov = *reinterpret_cast<const uint4*>(o + static_cast<size_t>(inv[t * K + k]) * kH + n);
+    const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ow[j]));
+      acc[2 * j] = fmaf(wk, f.x, acc[2 * j]);
+      acc[2 * j + 1] = fmaf(wk, f.y, acc[2 * j + 1]);
+    }
+  }
+  const float4 s0 = *reinterpret_cast<const float4*>(ys + static_cast<size_t>(t) * kH + n);
+  const float4 s1 = *reinterpret_cast<const float4*>(ys + static_cast<size_t>(t) * kH + n + 4);
+  const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+  uint4 out;
+  uint32_t* ou = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    ou[j] = pack_bf162(fmaf(routed_scale, acc[2 * j], sv[2 * j]), fmaf(routed_scale, acc[2 * j + 1], sv[2 * j + 1]));
+  *reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * kH + n) = out;
+}
+
 template <typename Kern>
 cudaError_t allow_smem(Kern kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -810,6 +845,13 @@ cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, c
   if (phase == kPhaseGateUp) pf_shared_kernel<kPhaseGateUp><<<grid, kShThreads, sh_smem<kPhaseGateUp>(), s>>>(p);
   else if (phase == kPhaseDown) pf_shared_kernel<kPhaseDown><<<grid, kShThreads, sh_smem<kPhaseDown>(), s>>>(p);
   else pf_shared_kernel<kPhaseRouter><<<grid, kShThreads, sh_smem<kPhaseRouter>(), s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_combine(const __half* o, const float* ys, const float* w, const int* inv, int T, int K,
+                                   float routed_scale, uint16_t* y, cudaStream_t s) {
+  static_assert(kH == 256 * 8, "one CTA of 256 threads x 8 columns per token");
+  pf_combine_kernel<<<T, 256, 0, s>>>(o, ys, w, inv, K, routed_scale, y);
   return cudaGetLastError();
 }
 

@@ -1,12 +1,14 @@
-// Routing stage of the Flint MoE layer: router logits, unbiased sigmoid top-k with the
+// Routing stage of the prefill path of the Flint MoE layer: unbiased sigmoid top-k with the
 // selected-sum floor, the expert-major permutation of (token, slot) pairs, and the activation
-// operand of the routed experts (x rotated per 128-segment for the int4 format).
+// operand of the routed experts (x rotated per 128-segment for the int4 format). The forward's
+// router logits come from the tensor-core kernel in prefill.cu; the CUDA-core kernel here serves the
+// routing-only entry point.
 #include "kernels.cuh"
 
 namespace flint {
 
 // ---------------------------------------------------------------------------------------------
-// Router logits on CUDA cores: logits[t][e] = sum_j W_r[e][j] * x[t][j]. The bf16 x bf16 products
+// Router logits on CUDA cores, for the routing-only entry point (small T): logits[t][e] = sum_j W_r[e][j] * x[t][j]. The bf16 x bf16 products
 // are exact in fp32 and accumulate in fp32 (the router rows are used widened to FP32 on the
 // pages: WaveCut/Flint-UD-Q4_K_XL-NInfer-v3, "What is inside"). One warp owns one expert row and
 // a chunk of up to 8 tokens; lane l covers elements 8l + 256i (i = 0..7) so every load is a
@@ -70,8 +72,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 #pragma unroll
   for (int j = 0; j < 8; ++j) v[j] = (j < per) ? logits[static_cast<size_t>(t) * E + lane + 32 * j] : -INFINITY;
   unsigned taken = 0;              // bit j: element lane+32j already chosen
-  int chosen[kMaxTopK];
-  float chosen_l[kMaxTopK];
+  int my_id = 0x7FFFFFFF;          // lane k < K: the k-th pick
+  float my_l = 0.f;
   for (int k = 0; k < K; ++k) {
     // local best: highest logit, then lowest index
     float bv = -INFINITY;
@@ -88,27 +90,31 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
       const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, m);
       if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
-    chosen[k] = bi;
-    chosen_l[k] = bv;
+    if (lane == k) {
+      my_id = bi;
+      my_l = bv;
+    }
     if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
   }
-  // order the slots by expert id; lane k < K writes slot k
-  float s_sorted[kMaxTopK];
-  int id_sorted[kMaxTopK];
-  for (int k = 0; k < K; ++k) {
-    int rank = 0;
-    for (int j = 0; j < K; ++j) rank += (chosen[j] < chosen[k]);
-    id_sorted[rank] = chosen[k];
-    s_sorted[rank] = 1.0f / (1.0f + expf(-chosen_l[k]));
+  // slot of the pick = its rank by expert id; lane r then takes the pick of rank r
+  int rank = 0;
+  for (int j = 0; j < K; ++j) rank += (__shfl_sync(0xFFFFFFFFu, my_id, j) < my_id);
+  const float my_s = 1.0f / (1.0f + expf(-my_l));
+  int id = 0;
+  float s = 0.f, sum = 0.f;
+  for (int r = 0; r < K; ++r) {
+    const unsigned who = __ballot_sync(0xFFFFFFFFu, lane < K && rank == r);
+    const int src = __ffs(who) - 1;
+    const int id_r = __shfl_sync(0xFFFFFFFFu, my_id, src);
+    const float s_r = __shfl_sync(0xFFFFFFFFu, my_s, src);
+    sum += s_r;                    // slot order
+    if (lane == r) {
+      id = id_r;
+      s = s_r;
+    }
   }
-  float sum = 0.f;
-  for (int k = 0; k < K; ++k) sum += s_sorted[k];
   const float denom = fmaxf(sum, floor_);
   if (lane < K) {
-    int id = 0;
-    float s = 0.f;
-    for (int k = 0; k < K; ++k)
-      if (k == lane) { id = id_sorted[k]; s = s_sorted[k]; }
     if ((flags & 1u) && (id < 0 || id >= E)) atomicOr(err, kErrBadId);
     ids[t * K + lane] = id;
     wts[t * K + lane] = s / denom;
@@ -116,121 +122,121 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 }
 
 // ---------------------------------------------------------------------------------------------
-// Expert-major permutation of the (token, slot) pairs, one CTA of 512 threads.
+// Expert-major permutation of the (token, slot) pairs: one CTA per expert e.
 // counts[e] = number of pairs routed to e; offsets = exclusive prefix (E+1 entries);
 // position p in [offsets[e], offsets[e+1]) lists the pairs of expert e by ascending token:
-// perm[p] = t*K+k and inv[t*K+k] = p. Ranks come from per-warp bitmasks and prefix sums, never
-// from the order atomics happen to run in, so the result is deterministic. Also lists the experts
-// that received tokens (ascending) in active[0..n_active).
-constexpr int kPermThreads = 512;
+// perm[p] = t*K+k and inv[t*K+k] = p. Every CTA reads all P = T*K expert ids (L2-resident):
+// pass 1 counts the pairs routed below e (its offset) and to e; a block scan over the threads'
+// contiguous shares gives each thread its first position; pass 2 writes the pairs of e in pair
+// order (a token routes to e at most once, so pair order is token order). No atomics decide an
+// order, so the result is deterministic. Invalid ids count as expert 0 (and are flagged).
+constexpr int kPermThreads = 1024;
 constexpr int kPermWarps = kPermThreads / 32;
+constexpr int kPermChunk = 16;                   // ids a thread holds in registers per round
 
-__global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __restrict__ ids, int T, int K, int E,
+__device__ __forceinline__ int clamp_id(int v, int E) { return (v < 0 || v >= E) ? 0 : v; }
+
+// Loads ids [i0, i0 + 16) as four 16-byte vectors (entries past P are not read); i0 is a multiple of 16.
+__device__ __forceinline__ void load_ids16(int (&v)[kPermChunk], const int* ids, int i0, int P) {
+  if (i0 + kPermChunk <= P) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int4 w = __ldg(reinterpret_cast<const int4*>(ids + i0) + q);
+      v[4 * q] = w.x;
+      v[4 * q + 1] = w.y;
+      v[4 * q + 2] = w.z;
+      v[4 * q + 3] = w.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kPermChunk; ++j) v[j] = (i0 + j < P) ? __ldg(ids + i0 + j) : 0;
+  }
+}
+
+// Counts the first `nv` of the thread's ids that are below e and equal to e.
+__device__ __forceinline__ void count_ids(const int (&v)[kPermChunk], int nv, int e, int E, int& lt, int& eq,
+                                          bool& bad) {
+#pragma unroll
+  for (int j = 0; j < kPermChunk; ++j) {
+    if (j >= nv) continue;
+    bad |= v[j] < 0 || v[j] >= E;
+    const int c = clamp_id(v[j], E);
+    lt += c < e;
+    eq += c == e;
+  }
+}
+
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __restrict__ ids, int P, int E,
                                                                int* __restrict__ counts, int* __restrict__ offsets,
                                                                int* __restrict__ perm, int* __restrict__ inv,
-                                                               int* __restrict__ active, int* __restrict__ n_active,
                                                                unsigned flags, unsigned* __restrict__ err) {
-  __shared__ int cnt[kMaxE];
-  __shared__ int run[kMaxE];
-  __shared__ unsigned mask[kPermWarps][kMaxE];
-  __shared__ int base[kPermWarps][kMaxE];
+  __shared__ int w_sum[kPermWarps], w_base[kPermWarps];
+  __shared__ int s_total;
+  const int e = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < kMaxE; e += kPermThreads) cnt[e] = 0;
-  __syncthreads();
-  const int P = T * K;
-  for (int i = tid; i < P; i += kPermThreads) {
-    int e = ids[i];
-    if (e < 0 || e >= E) {
-      if (flags & 1u) atomicOr(err, kErrBadId);
-      e = 0;
-    }
-    atomicAdd(&cnt[e], 1);
-  }
-  __syncthreads();
-  // exclusive scan over experts by warp 0 (8 experts per lane)
-  if (warp == 0) {
-    int loc[8];
-    int s = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = lane * 8 + j;
-      loc[j] = s;
-      s += (e < E) ? cnt[e] : 0;
-    }
-    int incl = s;
+  constexpr int kRound = kPermThreads * kPermChunk;
+  // warp-order exclusive scan of one value per thread over the CTA; returns the exclusive prefix and
+  // leaves the CTA total in s_total
+  auto block_scan = [&](int x) -> int {
+    int incl = x;
 #pragma unroll
     for (int m = 1; m < 32; m <<= 1) {
       const int o = __shfl_up_sync(0xFFFFFFFFu, incl, m);
       if (lane >= m) incl += o;
     }
-    const int excl = incl - s;
+    __syncthreads();                               // w_sum / s_total of a previous scan are consumed
+    if (lane == 31) w_sum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int c = w_sum[lane];
+      int s = c;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = lane * 8 + j;
-      if (e < E) {
-        offsets[e] = excl + loc[j];
-        run[e] = excl + loc[j];
-        counts[e] = cnt[e];
+      for (int m = 1; m < 32; m <<= 1) {
+        const int o = __shfl_up_sync(0xFFFFFFFFu, s, m);
+        if (lane >= m) s += o;
       }
+      w_base[lane] = s - c;
+      if (lane == 31) s_total = s;
     }
-    if (lane == 31) offsets[E] = incl;
-    // active experts (count > 0), ascending
-    int fl[8];
-    int fs = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = lane * 8 + j;
-      fl[j] = fs;
-      fs += (e < E && cnt[e] > 0) ? 1 : 0;
-    }
-    int finc = fs;
-#pragma unroll
-    for (int m = 1; m < 32; m <<= 1) {
-      const int o = __shfl_up_sync(0xFFFFFFFFu, finc, m);
-      if (lane >= m) finc += o;
-    }
-    const int fex = finc - fs;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = lane * 8 + j;
-      if (e < E && cnt[e] > 0) active[fex + fl[j]] = e;
-    }
-    if (lane == 31) *n_active = finc;
+    __syncthreads();
+    return w_base[warp] + incl - x;
+  };
+  // pass 1: pairs routed below e (the offset of e)
+  int v[kPermChunk];
+  int lt = 0, eq_unused = 0;
+  bool bad = false;
+  for (int r0 = 0; r0 < P; r0 += kRound) {
+    const int i0 = r0 + kPermChunk * tid;
+    load_ids16(v, ids, i0, P);
+    count_ids(v, min(max(P - i0, 0), kPermChunk), e, E, lt, eq_unused, bad);
   }
-  __syncthreads();
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int t0 = 0; t0 < T; t0 += kPermThreads) {
-    for (int e = lane; e < kMaxE; e += 32) mask[warp][e] = 0u;
-    __syncwarp();
-    const int t = t0 + tid;
-    int my_e[kMaxTopK];
-    if (t < T) {
-      for (int k = 0; k < K; ++k) {
-        int e = ids[t * K + k];
-        if (e < 0 || e >= E) e = 0;
-        my_e[k] = e;
-        atomicOr(&mask[warp][e], 1u << lane);
+  if (bad && (flags & 1u) && e == 0) atomicOr(err, kErrBadId);
+  block_scan(lt);
+  const int off = s_total;
+  // pass 2: the pairs of e in pair order at off, off + 1, ...
+  int run = 0;
+  for (int r0 = 0; r0 < P; r0 += kRound) {
+    const int i0 = r0 + kPermChunk * tid;
+    const int nv = min(max(P - i0, 0), kPermChunk);
+    if (P > kRound) load_ids16(v, ids, i0, P);     // one round: the ids are still in registers
+    int l2 = 0, eq = 0;
+    bool b2 = false;
+    count_ids(v, nv, e, E, l2, eq, b2);
+    int pos = off + run + block_scan(eq);
+    run += s_total;
+#pragma unroll
+    for (int j = 0; j < kPermChunk; ++j) {
+      if (j < nv && clamp_id(v[j], E) == e) {
+        perm[pos] = i0 + j;
+        inv[i0 + j] = pos;
+        ++pos;
       }
     }
-    __syncthreads();
-    for (int e = tid; e < E; e += kPermThreads) {
-      int b = run[e];
-      for (int w = 0; w < kPermWarps; ++w) {
-        base[w][e] = b;
-        b += __popc(mask[w][e]);
-      }
-      run[e] = b;
-    }
-    __syncthreads();
-    if (t < T) {
-      for (int k = 0; k < K; ++k) {
-        const int e = my_e[k];
-        const int p = base[warp][e] + __popc(mask[warp][e] & lt_mask);
-        perm[p] = t * K + k;
-        inv[t * K + k] = p;
-      }
-    }
-    __syncthreads();
+  }
+  if (tid == 0) {
+    counts[e] = run;
+    offsets[e] = off;
+    if (e == E - 1) offsets[E] = off + run;
   }
 }
 
@@ -273,8 +279,8 @@ cudaError_t launch_topk(const float* logits, int T, int E, int K, float floor_, 
 }
 
 cudaError_t launch_permute(const int* ids, int T, int K, int E, int* counts, int* offsets, int* perm, int* inv,
-                           int* active, int* n_active, unsigned flags, unsigned* err, cudaStream_t s) {
-  permute_kernel<<<1, kPermThreads, 0, s>>>(ids, T, K, E, counts, offsets, perm, inv, active, n_active, flags, err);
+                           unsigned flags, unsigned* err, cudaStream_t s) {
+  permute_kernel<<<E, kPermThreads, 0, s>>>(ids, T * K, E, counts, offsets, perm, inv, flags, err);
   return cudaGetLastError();
 }
 

@@ -91,6 +91,19 @@ def test_prefill_nvfp4_full_size():
     full_check(L, S.make_workload_x(2048, 256))
 
 
+def test_permutation_spans_rounds():
+    # T*K = 18000 (token, slot) pairs: more than one round of the permutation kernel's register
+    # blocking (16384 pairs); the permutation is rebuilt from the device's ids by the oracle
+    L = layer(32, "int4")
+    T = 3000
+    x = S.make_workload_x(T, 32)
+    dev, xd, y, ref, st = full_check(L, x)
+    r = dev.routing(T)
+    pr = R.permutation(r["ids"].cpu().numpy(), 32)
+    np.testing.assert_array_equal(r["offsets"].cpu().numpy(), pr["offsets"])
+    np.testing.assert_array_equal(r["perm"].cpu().numpy(), pr["perm"])
+
+
 def test_top1_routing():
     L = layer(32, "int4")
     x = S.make_x(16)
