@@ -54,6 +54,15 @@ struct flint_moe_ctx {
   // instrumentation (caller-owned cudaEvent_t handles)
   cudaEvent_t events[32];
   int n_events;
+  // prefill: the routing chain runs on `side` (higher priority) while the shared expert runs on the
+  // caller's stream; ev_fork / ev_join order the two
+  cudaStream_t side;
+  cudaEvent_t ev_fork, ev_join;
+  ~flint_moe_ctx() {
+    if (ev_join) cudaEventDestroy(ev_join);
+    if (ev_fork) cudaEventDestroy(ev_fork);
+    if (side) cudaStreamDestroy(side);
+  }
 };
 
 namespace {
@@ -128,6 +137,15 @@ bool encode_f16_rows64(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
 
 bool encode_code_tiles(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes) {
   return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, rows, row_bytes, 16, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// Side stream of the prefill routing chain, at the highest priority (it is the longer branch).
+bool create_side_stream(flint_moe_ctx* h) {
+  int lo = 0, hi = 0;
+  if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return false;
+  return cudaStreamCreateWithPriority(&h->side, cudaStreamNonBlocking, hi) == cudaSuccess &&
+         cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) == cudaSuccess;
 }
 
 // Lays the workspace out; with base == nullptr only the size is computed.
@@ -301,21 +319,41 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   pp.ys = h->ys;
   pp.err = h->err;
   // B = x as given (map encoded per call: x changes, rows past T read as zeros)
-  if (!encode_bf16_tiles(&pp.tm_b, x, T, kH)) return FLINT_ERR_CUDA;
+  CUtensorMap tm_x;
+  if (!encode_bf16_tiles(&tm_x, x, T, kH)) return FLINT_ERR_CUDA;
+  // The routing chain (router, top-k, permutation, activation operand) and the shared expert are
+  // independent; without instrumentation the chain runs on the side stream while the shared
+  // expert's kernels (which leave SMs free) run on `s`. With instrumentation everything runs on `s`
+  // in stage order.
+  const bool fork = h->n_events == 0 && h->side != nullptr;
+  cudaStream_t rs = fork ? h->side : s;
+  if (fork) {
+    FLINT_TRY(cudaEventRecord(h->ev_fork, s));
+    FLINT_TRY(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+  }
   pp.tm_a = h->tm_pf_router;
-  FLINT_TRY(launch_prefill_shared(pp, kPhaseRouter, h->n_sm, s));
+  pp.tm_b = tm_x;
+  FLINT_TRY(launch_prefill_shared(pp, kPhaseRouter, h->n_sm, rs));
   FLINT_TRY(m.mark());
-  FLINT_TRY(launch_topk(h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, s));
+  FLINT_TRY(launch_topk(h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, rs));
   FLINT_TRY(m.mark());
-  FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, c.flags,
-                           h->err, s));
+  FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, c.flags, h->err, rs));
   FLINT_TRY(m.mark());
-  FLINT_TRY(launch_xg(x, T, K, h->inv, fmt == kInt4 ? 1 : 0, h->xg, s));
+  FLINT_TRY(launch_xg(x, T, K, h->inv, fmt == kInt4 ? 1 : 0, h->xg, rs));
   FLINT_TRY(m.mark());
 
   pp.tm_a = h->tm_pf_sh_gu;                        // shared gate|up: B = x
+  pp.tm_b = tm_x;
   FLINT_TRY(launch_prefill_shared(pp, kPhaseGateUp, h->n_sm, s));
   FLINT_TRY(m.mark());
+  if (fork) {                                      // shared down right behind shared gate|up
+    pp.tm_a = h->tm_pf_sh_dn;
+    pp.tm_b = h->tm_pf_hs_hi;
+    pp.tm_b2 = h->tm_pf_hs_lo;
+    FLINT_TRY(launch_prefill_shared(pp, kPhaseDown, h->n_sm, s));
+    FLINT_TRY(cudaEventRecord(h->ev_join, h->side));
+    FLINT_TRY(cudaStreamWaitEvent(s, h->ev_join, 0));
+  }
   pp.tm_codes = h->tm_pf_gu;
   pp.tm_act = h->tm_pf_xg;
   pp.scales = h->w.gu_scales;
@@ -328,11 +366,13 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   pp.tscale = h->w.dn_tscale;
   FLINT_TRY(launch_prefill_routed(pp, fmt, kPhaseDown, h->n_sm, s));
   FLINT_TRY(m.mark());
-  pp.tm_a = h->tm_pf_sh_dn;
-  pp.tm_b = h->tm_pf_hs_hi;
-  pp.tm_b2 = h->tm_pf_hs_lo;
-  FLINT_TRY(launch_prefill_shared(pp, kPhaseDown, h->n_sm, s));
-  FLINT_TRY(m.mark());
+  if (!fork) {
+    pp.tm_a = h->tm_pf_sh_dn;
+    pp.tm_b = h->tm_pf_hs_hi;
+    pp.tm_b2 = h->tm_pf_hs_lo;
+    FLINT_TRY(launch_prefill_shared(pp, kPhaseDown, h->n_sm, s));
+    FLINT_TRY(m.mark());
+  }
   FLINT_TRY(launch_prefill_combine(reinterpret_cast<const __half*>(h->o), h->ys, h->wts, h->inv, T, K, c.routed_scale, y, s));
   FLINT_TRY(m.mark());
   return FLINT_OK;
@@ -388,7 +428,8 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
       !encode_bf16_tiles(&h->tm_pf_hs_hi, h->hs_hi, cfg->t_max, kIs) ||
       !encode_bf16_tiles(&h->tm_pf_hs_lo, h->hs_lo, cfg->t_max, kIs) ||
       !encode_f16_rows64(&h->tm_pf_xg, h->xg, static_cast<uint64_t>(cfg->t_max) * cfg->top_k, kH) ||
-      !encode_f16_rows64(&h->tm_pf_hq, h->hq, static_cast<uint64_t>(cfg->t_max) * cfg->top_k, kI)) {
+      !encode_f16_rows64(&h->tm_pf_hq, h->hq, static_cast<uint64_t>(cfg->t_max) * cfg->top_k, kI) ||
+      !create_side_stream(h)) {
     delete h;
     return FLINT_ERR_CUDA;
   }

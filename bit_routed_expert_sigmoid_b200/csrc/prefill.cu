@@ -261,38 +261,27 @@ __device__ __forceinline__ uint32_t scale_half2(uint32_t bf16_bits, bool& bad) {
   return pack_half2(s, s);
 }
 
-// Turns the 128 codes of one row of one stage into 64 fp16 pairs in tensor memory.
-// int4: word w of the row gives columns 4w..4w+3 = pairs (n0,n4),(n1,n5),(n2,n6),(n3,n7) of its
-// eight codes (the order the activation operand is stored in). NVFP4: natural order.
+// Turns 64 codes (8 words) of one row into 32 fp16 pairs: 32 tensor-memory columns of the row.
+// int4: word w gives columns 4w..4w+3 = pairs (n0,n4),(n1,n5),(n2,n6),(n3,n7) of its eight codes
+// (the order the activation operand is stored in). NVFP4: natural order; `s_blk` holds the four
+// E4M3 scales of the 16-code blocks.
 template <int FMT>
-__device__ __forceinline__ void dequant_stage(uint32_t taddr, const uint4 (&w)[4], uint32_t s_int4, uint2 s_fp4) {
+__device__ __forceinline__ void dequant_half(uint32_t (&v)[32], const uint4& wa, const uint4& wb, uint32_t s_int4,
+                                             uint32_t s_blk) {
+  const uint32_t words[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    uint32_t v[32];
+  for (int k = 0; k < 8; ++k) {
+    if constexpr (FMT == kInt4) {
+      uint32_t pr[4];
+      int4x8_to_half2x4(words[k], pr);
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const uint4 wv = w[2 * half + q];
-      const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+      for (int j = 0; j < 4; ++j) v[4 * k + j] = hmul2_u32(pr[j], s_int4);
+    } else {
+      const uint32_t h = e4m3_to_half_bits((s_blk >> (8 * (k >> 1))) & 0xFFu);
+      const uint32_t s2 = h | (h << 16);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int col = 16 * q + 4 * k;            // column within this half
-        if constexpr (FMT == kInt4) {
-          uint32_t pr[4];
-          int4x8_to_half2x4(words[k], pr);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) v[col + j] = hmul2_u32(pr[j], s_int4);
-        } else {
-          // word index within the stage = 8 half + 4 q + k; 16-code block = that / 2
-          const int blk = (8 * half + 4 * q + k) >> 1;
-          const uint32_t sb = (blk < 4 ? (s_fp4.x >> (8 * blk)) : (s_fp4.y >> (8 * (blk - 4)))) & 0xFFu;
-          const uint32_t h = e4m3_to_half_bits(sb);
-          const uint32_t s2 = h | (h << 16);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) v[col + j] = hmul2_u32(e2m1x2_to_half2(words[k] >> (8 * j)), s2);
-        }
-      }
+      for (int j = 0; j < 4; ++j) v[4 * k + j] = hmul2_u32(e2m1x2_to_half2(words[k] >> (8 * j)), s2);
     }
-    tc_st32(taddr + 32 * half, v);
   }
 }
 
@@ -497,12 +486,18 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_c
             for (int k = 0; k + 1 < kSc4; ++k) sc[k] = sc[k + 1];
           }
         }
+        // the first half's arithmetic runs before the tensor-memory stage is free
+        uint32_t v[32];
+        dequant_half<FMT>(v, w[0], w[1], s_int4, s_fp4.x);
         if (it >= 2 && !pf_wait_all(&bb.a_empty[ts][b], ((it >> 1) - 1) & 1, abort, p.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        dequant_stage<FMT>(lane_base + kColA + ts * 128 + b * 64, w, s_int4, s_fp4);
+        const uint32_t ta = lane_base + kColA + ts * 128 + b * 64;
+        tc_st32(ta, v);
+        dequant_half<FMT>(v, w[2], w[3], s_int4, s_fp4.y);
+        tc_st32(ta + 32, v);
         tc_wait_st();
         tc_fence_before();
         __syncwarp();

@@ -106,8 +106,9 @@ size_t flint_moe_workspace_size(const flint_moe_cfg* cfg);
 /* Validates cfg and the weight pointers, and records them with the caller's workspace (device,
  * 256-byte aligned, at least flint_moe_workspace_size bytes, owned by the caller). Allocates no
  * device memory; its only device work is two synchronous cudaMemsets that clear the handle's
- * 16-byte error word and its arrival counters inside the workspace. On success *out receives a
- * handle. */
+ * 16-byte error word and its arrival counters inside the workspace. It creates one non-blocking
+ * stream and two events of its own (released by flint_moe_destroy), on which forward() runs part
+ * of a T > 8 forward. On success *out receives a handle. */
 flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights* weights, void* workspace,
                               size_t workspace_bytes, flint_moe_t* out);
 
@@ -115,7 +116,10 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
  * 0 <= T <= t_max (T = 0 is a no-op). Enqueues the kernels on `stream` and returns; the host never
  * waits and nothing is copied back. T <= 8 takes the decode path: three kernels (route, gate|up,
  * down + combine) chained by programmatic dependent launch, so each one starts streaming weights
- * before its predecessor ends; larger T takes one kernel per step. */
+ * before its predecessor ends. Larger T takes the tensor-core path: the routing chain (router,
+ * top-k, permutation, activation operand) runs on the handle's own stream, forked from and joined
+ * back into `stream` with events (so graph capture of `stream` captures it too), while the shared
+ * expert runs on `stream`; then the routed gate|up and down grouped GEMMs and the combine. */
 flint_status flint_moe_forward(flint_moe_t h, const void* x, int T, void* y, void* stream);
 
 /* As flint_moe_forward, with x_host and y_host in host memory (pinned memory gives asynchronous
