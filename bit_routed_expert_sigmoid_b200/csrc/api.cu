@@ -18,6 +18,7 @@ struct flint_moe_ctx {
   size_t ws_bytes;
   // workspace carve-up
   float* logits;
+  float* logits_part;
   int* ids;
   float* wts;
   int* counts;
@@ -50,7 +51,7 @@ struct flint_moe_ctx {
   CUtensorMap tm_pf_sh_gu, tm_pf_sh_dn;    // prefill: shared-expert weights, 64 x 128 bf16 boxes
   CUtensorMap tm_pf_router;                // prefill: router rows [E][H], 64 x 128 bf16 boxes
   CUtensorMap tm_pf_hs_hi, tm_pf_hs_lo;    // prefill: shared-expert hidden pair [t_max][Is]
-  CUtensorMap tm_pf_xg, tm_pf_hq;          // prefill: routed activation rows (fp16, 64 x 64 boxes)
+  CUtensorMap tm_pf_xg, tm_pf_hq;          // prefill: routed activation rows (fp16, 64 x 16 boxes)
   // instrumentation (caller-owned cudaEvent_t handles)
   cudaEvent_t events[32];
   int n_events;
@@ -131,8 +132,8 @@ bool encode_bf16_tiles(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-bool encode_f16_rows64(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
-  return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rows, cols * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+bool encode_f16_rows16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rows, cols * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 bool encode_code_tiles(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes) {
@@ -158,6 +159,7 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
     return p;
   };
   char* p_logits = take(T * E * 4);
+  char* p_lpart = take(kRouterSplit * T * E * 4);
   char* p_ids = take(P * 4);
   char* p_wts = take(P * 4);
   char* p_counts = take(E * 4);
@@ -185,6 +187,7 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
   char* p_ys2 = take(T * kH * 2);
   if (h) {
     h->logits = reinterpret_cast<float*>(p_logits);
+    h->logits_part = reinterpret_cast<float*>(p_lpart);
     h->ids = reinterpret_cast<int*>(p_ids);
     h->wts = reinterpret_cast<float*>(p_wts);
     h->counts = reinterpret_cast<int*>(p_counts);
@@ -309,7 +312,7 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   pp.T = T;
   pp.top_k = K;
   pp.E = E;
-  pp.logits = h->logits;
+  pp.logits = h->logits_part;
   pp.offsets = h->offsets;
   pp.perm = h->perm;
   pp.hq = h->hq;
@@ -335,7 +338,7 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   pp.tm_b = tm_x;
   FLINT_TRY(launch_prefill_shared(pp, kPhaseRouter, h->n_sm, rs));
   FLINT_TRY(m.mark());
-  FLINT_TRY(launch_topk(h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, rs));
+  FLINT_TRY(launch_topk(h->logits_part, kRouterSplit, h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, rs));
   FLINT_TRY(m.mark());
   FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, c.flags, h->err, rs));
   FLINT_TRY(m.mark());
@@ -427,8 +430,8 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
       !encode_bf16_tiles(&h->tm_pf_router, w.router_w, cfg->n_experts, kH) ||
       !encode_bf16_tiles(&h->tm_pf_hs_hi, h->hs_hi, cfg->t_max, kIs) ||
       !encode_bf16_tiles(&h->tm_pf_hs_lo, h->hs_lo, cfg->t_max, kIs) ||
-      !encode_f16_rows64(&h->tm_pf_xg, h->xg, static_cast<uint64_t>(cfg->t_max) * cfg->top_k, kH) ||
-      !encode_f16_rows64(&h->tm_pf_hq, h->hq, static_cast<uint64_t>(cfg->t_max) * cfg->top_k, kI) ||
+      !encode_f16_rows16(&h->tm_pf_xg, h->xg, static_cast<uint64_t>(cfg->t_max) * cfg->top_k, kH) ||
+      !encode_f16_rows16(&h->tm_pf_hq, h->hq, static_cast<uint64_t>(cfg->t_max) * cfg->top_k, kI) ||
       !create_side_stream(h)) {
     delete h;
     return FLINT_ERR_CUDA;

@@ -69,15 +69,16 @@ cudaError_t launch_decode(const DecodeParams& p, int n_sm, cudaStream_t s, cudaE
 
 // ---- prefill path (T > kDecodeMaxT): tcgen05 grouped GEMMs ----
 enum PfPhase : int { kPhaseGateUp = 0, kPhaseDown = 1, kPhaseRouter = 2 };
+constexpr int kRouterSplit = 4;            // K slices of the prefill router (partial logits summed by top-k)
 
 struct PrefillParams {
   CUtensorMap tm_codes;           // routed: codes as 32-bit words [rows][K/8], box 16 words x 128 rows, 64-byte swizzle
-  CUtensorMap tm_act;             // routed: fp16 activation rows (xg or hq), box 64 x 64 rows, 128-byte swizzle
+  CUtensorMap tm_act;             // routed: fp16 activation rows (xg or hq), box 64 x 16 rows, 128-byte swizzle
   CUtensorMap tm_a;               // dense phases: bf16 weights (shared expert, router), box 64 x 128 rows, 128-byte swizzle
   CUtensorMap tm_b;               // shared: bf16 activations (x, or hs_hi), box 64 x 128 rows, 128-byte swizzle
   CUtensorMap tm_b2;              // shared down: hs_lo
   int T, top_k, E;
-  float* logits;                  // router phase output [T][E]
+  float* logits;                  // router phase output: partial logits [kRouterSplit][T][E]
   const int* offsets;             // [E+1]
   const int* perm;                // [P]
   const void* scales;             // int4 bf16 / nvfp4 e4m3, layout of the codes
@@ -94,8 +95,10 @@ cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, in
 cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, cudaStream_t s);
 
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* wr, int T, int E, float* logits, cudaStream_t s);
-cudaError_t launch_topk(const float* logits, int T, int E, int K, float floor_, int* ids, float* wts, unsigned flags,
-                        unsigned* err, cudaStream_t s);
+// logits: `nsplit` partial logit arrays [nsplit][T][E], summed in slice order; the sums are also
+// written to logits_out [T][E] when it is not null.
+cudaError_t launch_topk(const float* logits, int nsplit, float* logits_out, int T, int E, int K, float floor_, int* ids,
+                        float* wts, unsigned flags, unsigned* err, cudaStream_t s);
 cudaError_t launch_permute(const int* ids, int T, int K, int E, int* counts, int* offsets, int* perm, int* inv,
                            unsigned flags, unsigned* err, cudaStream_t s);
 cudaError_t launch_xg(const uint16_t* x, int T, int K, const int* inv, int rotate, __half* xg, cudaStream_t s);

@@ -69,7 +69,7 @@ extern "C" flint_status flint_moe_route_noalloc(const void* x, const void* route
                                   n_experts, logits, s) != cudaSuccess)
     return FLINT_ERR_CUDA;
   // flags = 0: the debug checks (which would write status_word) stay off
-  if (flint::launch_topk(logits, T, n_experts, top_k, norm_floor, ids, w, 0u, status_word, s) != cudaSuccess)
+  if (flint::launch_topk(logits, 1, nullptr, T, n_experts, top_k, norm_floor, ids, w, 0u, status_word, s) != cudaSuccess)
     return FLINT_ERR_CUDA;
   return FLINT_OK;
 }

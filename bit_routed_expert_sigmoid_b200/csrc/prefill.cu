@@ -7,7 +7,7 @@
 // and [256r+128, 256r+256). One persistent CTA per SM walks the tiles; its warps specialise:
 //   warp 0       TMA copies of the 4-bit codes, 128 K per stage, into a shared-memory ring
 //   warp 3       TMA copies of the chunk's activation rows (fp16, stored per permuted row so that
-//                an expert's rows are contiguous; 128-byte swizzled K-major) into a second ring
+//                an expert's rows are contiguous; 128-byte swizzled K-major, 16-row boxes) into a ring
 //   warps 4-11   dequantisation: a thread owns one weight row of one block, turns its 128 codes of
 //                the stage into exact fp16 (int4: code x bf16 group scale; NVFP4: E2M1 x E4M3) and
 //                writes them to tensor memory with tcgen05.st, where the MMA reads its A operand.
@@ -354,12 +354,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_c
       for (int j = max(it - kPfDA, 0); j < it; ++j) pf_wait(&bb.code_full[j % kPfDA], (j / kPfDA) & 1, abort, p.err);
     }
   } else if (warp == 3) {
-    // ---- activations: the chunk's rows are contiguous (permuted order), two TMA boxes of 64 rows x
-    // 64 fp16 (128-byte swizzled) per stage; rows past the chunk only feed unused accumulator columns
+    // ---- activations: the chunk's rows are contiguous (permuted order); per stage and 64-K half, the
+    // chunk's rows rounded up to 16 in boxes of 16 rows x 64 fp16 (128-byte swizzled, 2 KB each);
+    // rows past the chunk only feed unused accumulator columns
     if (lane == 0) {
       int it = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
         const PfTile tl = tile_at(tt, t);
+        const int nbox = (tl.n + 15) >> 4;
         bool ok = true;
         for (int s = 0; s < G::S; ++s, ++it) {
           const int slot = it % kPfDB;
@@ -368,9 +370,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_c
             break;
           }
           uint8_t* st = sm + kOffAct + slot * kPfActStage;
-          mbar_arrive_expect_tx(&bb.act_full[slot], kPfActStage);
-          tma_2d(st, &p.tm_act, s * kPfSK, tl.row0, &bb.act_full[slot]);
-          tma_2d(st + kPfActChunk, &p.tm_act, s * kPfSK + 64, tl.row0, &bb.act_full[slot]);
+          mbar_arrive_expect_tx(&bb.act_full[slot], nbox * 2 * 2048);
+          for (int q = 0; q < nbox; ++q) {
+            tma_2d(st + q * 2048, &p.tm_act, s * kPfSK, tl.row0 + 16 * q, &bb.act_full[slot]);
+            tma_2d(st + kPfActChunk + q * 2048, &p.tm_act, s * kPfSK + 64, tl.row0 + 16 * q, &bb.act_full[slot]);
+          }
         }
         if (!ok) break;
       }
@@ -600,10 +604,11 @@ struct ShGeom<kPhaseDown> {
   static constexpr int S = kIs / 64, RP = kH / 256, NB = 2, D = 3;
   __device__ static int row(int rp, int b) { return rp * 256 + b * 128; }
 };
-// router logits: A = router rows (experts rp*256 + b*128 ..), B = x; RP = ceil(E / 256) at run time
+// router logits: A = router rows (experts rp*256 + b*128 ..), B = x; RP = ceil(E / 256) at run time;
+// K is split in kRouterSplit slices (one per tile) whose partial logits the top-k kernel sums
 template <>
 struct ShGeom<kPhaseRouter> {
-  static constexpr int S = kH / 64, RP = 0, NB = 1, D = 4;
+  static constexpr int S = kH / 64 / kRouterSplit, RP = 0, NB = 1, D = 4;
   __device__ static int row(int rp, int b) { return rp * 256 + b * 128; }
 };
 
@@ -639,7 +644,8 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shared_kernel(const __grid_c
   volatile int* abort = &bb.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nch = (p.T + 127) / 128;
-  const int total = (PHASE == kPhaseRouter ? (p.E + 255) / 256 : G::RP) * nch;
+  const int nrp = PHASE == kPhaseRouter ? (p.E + 255) / 256 : G::RP;
+  const int total = nrp * nch * (PHASE == kPhaseRouter ? kRouterSplit : 1);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < G::D; ++i) {
@@ -667,16 +673,18 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shared_kernel(const __grid_c
     if (lane == 0) {
       int it = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-        const int rp = t / nch, c0 = (t - rp * nch) * 128;
+        const int ks = t / (nrp * nch), tr = t - ks * (nrp * nch);   // K slice (router only)
+        const int rp = tr / nch, c0 = (tr - rp * nch) * 128;
         for (int s = 0; s < G::S; ++s, ++it) {
           const int slot = it % G::D;
           if (it >= G::D && !pf_wait(&bb.empty[slot], ((it / G::D) - 1) & 1, abort, p.err)) break;
           uint8_t* st = sm + slot * L::kStage;
+          const int kx = (ks * G::S + s) * 64;
           mbar_arrive_expect_tx(&bb.full[slot], L::kStage);
-          tma_2d(st, &p.tm_a, s * 64, G::row(rp, 0), &bb.full[slot]);
-          tma_2d(st + kShBox, &p.tm_a, s * 64, G::row(rp, 1), &bb.full[slot]);
-          tma_2d(st + 2 * kShBox, &p.tm_b, s * 64, c0, &bb.full[slot]);
-          if constexpr (G::NB == 2) tma_2d(st + 3 * kShBox, &p.tm_b2, s * 64, c0, &bb.full[slot]);
+          tma_2d(st, &p.tm_a, kx, G::row(rp, 0), &bb.full[slot]);
+          tma_2d(st + kShBox, &p.tm_a, kx, G::row(rp, 1), &bb.full[slot]);
+          tma_2d(st + 2 * kShBox, &p.tm_b, kx, c0, &bb.full[slot]);
+          if constexpr (G::NB == 2) tma_2d(st + 3 * kShBox, &p.tm_b2, kx, c0, &bb.full[slot]);
         }
       }
       for (int j = max(it - G::D, 0); j < it; ++j) pf_wait(&bb.full[j % G::D], (j / G::D) & 1, abort, p.err);
@@ -716,8 +724,10 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shared_kernel(const __grid_c
     const int q = warp & 3, r = 32 * q + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
     for (int t = blockIdx.x, ti = 0; t < total; t += gridDim.x, ++ti) {
-      const int rp = t / nch, c0 = (t - rp * nch) * 128;
+      const int ks = t / (nrp * nch), tr = t - ks * (nrp * nch);
+      const int rp = tr / nch, c0 = (tr - rp * nch) * 128;
       const int n = min(128, p.T - c0);
+      float* lg = p.logits + static_cast<size_t>(ks) * p.T * p.E;
       if (!pf_wait_all(&bb.acc_full[0], ti & 1, abort, p.err) || !pf_wait_all(&bb.acc_full[1], ti & 1, abort, p.err))
         break;
       tc_fence_after();
@@ -732,8 +742,8 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shared_kernel(const __grid_c
           const size_t tok = static_cast<size_t>(c0 + j0 + c);
           if constexpr (PHASE == kPhaseRouter) {
             const int e0 = rp * 256 + r;
-            if (e0 < p.E) p.logits[tok * p.E + e0] = __uint_as_float(d0[c]);
-            if (e0 + 128 < p.E) p.logits[tok * p.E + e0 + 128] = __uint_as_float(d1[c]);
+            if (e0 < p.E) lg[tok * p.E + e0] = __uint_as_float(d0[c]);
+            if (e0 + 128 < p.E) lg[tok * p.E + e0 + 128] = __uint_as_float(d1[c]);
           } else if constexpr (PHASE == kPhaseGateUp) {
             const float hs = silu_fast(__uint_as_float(d0[c])) * __uint_as_float(d1[c]);
             const uint16_t hi = f32_to_bf16_bits(hs);
@@ -834,7 +844,7 @@ cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, c
   }
   const int rp = phase == kPhaseGateUp ? ShGeom<kPhaseGateUp>::RP
                  : phase == kPhaseDown ? ShGeom<kPhaseDown>::RP
-                                       : (p.E + 255) / 256;
+                                       : (p.E + 255) / 256 * kRouterSplit;
   const int tiles = rp * ((p.T + 127) / 128);
   const int grid = tiles < n_sm ? tiles : n_sm;
   if (phase == kPhaseGateUp) pf_shared_kernel<kPhaseGateUp><<<grid, kShThreads, sh_smem<kPhaseGateUp>(), s>>>(p);

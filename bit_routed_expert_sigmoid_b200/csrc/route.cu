@@ -61,7 +61,9 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
 // would create. Ties go to the lower expert id. The chosen slots are listed by ascending expert
 // id, and w_k = s_k / max(sum of the chosen s, floor) with s = sigmoid(logit) (the SelectedSumFloor
 // policy, same issue, host-policy comment). The sum runs in slot order.
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int K,
+template <int NS>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
+                                                   float* __restrict__ logits_out, int T, int E, int K,
                                                    float floor_, int* __restrict__ ids, float* __restrict__ wts,
                                                    unsigned flags, unsigned* __restrict__ err) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -70,7 +72,22 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   const int per = E >> 5;          // logits per lane (E is a multiple of 32, at most 256)
   float v[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) v[j] = (j < per) ? logits[static_cast<size_t>(t) * E + lane + 32 * j] : -INFINITY;
+  for (int j = 0; j < 8; ++j) {
+    float part[NS];
+#pragma unroll
+    for (int q = 0; q < NS; ++q)
+      part[q] = (j < per) ? __ldg(logits + static_cast<size_t>(q) * T * E + static_cast<size_t>(t) * E + lane + 32 * j)
+                          : 0.f;
+    float a = part[0];
+#pragma unroll
+    for (int q = 1; q < NS; ++q) a += part[q];     // slice order
+    v[j] = (j < per) ? a : -INFINITY;
+  }
+  if (logits_out) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j < per) logits_out[static_cast<size_t>(t) * E + lane + 32 * j] = v[j];
+  }
   unsigned taken = 0;              // bit j: element lane+32j already chosen
   int my_id = 0x7FFFFFFF;          // lane k < K: the k-th pick
   float my_l = 0.f;
@@ -122,7 +139,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 }
 
 // ---------------------------------------------------------------------------------------------
-// Expert-major permutation of the (token, slot) pairs: one CTA per expert e.
+// Expert-major permutation of the (token, slot) pairs: one CTA per two experts.
 // counts[e] = number of pairs routed to e; offsets = exclusive prefix (E+1 entries);
 // position p in [offsets[e], offsets[e+1]) lists the pairs of expert e by ascending token:
 // perm[p] = t*K+k and inv[t*K+k] = p. Every CTA reads all P = T*K expert ids (L2-resident):
@@ -133,6 +150,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 constexpr int kPermThreads = 1024;
 constexpr int kPermWarps = kPermThreads / 32;
 constexpr int kPermChunk = 16;                   // ids a thread holds in registers per round
+constexpr int kPermExperts = 2;                  // experts per CTA
 
 __device__ __forceinline__ int clamp_id(int v, int E) { return (v < 0 || v >= E) ? 0 : v; }
 
@@ -172,7 +190,6 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __rest
                                                                unsigned flags, unsigned* __restrict__ err) {
   __shared__ int w_sum[kPermWarps], w_base[kPermWarps];
   __shared__ int s_total;
-  const int e = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int kRound = kPermThreads * kPermChunk;
   // warp-order exclusive scan of one value per thread over the CTA; returns the exclusive prefix and
@@ -201,42 +218,45 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __rest
     __syncthreads();
     return w_base[warp] + incl - x;
   };
-  // pass 1: pairs routed below e (the offset of e)
+  // the CTA's experts share the ids it loads (all of them in registers when P fits one round)
   int v[kPermChunk];
-  int lt = 0, eq_unused = 0;
-  bool bad = false;
-  for (int r0 = 0; r0 < P; r0 += kRound) {
-    const int i0 = r0 + kPermChunk * tid;
-    load_ids16(v, ids, i0, P);
-    count_ids(v, min(max(P - i0, 0), kPermChunk), e, E, lt, eq_unused, bad);
-  }
-  if (bad && (flags & 1u) && e == 0) atomicOr(err, kErrBadId);
-  block_scan(lt);
-  const int off = s_total;
-  // pass 2: the pairs of e in pair order at off, off + 1, ...
-  int run = 0;
-  for (int r0 = 0; r0 < P; r0 += kRound) {
-    const int i0 = r0 + kPermChunk * tid;
-    const int nv = min(max(P - i0, 0), kPermChunk);
-    if (P > kRound) load_ids16(v, ids, i0, P);     // one round: the ids are still in registers
-    int l2 = 0, eq = 0;
-    bool b2 = false;
-    count_ids(v, nv, e, E, l2, eq, b2);
-    int pos = off + run + block_scan(eq);
-    run += s_total;
+  for (int e = blockIdx.x * kPermExperts; e < min(E, blockIdx.x * kPermExperts + kPermExperts); ++e) {
+    // pass 1: pairs routed below e (the offset of e)
+    int lt = 0, eq_unused = 0;
+    bool bad = false;
+    for (int r0 = 0; r0 < P; r0 += kRound) {
+      const int i0 = r0 + kPermChunk * tid;
+      if (P > kRound || e == blockIdx.x * kPermExperts) load_ids16(v, ids, i0, P);
+      count_ids(v, min(max(P - i0, 0), kPermChunk), e, E, lt, eq_unused, bad);
+    }
+    if (bad && (flags & 1u) && e == 0) atomicOr(err, kErrBadId);
+    block_scan(lt);
+    const int off = s_total;
+    // pass 2: the pairs of e in pair order at off, off + 1, ...
+    int run = 0;
+    for (int r0 = 0; r0 < P; r0 += kRound) {
+      const int i0 = r0 + kPermChunk * tid;
+      const int nv = min(max(P - i0, 0), kPermChunk);
+      if (P > kRound) load_ids16(v, ids, i0, P);   // one round: the ids are still in registers
+      int l2 = 0, eq = 0;
+      bool b2 = false;
+      count_ids(v, nv, e, E, l2, eq, b2);
+      int pos = off + run + block_scan(eq);
+      run += s_total;
 #pragma unroll
-    for (int j = 0; j < kPermChunk; ++j) {
-      if (j < nv && clamp_id(v[j], E) == e) {
-        perm[pos] = i0 + j;
-        inv[i0 + j] = pos;
-        ++pos;
+      for (int j = 0; j < kPermChunk; ++j) {
+        if (j < nv && clamp_id(v[j], E) == e) {
+          perm[pos] = i0 + j;
+          inv[i0 + j] = pos;
+          ++pos;
+        }
       }
     }
-  }
-  if (tid == 0) {
-    counts[e] = run;
-    offsets[e] = off;
-    if (e == E - 1) offsets[E] = off + run;
+    if (tid == 0) {
+      counts[e] = run;
+      offsets[e] = off;
+      if (e == E - 1) offsets[E] = off + run;
+    }
   }
 }
 
@@ -272,15 +292,21 @@ cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* wr, int T, i
   return cudaGetLastError();
 }
 
-cudaError_t launch_topk(const float* logits, int T, int E, int K, float floor_, int* ids, float* wts, unsigned flags,
-                        unsigned* err, cudaStream_t s) {
-  topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, T, E, K, floor_, ids, wts, flags, err);
+cudaError_t launch_topk(const float* logits, int nsplit, float* logits_out, int T, int E, int K, float floor_, int* ids,
+                        float* wts, unsigned flags, unsigned* err, cudaStream_t s) {
+  if (nsplit == kRouterSplit)
+    topk_kernel<kRouterSplit><<<(T + 7) / 8, 256, 0, s>>>(logits, logits_out, T, E, K, floor_, ids, wts, flags, err);
+  else if (nsplit == 1)
+    topk_kernel<1><<<(T + 7) / 8, 256, 0, s>>>(logits, logits_out, T, E, K, floor_, ids, wts, flags, err);
+  else
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
 cudaError_t launch_permute(const int* ids, int T, int K, int E, int* counts, int* offsets, int* perm, int* inv,
                            unsigned flags, unsigned* err, cudaStream_t s) {
-  permute_kernel<<<E, kPermThreads, 0, s>>>(ids, T * K, E, counts, offsets, perm, inv, flags, err);
+  permute_kernel<<<(E + kPermExperts - 1) / kPermExperts, kPermThreads, 0, s>>>(ids, T * K, E, counts, offsets, perm, inv,
+                                                                                  flags, err);
   return cudaGetLastError();
 }
 
