@@ -58,24 +58,26 @@ constexpr uint32_t kColA = 256;
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
+// Warp-wide MMA and commit: every lane of the warp executes the call with the same operands (so they can stay
+// in uniform registers) and one elected lane issues the instruction.
+__device__ __forceinline__ void tc_commit_w(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+      "@p tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
 }
 
-// D[tmem d] (+)= A[tmem a] * B[smem desc]^T
-__device__ __forceinline__ void tc_mma_ta(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+__device__ __forceinline__ void tc_mma_ta_w(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
       "r"(a), "l"(bdesc), "r"(idesc), "r"(acc));
 }
 
-// D[tmem d] (+)= A[smem desc] * B[smem desc]^T
-__device__ __forceinline__ void tc_mma_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+__device__ __forceinline__ void tc_mma_ss_w(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc));
 }
 
@@ -381,41 +383,39 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_c
       for (int j = max(it - kPfDB, 0); j < it; ++j) pf_wait(&bb.act_full[j % kPfDB], (j / kPfDB) & 1, abort, p.err);
     }
   } else if (warp == 1 || warp == 2) {
-    // ---- MMA issue, one thread per block
+    // ---- MMA issue, one warp per block (uniform control flow; an elected lane issues)
     const int b = warp - 1;
-    if (lane == 0) {
-      int it = 0, ti = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++ti) {
-        const PfTile tl = tile_at(tt, t);
-        const int npad = (tl.n + 15) & ~15;
-        const uint32_t idesc = idesc_m128(npad, false);
-        const int as = ti & 1;
-        const uint32_t d = tmem + as * kColSlot + b * kColD1;
-        if (ti >= 2 && !pf_wait(&bb.acc_empty[as], ((ti >> 1) - 1) & 1, abort, p.err)) break;
-        tc_fence_after();
-        for (int s = 0; s < G::S; ++s, ++it) {
-          const int ts = it & 1, bs = it % kPfDB;
-          if (!pf_wait(&bb.a_full[ts][b], (it >> 1) & 1, abort, p.err) ||
-              !pf_wait(&bb.act_full[bs], (it / kPfDB) & 1, abort, p.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a0 = tmem + kColA + ts * 128 + b * 64;
-          const uint32_t b0 = smem_u32(sm + kOffAct + bs * kPfActStage);
-#pragma unroll
-          for (int ks = 0; ks < kPfSK / 16; ++ks)
-            tc_mma_ta(d, a0 + ks * 8, sdesc_sw128(b0 + (ks >> 2) * kPfActChunk + (ks & 3) * 32), idesc,
-                      (s | ks) ? 1u : 0u);
-          tc_commit(&bb.a_empty[ts][b]);
-          tc_commit(&bb.act_empty[bs]);
+    int it = 0, ti = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++ti) {
+      const PfTile tl = tile_at(tt, t);
+      const int npad = (tl.n + 15) & ~15;
+      const uint32_t idesc = idesc_m128(npad, false);
+      const int as = ti & 1;
+      const uint32_t d = tmem + as * kColSlot + b * kColD1;
+      if (ti >= 2 && !pf_wait_all(&bb.acc_empty[as], ((ti >> 1) - 1) & 1, abort, p.err)) break;
+      tc_fence_after();
+      for (int s = 0; s < G::S; ++s, ++it) {
+        const int ts = it & 1, bs = it % kPfDB;
+        if (!pf_wait_all(&bb.a_full[ts][b], (it >> 1) & 1, abort, p.err) ||
+            !pf_wait_all(&bb.act_full[bs], (it / kPfDB) & 1, abort, p.err)) {
+          ok = false;
+          break;
         }
-        if (ok) tc_commit(&bb.acc_full[as][b]);
+        tc_fence_after();
+        const uint32_t a0 = tmem + kColA + ts * 128 + b * 64;
+        const uint32_t b0 = smem_u32(sm + kOffAct + bs * kPfActStage);
+#pragma unroll
+        for (int ks = 0; ks < kPfSK / 16; ++ks)
+          tc_mma_ta_w(d, a0 + ks * 8, sdesc_sw128(b0 + (ks >> 2) * kPfActChunk + (ks & 3) * 32), idesc,
+                      (s | ks) ? 1u : 0u);
+        tc_commit_w(&bb.a_empty[ts][b]);
+        tc_commit_w(&bb.act_empty[bs]);
       }
-      tc_commit(&bb.done[b]);                       // every MMA of this thread has completed
-      pf_wait(&bb.done[b], 0, abort, p.err);
+      if (ok) tc_commit_w(&bb.acc_full[as][b]);
     }
+    tc_commit_w(&bb.done[b]);                     // every MMA of this warp has completed
+    pf_wait_all(&bb.done[b], 0, abort, p.err);
   } else if (warp >= 4 && warp < 12) {
     // ---- dequantisation into tensor memory
     const int b = (warp - 4) >> 2, q = warp & 3;
@@ -690,36 +690,34 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shared_kernel(const __grid_c
       for (int j = max(it - G::D, 0); j < it; ++j) pf_wait(&bb.full[j % G::D], (j / G::D) & 1, abort, p.err);
     }
   } else if (warp == 1 || warp == 2) {
-    const int b = warp - 1;
-    if (lane == 0) {
-      int it = 0;
-      bool ok = true;
-      const uint32_t idesc = idesc_m128(128, true);
-      const uint32_t d = tmem + b * kShColD1;
-      for (int t = blockIdx.x, ti = 0; t < total && ok; t += gridDim.x, ++ti) {
-        if (ti > 0 && !pf_wait(&bb.acc_empty[b], (ti - 1) & 1, abort, p.err)) break;   // D drained
-        tc_fence_after();
-        for (int s = 0; s < G::S; ++s, ++it) {
-          const int slot = it % G::D;
-          if (!pf_wait(&bb.full[slot], (it / G::D) & 1, abort, p.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t st = smem_u32(sm + slot * L::kStage);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = sdesc_sw128(st + b * kShBox + ks * 32);
-            tc_mma_ss(d, ad, sdesc_sw128(st + 2 * kShBox + ks * 32), idesc, (s | ks) ? 1u : 0u);
-            if constexpr (G::NB == 2) tc_mma_ss(d, ad, sdesc_sw128(st + 3 * kShBox + ks * 32), idesc, 1u);
-          }
-          tc_commit(&bb.empty[slot]);
+    const int b = warp - 1;                       // one warp per block; an elected lane issues
+    int it = 0;
+    bool ok = true;
+    const uint32_t idesc = idesc_m128(128, true);
+    const uint32_t d = tmem + b * kShColD1;
+    for (int t = blockIdx.x, ti = 0; t < total && ok; t += gridDim.x, ++ti) {
+      if (ti > 0 && !pf_wait_all(&bb.acc_empty[b], (ti - 1) & 1, abort, p.err)) break;   // D drained
+      tc_fence_after();
+      for (int s = 0; s < G::S; ++s, ++it) {
+        const int slot = it % G::D;
+        if (!pf_wait_all(&bb.full[slot], (it / G::D) & 1, abort, p.err)) {
+          ok = false;
+          break;
         }
-        if (ok) tc_commit(&bb.acc_full[b]);
+        tc_fence_after();
+        const uint32_t st = smem_u32(sm + slot * L::kStage);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ad = sdesc_sw128(st + b * kShBox + ks * 32);
+          tc_mma_ss_w(d, ad, sdesc_sw128(st + 2 * kShBox + ks * 32), idesc, (s | ks) ? 1u : 0u);
+          if constexpr (G::NB == 2) tc_mma_ss_w(d, ad, sdesc_sw128(st + 3 * kShBox + ks * 32), idesc, 1u);
+        }
+        tc_commit_w(&bb.empty[slot]);
       }
-      tc_commit(&bb.fin[b]);                        // every MMA of this thread has completed
-      pf_wait(&bb.fin[b], 0, abort, p.err);
+      if (ok) tc_commit_w(&bb.acc_full[b]);
     }
+    tc_commit_w(&bb.fin[b]);                      // every MMA of this warp has completed
+    pf_wait_all(&bb.fin[b], 0, abort, p.err);
   } else if (warp >= 4) {
     const int q = warp & 3, r = 32 * q + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
