@@ -76,6 +76,8 @@ def _load():
         "flint_moe_stage_count": (I, [V, I]),
         "flint_moe_stage_name": (ctypes.c_char_p, [V, I, I]),
         "flint_moe_route_noalloc": (I, [V, V, I, I, I, ctypes.c_float, V, V, V]),
+        "flint_residual_rmsnorm": (I, [V, V, I, ctypes.c_float, V, V]),
+        "flint_moe_stack_forward": (I, [P(V), I, V, I, ctypes.c_float, V, V, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -132,6 +134,18 @@ def flint_moe_error_word(h: int) -> int:
     out = ctypes.c_uint(0)
     _check(_lib.flint_moe_error_word(ctypes.c_void_p(h), ctypes.byref(out)), "flint_moe_error_word")
     return int(out.value)
+
+
+def flint_residual_rmsnorm(x: int, y: int, T: int, eps: float, z: int, stream: int = 0) -> None:
+    _check(_lib.flint_residual_rmsnorm(ctypes.c_void_p(x), ctypes.c_void_p(y), int(T), ctypes.c_float(eps),
+                                       ctypes.c_void_p(z), ctypes.c_void_p(stream)), "flint_residual_rmsnorm")
+
+
+def flint_moe_stack_forward(handles, x: int, T: int, eps: float, z: int, y: int, stream: int = 0) -> None:
+    arr = (ctypes.c_void_p * len(handles))(*handles)
+    _check(_lib.flint_moe_stack_forward(arr, len(handles), ctypes.c_void_p(x), int(T), ctypes.c_float(eps),
+                                        ctypes.c_void_p(z), ctypes.c_void_p(y), ctypes.c_void_p(stream)),
+           "flint_moe_stack_forward")
 
 
 def flint_moe_destroy(h: int) -> None:

@@ -466,6 +466,35 @@ flint_status flint_moe_forward_host(flint_moe_t h, const void* x_host, int T, vo
   return FLINT_OK;
 }
 
+flint_status flint_residual_rmsnorm(float* x, const void* y, int T, float eps, void* z, void* stream) {
+  if (T < 0 || !(eps > 0.f)) return FLINT_ERR_INVALID_ARG;
+  if (T == 0) return FLINT_OK;
+  if (!aligned16(x) || (y && !aligned16(y)) || (z && !aligned16(z))) return FLINT_ERR_INVALID_ARG;
+  FLINT_TRY(launch_residual_rmsnorm(x, static_cast<const uint16_t*>(y), T, eps, static_cast<uint16_t*>(z),
+                                    static_cast<cudaStream_t>(stream)));
+  return FLINT_OK;
+}
+
+flint_status flint_moe_stack_forward(const flint_moe_t* layers, int n_layers, float* x, int T, float eps, void* z,
+                                     void* y, void* stream) {
+  if (!layers || n_layers < 1 || T < 0 || !(eps > 0.f)) return FLINT_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l)
+    if (!layers[l] || T > layers[l]->cfg.t_max) return FLINT_ERR_INVALID_ARG;
+  if (T == 0) return FLINT_OK;
+  if (!aligned16(x) || !aligned16(z) || !aligned16(y) || z == y) return FLINT_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* zb = static_cast<uint16_t*>(z);
+  uint16_t* yb = static_cast<uint16_t*>(y);
+  for (int l = 0; l < n_layers; ++l) {
+    FLINT_TRY(launch_residual_rmsnorm(x, l ? yb : nullptr, T, eps, zb, s));
+    flint_status st = run_forward(layers[l], zb, T, yb, s);
+    if (st != FLINT_OK) return st;
+    layers[l]->last_T = T;
+  }
+  FLINT_TRY(launch_residual_rmsnorm(x, yb, T, eps, nullptr, s));
+  return FLINT_OK;
+}
+
 flint_status flint_moe_routing(flint_moe_t h, int* ids, float* w, int* offsets, int* perm, void* stream) {
   if (!h) return FLINT_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -94,6 +94,9 @@ struct PrefillParams {
 cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, int n_sm, cudaStream_t s);
 cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, cudaStream_t s);
 
+// Residual stream of a layer stack: x (f32 [T][H]) += y (bf16, when not null); then, when z is not
+// null, z = bf16(rmsnorm(x)) with eps.
+cudaError_t launch_residual_rmsnorm(float* x, const uint16_t* y, int T, float eps, uint16_t* z, cudaStream_t s);
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* wr, int T, int E, float* logits, cudaStream_t s);
 // logits: `nsplit` partial logit arrays [nsplit][T][E], summed in slice order; the sums are also
 // written to logits_out [T][E] when it is not null.

@@ -108,6 +108,34 @@ class FlintMoELayer:
             pass
 
 
+class FlintMoEStack:
+    """A stack of Flint MoE layers on one device, run on an fp32 residual stream:
+    for each layer, z = bf16(rmsnorm(x)); x += layer(z) (flint_moe_stack_forward)."""
+
+    def __init__(self, layers: list, t_max: int, *, eps: float = 1e-6, device="cuda", **kw):
+        self.device = torch.device(device)
+        self.eps = float(eps)
+        self.t_max = t_max
+        self.layers = [FlintMoELayer(L, t_max=t_max, device=device, **kw) for L in layers]
+        self.z = torch.empty((t_max, H), dtype=torch.bfloat16, device=self.device)
+        self.y = torch.empty((t_max, H), dtype=torch.bfloat16, device=self.device)
+
+    def weight_bytes(self) -> int:
+        return sum(layer.weight_bytes() for layer in self.layers)
+
+    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        """x: [T][H] fp32 residual on the device, updated in place and returned."""
+        T = x.shape[0]
+        s = (stream or torch.cuda.current_stream(self.device)).cuda_stream
+        B.flint_moe_stack_forward([layer.handle for layer in self.layers], x.data_ptr(), T, self.eps,
+                                  self.z.data_ptr(), self.y.data_ptr(), s)
+        return x
+
+    def close(self) -> None:
+        for layer in self.layers:
+            layer.close()
+
+
 def x_to_device(x_bits: np.ndarray, device="cuda") -> torch.Tensor:
     """bf16 bit patterns [T][H] (uint16) -> device bf16 tensor."""
     return torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).to(device).view(torch.bfloat16)

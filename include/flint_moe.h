@@ -127,6 +127,20 @@ flint_status flint_moe_forward(flint_moe_t h, const void* x, int T, void* y, voi
  * The caller synchronises the stream before reading y_host. */
 flint_status flint_moe_forward_host(flint_moe_t h, const void* x_host, int T, void* y_host, void* stream);
 
+/* Residual stream step of a stack of layers (the model's routed blocks with their weightless
+ * RMSNorm; Aijuus/flint-w4exp, model summary): x f32 [T][H] (device, in/out) += y bf16 [T][H] when y is
+ * not NULL; then, when z is not NULL, z bf16 [T][H] = bf16( x / sqrt(mean_j x[t][j]^2 + eps) ) per token,
+ * the sum of squares reduced in a fixed order. One kernel, enqueued on `stream`. */
+flint_status flint_residual_rmsnorm(float* x, const void* y, int T, float eps, void* z, void* stream);
+
+/* n_layers layers in sequence on the residual x f32 [T][H] (device, in/out):
+ *   for each layer l: z = bf16(rmsnorm(x)); y = layer_l(z); x += y
+ * (the residual add of one layer is fused with the RMSNorm of the next). z and y are caller-owned
+ * bf16 [T][H] scratch buffers (distinct). The handles must not run forwards concurrently. Each
+ * layer's forward is the same launch sequence as flint_moe_forward; T <= every layer's t_max. */
+flint_status flint_moe_stack_forward(const flint_moe_t* layers, int n_layers, float* x, int T, float eps, void* z,
+                                     void* y, void* stream);
+
 /* Device-to-device copies of the last forward's routing, enqueued on `stream` (any pointer may be
  * NULL to skip it): ids int32 [T][top_k] and w f32 [T][top_k] in slot order (ascending expert id),
  * offsets int32 [E+1] (exclusive prefix of per-expert counts), perm int32 [T*top_k] (position p

@@ -313,3 +313,34 @@ def router_gap(L: dict, x_bits: np.ndarray, top_k: int = TOP_K) -> np.ndarray:
     x = bf16_to_f64(x_bits)
     s = np.sort(sigmoid(x @ bf16_to_f64(L["router_w"]).T), axis=1)[:, ::-1]
     return s[:, top_k - 1] - s[:, top_k]
+
+# ----------------------------------------------------------------------------------------------
+# stack of layers (the model's routed blocks in sequence)
+# ----------------------------------------------------------------------------------------------
+
+RMS_EPS = 1e-6
+
+
+def rmsnorm(x, eps: float = RMS_EPS) -> np.ndarray:
+    """Weightless RMSNorm of each row, in fp64: x / sqrt(mean(x^2) + eps).
+
+    The pages name the 47 routed blocks but not the norm between them; this reading takes the
+    plain RMSNorm with its weight folded into the next layer (no weight) and eps = 1e-6."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+
+
+def f64_to_bf16_bits(x) -> np.ndarray:
+    """Round fp64 values to bf16 (8 significant bits, round half to even); uint16 bit patterns."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                                  # x = m * 2^e, 0.5 <= |m| < 1
+    r = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)        # exact in fp64; a bf16 value, exact in f32
+    return (r.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def stack_step(L: dict, x_resid: np.ndarray, *, top_k: int = TOP_K, eps: float = RMS_EPS) -> dict:
+    """One layer of a stack on the fp64 residual x: z = bf16(rmsnorm(x)) (the layer's input format),
+    y = layer(z), x_next = x + y. Returns z (bf16 bits), y (fp64, unrounded) and x_next."""
+    z = f64_to_bf16_bits(rmsnorm(x_resid, eps))
+    y = moe_forward(L, z, top_k=top_k)["y"]
+    return {"z": z, "y": y, "x_next": np.asarray(x_resid, dtype=np.float64) + y}

@@ -316,3 +316,29 @@ def test_redraw_tables_leave_no_near_tie():
         L = S.make_layer(E, H=2048, I=128, Is=8)          # router rows do not depend on I / Is
         x = S.make_workload_x(2048 if E == 256 else 4096, E)
         assert R.router_gap(L, x).min() >= 1e-4
+
+
+def test_rmsnorm_closed_forms():
+    # a constant row c has mean square c^2: every element becomes c / sqrt(c^2 + eps)
+    eps = 1e-6
+    for c in (-3.0, 0.5, 7.25):
+        row = np.full((1, 2048), c)
+        np.testing.assert_allclose(R.rmsnorm(row, eps), c / math.sqrt(c * c + eps), rtol=1e-15)
+    # the two-element row (3, 4): mean square 12.5
+    np.testing.assert_allclose(R.rmsnorm(np.array([[3.0, 4.0]]), 0.0), [[3 / math.sqrt(12.5), 4 / math.sqrt(12.5)]])
+    # without eps the result has unit mean square and is invariant to positive scaling, odd in x
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((4, 2048))
+    z = R.rmsnorm(x, 0.0)
+    np.testing.assert_allclose(np.mean(z * z, axis=-1), 1.0, rtol=1e-12)
+    np.testing.assert_allclose(R.rmsnorm(37.5 * x, 0.0), z, rtol=1e-12)
+    np.testing.assert_allclose(R.rmsnorm(-x, 0.0), -z, rtol=1e-12)
+
+
+def test_f64_to_bf16_rounding_matches_torch():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(6)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-6, 6, 20000),
+                        [0.0, -0.0, 1.0, 1.00390625, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -9]])
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(R.f64_to_bf16_bits(x), ref)
