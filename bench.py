@@ -44,7 +44,11 @@ WORKLOADS = {
     "prefill_int4_skew": (256, "int4", 2048, True),
     "decode_nvfp4": (256, "nvfp4", 8, False),
     "prefill_nvfp4": (256, "nvfp4", 2048, False),
+    "stack47_int4": (256, "int4", 8, False),
 }
+# stacks: layers of the workload (layer l drawn with seed 1000 + l); T tokens decode through all of them
+STACK_LAYERS = {"stack47_int4": 47}
+STACK_EPS = 1e-6
 
 
 def parse_args():
@@ -431,6 +435,28 @@ def run_reference(args) -> dict:
     from bit_routed_expert_sigmoid_b200 import synthetic as S
     from oracle import flint_moe_ref as R
     E, fmt, T, skew = WORKLOADS[args.workload]
+    if args.workload in STACK_LAYERS:
+        # bounded sample: whole oracle stack steps on the first layers, the per-layer time scaled
+        n = STACK_LAYERS[args.workload]
+        x_bits = S.make_x(T, redraws=S.redraw_table(E))
+        xs, times = R.bf16_to_f64(x_bits), []
+        for l in range(max(1, min(args.steps, 3))):
+            L = S.make_layer(E, fmt, seed=1000 + l)
+            t1 = time.perf_counter()
+            xs = R.stack_step(L, xs, eps=STACK_EPS)["x_next"]
+            times.append(time.perf_counter() - t1)
+        per_layer = float(np.mean(times))
+        value = T / (per_layer * n)
+        sample = f"fp64 oracle stack step on the first {len(times)} of {n} layers, per-layer time scaled to {n}"
+        return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": 1,
+                "steps": len(times), "warmup": 0, "ms_per_step": round(per_layer * n * 1e3, 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": f"{args.workload}: {n} layers, E={E} top-6, H=2048, {fmt}, T={T}", "E": E,
+                           "T": T, "fmt": fmt, "layers": n},
+                "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": blas_threads(),
+                                 "kind": "oracle", "sample": sample},
+                "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
     L = S.make_layer(E, fmt, skew=skew)
     # bounded sample: decode steps run whole; a prefill step runs the first 64 tokens of the batch
     Ts = T if T <= 64 else 64
@@ -455,6 +481,136 @@ def run_reference(args) -> dict:
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_stack(args) -> dict:
+    """Decode of T tokens through a stack of independent seeded layers on the fp32 residual stream
+    (z = bf16(rmsnorm(x)); x += layer(z)); the weights (20 GB at 47 layers) never stay in L2."""
+    import torch
+
+    from bit_routed_expert_sigmoid_b200 import binding as B
+    from bit_routed_expert_sigmoid_b200 import synthetic as S
+    from bit_routed_expert_sigmoid_b200.layer import FlintMoEStack
+
+    E, fmt, T, skew = WORKLOADS[args.workload]
+    n = STACK_LAYERS[args.workload]
+    dev = "cuda:0"
+    torch.cuda.set_device(dev)
+    stack = FlintMoEStack((S.make_layer(E, fmt, seed=1000 + l) for l in range(n)), t_max=T, eps=STACK_EPS,
+                          device=dev)
+    x_bits = S.make_x(T, redraws=S.redraw_table(E))
+    x0 = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).float().to(dev)     # residual = input
+    x = x0.clone()
+    stream = torch.cuda.current_stream()
+
+    def timed_steps(fn, K):
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        for i in range(K):
+            starts[i].record(stream)
+            fn()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+    fwd = lambda: stack.forward(x)  # noqa: E731
+    for _ in range(args.warmup):
+        fwd()
+    torch.cuda.synchronize()
+    n_active = [int((torch.diff(layer.routing(T)["offsets"]) > 0).sum().item()) for layer in stack.layers]
+    clocks = ClockSampler(0)
+    clocks.start()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    step_ms = timed_steps(fwd, args.steps)
+    wall1 = time.perf_counter()
+    total_ms = float(sum(step_ms))
+    ms_per_step = total_ms / args.steps
+    value = T * args.steps / (total_ms / 1e3)
+    glue = (n + 1) * T * H * (4 + 4 + 2 + 2)          # residual read + write, y read, z write per boundary
+    ab = sum(algorithmic_bytes(E, fmt, T, a) for a in n_active) + glue
+
+    # gate|up of every layer, timed with the library's stage events (instrumented pass)
+    n_st = B.flint_moe_stage_count(stack.layers[0].handle, T)
+    names = [B.flint_moe_stage_name(stack.layers[0].handle, T, i) for i in range(n_st)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)] for _ in stack.layers]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    for layer, row in zip(stack.layers, evs):
+        B.flint_moe_set_stage_events(layer.handle, [e.cuda_event for e in row])
+    acc = np.zeros((n, n_st))
+    n_prof = max(1, min(args.steps, 20))
+    for _ in range(n_prof):
+        fwd()
+        torch.cuda.synchronize()
+        acc += [[row[i].elapsed_time(row[i + 1]) for i in range(n_st)] for row in evs]
+    for layer in stack.layers:
+        B.flint_moe_set_stage_events(layer.handle, None)
+    stage_ms = acc / n_prof
+    gi = names.index("gate_up")
+    gu_bytes = sum(stage_bytes("gate_up", E, fmt, T, 6, a) for a in n_active)
+    gu_ms = float(stage_ms[:, gi].sum())
+    peaks = measured_peaks()
+    achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "gate_up (every layer)", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": None, "algorithmic_bytes": gu_bytes, "peak_source": peaks["source"] + " (burst copy)"}
+
+    # end to end through the public API: H2D of the residual, the stack, D2H of the residual
+    xh = torch.empty((T, H), dtype=torch.float32).pin_memory()
+    xh.copy_(x0.cpu())
+
+    def e2e_step():
+        x.copy_(xh, non_blocking=True)
+        stack.forward(x)
+        xh.copy_(x, non_blocking=True)
+    e2e_ms = timed_steps(e2e_step, min(args.steps, 200))
+    e2e = {"value": round(T * len(e2e_ms) / (sum(e2e_ms) / 1e3), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4,
+           "ms_per_step": round(float(sum(e2e_ms)) / len(e2e_ms), 5)}
+    clk = clocks.stop()
+    errors = [layer.error_word() for layer in stack.layers]
+
+    # bounded CPU baseline (the oracle leg): the oracle on the first layers, per-layer time scaled
+    from oracle import flint_moe_ref as R
+    t0 = time.perf_counter()
+    done, xs = 0, R.bf16_to_f64(x_bits)
+    while done < n:
+        L = S.make_layer(E, fmt, seed=1000 + done)
+        t1 = time.perf_counter()
+        xs = R.stack_step(L, xs, eps=STACK_EPS)["x_next"]
+        el_layer = time.perf_counter() - t1
+        done += 1
+        if time.perf_counter() - t0 >= args.cpu_seconds:
+            break
+    cpu_layer_s = el_layer
+    cpu = {"value": round(T / (cpu_layer_s * n), 4), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": f"fp64 oracle stack step on {done} of the {n} layers ({cpu_layer_s:.2f} s for the last), "
+                     f"scaled to {n} layers"}
+    stack.close()
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "w4a16: int4 codes as exact int8 on the integer tensor cores against 16-bit fixed-point "
+                 "activations (int32 sums), fp32 accumulate; fp32 residual stream",
+        "data": "synthetic (seeded; random-init weights of the Flint MoE layer shape, layer l seed 1000+l)",
+        "config": {"workload": f"{args.workload}: {n} layers x (E={E} top-6, H=2048, I=512, shared 1024, {fmt}), "
+                               f"T={T}, x <- x + moe(rmsnorm(x))", "E": E, "T": T, "fmt": fmt, "layers": n,
+                   "distinct_experts_per_layer": round(float(np.mean(n_active)), 2),
+                   "l2": f"not flushed: {stack.weight_bytes() / 1e9:.1f} GB of weights stream through the 126 MB L2",
+                   "parallelism": "single GPU"},
+        "hbm": {"algorithmic_bytes": ab, "GB_per_s": round(ab / (ms_per_step * 1e-3) / 1e9, 1),
+                "pct_of_8TBps": round(100 * ab / (ms_per_step * 1e-3) / 1e9 / HBM_NOMINAL_GBS, 2),
+                "pct_of_measured": round(100 * ab / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 2)},
+        "per_layer_us": round(ms_per_step * 1e3 / n, 2),
+        "roofline": roofline,
+        "stage_us_per_layer": {nm: round(float(stage_ms[:, i].mean()) * 1e3, 2) for i, nm in enumerate(names)},
+        "e2e": e2e, "gpu_launches": (n * (n_st + 1) + 1) * args.steps, "clocks": clk, "cpu_baseline": cpu,
+        "error_words": sorted(set(errors)), "wall_s_timed_region": round(wall1 - wall0, 4),
+    }
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -465,6 +621,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.workload in STACK_LAYERS:
+        if rank == 0:
+            print(json.dumps(run_stack(args)), flush=True)
         return
     res = run_ours(args, rank, world, local_rank)
     if rank == 0:

@@ -112,7 +112,9 @@ class FlintMoEStack:
     """A stack of Flint MoE layers on one device, run on an fp32 residual stream:
     for each layer, z = bf16(rmsnorm(x)); x += layer(z) (flint_moe_stack_forward)."""
 
-    def __init__(self, layers: list, t_max: int, *, eps: float = 1e-6, device="cuda", **kw):
+    def __init__(self, layers, t_max: int, *, eps: float = 1e-6, device="cuda", **kw):
+        """layers: an iterable of host weight dicts; each is copied to the device as it comes, so a
+        generator keeps at most one layer on the host."""
         self.device = torch.device(device)
         self.eps = float(eps)
         self.t_max = t_max
