@@ -773,28 +773,42 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shared_kernel(const __grid_c
 // ---------------------------------------------------------------------------------------------
 // combine: y[t][n] = bf16(routed_scale * sum_k w[t][k] * o[inv[t][k]][n] + ys[t][n]), the slots
 // summed in slot order (ascending expert id) in fp32, one rounding at the end. One CTA per token,
-// 8 columns per thread.
+// 8 columns per thread; the loads of all slots are issued before the sum.
+template <int KMAX>
 __global__ void __launch_bounds__(256) pf_combine_kernel(const __half* __restrict__ o, const float* __restrict__ ys,
                                                          const float* __restrict__ w, const int* __restrict__ inv,
                                                          int K, float routed_scale, uint16_t* __restrict__ y) {
   const int t = blockIdx.x;
   const int n = threadIdx.x * 8;
+  // every slot's row index and weight first, then all rows' loads in flight together
+  int row[KMAX];
+  float wk[KMAX];
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k) {
+    row[k] = k < K ? __ldg(inv + t * K + k) : 0;
+    wk[k] = k < K ? __ldg(w + t * K + k) : 0.f;
+  }
+  uint4 ov[KMAX];
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k)
+    ov[k] = k < K ? __ldg(reinterpret_cast<const uint4*>(o + static_cast<size_t>(row[k]) * kH + n)) : make_uint4(0, 0, 0, 0);
+  const float4 s0 = __ldg(reinterpret_cast<const float4*>(ys + static_cast<size_t>(t) * kH + n));
+  const float4 s1 = __ldg(reinterpret_cast<const float4*>(ys + static_cast<size_t>(t) * kH + n + 4));
   float acc[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-  for (int k = 0; k < K; ++k) {
-    const float wk = w[t * K + k];
-    const uint4 ov = *reinterpret_cast<const uint4*>(o + static_cast<size_t>(inv[t * K + k]) * kH + n);
-    const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ow[j]));
-      acc[2 * j] = fmaf(wk, f.x, acc[2 * j]);
-      acc[2 * j + 1] = fmaf(wk, f.y, acc[2 * j + 1]);
+  for (int k = 0; k < KMAX; ++k) {                 // slot order
+    if (k < K) {
+      const uint32_t ow[4] = {ov[k].x, ov[k].y, ov[k].z, ov[k].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ow[j]));
+        acc[2 * j] = fmaf(wk[k], f.x, acc[2 * j]);
+        acc[2 * j + 1] = fmaf(wk[k], f.y, acc[2 * j + 1]);
+      }
     }
   }
-  const float4 s0 = *reinterpret_cast<const float4*>(ys + static_cast<size_t>(t) * kH + n);
-  const float4 s1 = *reinterpret_cast<const float4*>(ys + static_cast<size_t>(t) * kH + n + 4);
   const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
   uint4 out;
   uint32_t* ou = reinterpret_cast<uint32_t*>(&out);
@@ -854,7 +868,7 @@ cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, c
 cudaError_t launch_prefill_combine(const __half* o, const float* ys, const float* w, const int* inv, int T, int K,
                                    float routed_scale, uint16_t* y, cudaStream_t s) {
   static_assert(kH == 256 * 8, "one CTA of 256 threads x 8 columns per token");
-  pf_combine_kernel<<<T, 256, 0, s>>>(o, ys, w, inv, K, routed_scale, y);
+  pf_combine_kernel<kMaxTopK><<<T, 256, 0, s>>>(o, ys, w, inv, K, routed_scale, y);
   return cudaGetLastError();
 }
 
