@@ -34,7 +34,7 @@ EXPORTS = (
     "flint_moe_workspace_size", "flint_moe_create", "flint_moe_forward", "flint_moe_forward_host",
     "flint_moe_routing", "flint_moe_intermediate", "flint_moe_error_word", "flint_moe_destroy",
     "flint_moe_status_string", "flint_moe_set_stage_events", "flint_moe_stage_count", "flint_moe_stage_name",
-    "flint_moe_route_noalloc",
+    "flint_moe_route_noalloc", "flint_residual_rmsnorm", "flint_moe_stack_forward",
 )
 
 

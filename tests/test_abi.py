@@ -88,6 +88,24 @@ def test_calls_on_a_null_handle_fail_cleanly():
         B.flint_moe_forward(0, 0x1000, 1, 0x2000)
 
 
+def test_stack_entry_points_check_arguments_on_the_host():
+    V, F = ctypes.c_void_p, ctypes.c_float
+    # residual + norm: negative T, non-positive eps, misaligned or missing residual -> rejected before a launch
+    assert B.raw_status("flint_residual_rmsnorm", V(0x1000), V(0), -1, F(1e-6), V(0x2000), V(0)) == B.FLINT_ERR_INVALID_ARG
+    assert B.raw_status("flint_residual_rmsnorm", V(0x1000), V(0), 4, F(0.0), V(0x2000), V(0)) == B.FLINT_ERR_INVALID_ARG
+    assert B.raw_status("flint_residual_rmsnorm", V(0x1004), V(0), 4, F(1e-6), V(0x2000), V(0)) == B.FLINT_ERR_INVALID_ARG
+    assert B.raw_status("flint_residual_rmsnorm", V(0), V(0), 4, F(1e-6), V(0x2000), V(0)) == B.FLINT_ERR_INVALID_ARG
+    assert B.raw_status("flint_residual_rmsnorm", V(0), V(0), 0, F(1e-6), V(0), V(0)) == B.FLINT_OK      # T = 0: no-op
+    # stack: no layers, a null layer handle
+    arr = (ctypes.c_void_p * 2)(None, None)
+    assert B.raw_status("flint_moe_stack_forward", None, 1, V(0x1000), 4, F(1e-6), V(0x2000), V(0x3000), V(0)) == \
+        B.FLINT_ERR_INVALID_ARG
+    assert B.raw_status("flint_moe_stack_forward", arr, 0, V(0x1000), 4, F(1e-6), V(0x2000), V(0x3000), V(0)) == \
+        B.FLINT_ERR_INVALID_ARG
+    assert B.raw_status("flint_moe_stack_forward", arr, 2, V(0x1000), 4, F(1e-6), V(0x2000), V(0x3000), V(0)) == \
+        B.FLINT_ERR_INVALID_ARG
+
+
 def test_status_strings():
     for s in range(7):
         assert B.flint_moe_status_string(s)
