@@ -8,14 +8,14 @@
 //   warp 0       TMA copies of the 4-bit codes, 128 K per stage, into a shared-memory ring
 //   warp 3       TMA copies of the chunk's activation rows (fp16, stored per permuted row so that
 //                an expert's rows are contiguous; 128-byte swizzled K-major, 16-row boxes) into a ring
-//   warps 4-11   dequantisation: a thread owns one weight row of one block, turns its 128 codes of
-//                the stage into exact fp16 (int4: code x bf16 group scale; NVFP4: E2M1 x E4M3) and
+//   warps 4..    dequantisation (8 or 16 warps): a thread owns one weight row of one block and both
+//                64-code halves of the stage, or one of them, turns those codes into exact fp16 (int4: code x bf16 group scale; NVFP4: E2M1 x E4M3) and
 //                writes them to tensor memory with tcgen05.st, where the MMA reads its A operand.
 //                A in tensor memory costs no shared-memory bandwidth, which a 128 x 48 MMA with A
 //                in shared memory would exhaust.
 //   warps 1, 2   one MMA-issuing thread per block (an MMA instruction takes ~45 cycles to issue, so
 //                two issuers keep N = 48 tiles near the tensor-core rate); D[128 x N] per block
-//   warps 12-15  epilogue: gate|up -> h = silu(g) u, int4: rotated per 128-segment by the Hadamard
+//   last 4 warps epilogue: gate|up -> h = silu(g) u, int4: rotated per 128-segment by the Hadamard
 //                butterfly, stored fp16 in the order of the down operand; down -> o in fp16.
 // Every dependency is an mbarrier: TMA transaction counts, cp.async arrivals, tcgen05.commit
 // arrivals and thread arrivals; every wait is bounded and sets a timeout bit on expiry.
@@ -44,7 +44,14 @@ constexpr int kPfCodeStage = 2 * 128 * kPfSK / 2;    // 16 KB: two blocks of 128
 constexpr int kPfActChunk = kPfN * 128;              // 64 K of every row, 128-byte swizzled
 constexpr int kPfActStage = 2 * kPfActChunk;         // 16 KB
 constexpr int kSlabPitch = 132;              // floats per token row of the epilogue's transpose slab
-constexpr int kPfThreads = 512;
+// Dequantisation warps: 4 lane quarters x 2 blocks, x 2 halves of the stage when there are 16. The
+// int4 gate|up tiles run fastest with 8 (two halves per thread), the others with 16 (measured).
+template <int FMT, int PHASE>
+struct PfRoles {
+  static constexpr int kDq = (FMT == kInt4 && PHASE == kPhaseGateUp) ? 8 : 16;
+  static constexpr int kHalves = 16 / kDq;          // stage halves per dequantisation thread
+  static constexpr int kThreads = 32 * (4 + kDq + 4);
+};
 
 // tensor-memory columns: two accumulator slots of (D0 | D1) x 64 columns, then two A stages of two
 // blocks x 64 columns (128 fp16 of K)
@@ -291,8 +298,9 @@ __device__ __forceinline__ void dequant_half(uint32_t (&v)[32], const uint4& wa,
 // routed grouped GEMM
 
 template <int FMT, int PHASE>
-__global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_constant__ PrefillParams p) {
+__global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_kernel(const __grid_constant__ PrefillParams p) {
   using G = PfGeom<PHASE>;
+  using R = PfRoles<FMT, PHASE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   TileTab& tt = *reinterpret_cast<TileTab*>(sm + kOffTab);
@@ -304,7 +312,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_c
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPfDA; ++i) {
       mbar_init(&bb.code_full[i], 1);
-      mbar_init(&bb.code_empty[i], 8);
+      mbar_init(&bb.code_empty[i], R::kDq);
     }
     for (int i = 0; i < kPfDB; ++i) {
       mbar_init(&bb.act_full[i], 1);
@@ -312,7 +320,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_c
     }
     for (int t = 0; t < 2; ++t)
       for (int b = 0; b < 2; ++b) {
-        mbar_init(&bb.a_full[t][b], 4);
+        mbar_init(&bb.a_full[t][b], R::kDq / 2);
         mbar_init(&bb.a_empty[t][b], 1);
       }
     for (int a = 0; a < 2; ++a) {
@@ -416,9 +424,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_c
     }
     tc_commit_w(&bb.done[b]);                     // every MMA of this warp has completed
     pf_wait_all(&bb.done[b], 0, abort, p.err);
-  } else if (warp >= 4 && warp < 12) {
+  } else if (warp >= 4 && warp < 4 + R::kDq) {
     // ---- dequantisation into tensor memory
-    const int b = (warp - 4) >> 2, q = warp & 3;
+    const int b = ((warp - 4) >> 2) & 1, h0 = (warp - 4) >> 3, q = warp & 3;   // h0: first half
     const int r = 32 * q + lane;
     const int swz = (lane >> 1) & 3;               // 64-byte swizzle of the code rows (row r at r*64)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
@@ -477,9 +485,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_c
           break;
         }
         const uint8_t* src = sm + kOffCode + slot * kPfCodeStage + b * (kPfCodeStage / 2) + r * (kPfSK / 2);
-        uint4 w[4];
+        uint4 w[2 * R::kHalves];                  // the row's 16-byte chunks of its halves
 #pragma unroll
-        for (int k = 0; k < 4; ++k) w[k] = *reinterpret_cast<const uint4*>(src + ((k ^ swz) << 4));
+        for (int k = 0; k < 2 * R::kHalves; ++k) w[k] = *reinterpret_cast<const uint4*>(src + (((2 * h0 + k) ^ swz) << 4));
         __syncwarp();
         if (lane == 0) mbar_arrive(&bb.code_empty[slot]);
         uint32_t s_int4 = 0;
@@ -492,16 +500,18 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_c
         }
         // the first half's arithmetic runs before the tensor-memory stage is free
         uint32_t v[32];
-        dequant_half<FMT>(v, w[0], w[1], s_int4, s_fp4.x);
+        dequant_half<FMT>(v, w[0], w[1], s_int4, h0 ? s_fp4.y : s_fp4.x);
         if (it >= 2 && !pf_wait_all(&bb.a_empty[ts][b], ((it >> 1) - 1) & 1, abort, p.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t ta = lane_base + kColA + ts * 128 + b * 64;
+        const uint32_t ta = lane_base + kColA + ts * 128 + b * 64 + h0 * 32;
         tc_st32(ta, v);
-        dequant_half<FMT>(v, w[2], w[3], s_int4, s_fp4.y);
-        tc_st32(ta + 32, v);
+        if constexpr (R::kHalves == 2) {
+          dequant_half<FMT>(v, w[2], w[3], s_int4, s_fp4.y);
+          tc_st32(ta + 32, v);
+        }
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -512,7 +522,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_routed_kernel(const __grid_c
       row = row_next;
     }
     if (bad) atomicOr(p.err, kErrRange);
-  } else if (warp >= 12) {
+  } else if (warp >= 4 + R::kDq) {
     // ---- epilogue
     const int q = warp & 3, r = 32 * q + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
@@ -836,11 +846,15 @@ cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, in
     smem_set = true;
   }
   if (fmt == kInt4) {
-    if (phase == kPhaseGateUp) pf_routed_kernel<kInt4, kPhaseGateUp><<<n_sm, kPfThreads, kPfSmem, s>>>(p);
-    else pf_routed_kernel<kInt4, kPhaseDown><<<n_sm, kPfThreads, kPfSmem, s>>>(p);
+    if (phase == kPhaseGateUp)
+      pf_routed_kernel<kInt4, kPhaseGateUp><<<n_sm, PfRoles<kInt4, kPhaseGateUp>::kThreads, kPfSmem, s>>>(p);
+    else
+      pf_routed_kernel<kInt4, kPhaseDown><<<n_sm, PfRoles<kInt4, kPhaseDown>::kThreads, kPfSmem, s>>>(p);
   } else {
-    if (phase == kPhaseGateUp) pf_routed_kernel<kNvfp4, kPhaseGateUp><<<n_sm, kPfThreads, kPfSmem, s>>>(p);
-    else pf_routed_kernel<kNvfp4, kPhaseDown><<<n_sm, kPfThreads, kPfSmem, s>>>(p);
+    if (phase == kPhaseGateUp)
+      pf_routed_kernel<kNvfp4, kPhaseGateUp><<<n_sm, PfRoles<kNvfp4, kPhaseGateUp>::kThreads, kPfSmem, s>>>(p);
+    else
+      pf_routed_kernel<kNvfp4, kPhaseDown><<<n_sm, PfRoles<kNvfp4, kPhaseDown>::kThreads, kPfSmem, s>>>(p);
   }
   return cudaGetLastError();
 }

@@ -61,6 +61,20 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
 // would create. Ties go to the lower expert id. The chosen slots are listed by ascending expert
 // id, and w_k = s_k / max(sum of the chosen s, floor) with s = sigmoid(logit) (the SelectedSumFloor
 // policy, same issue, host-policy comment). The sum runs in slot order.
+// Selection runs on order-preserving 32-bit keys so that each of the k rounds is two warp reductions
+// (redux.sync): the largest key, then the lowest index holding it. -0 is keyed as +0 (the two compare
+// equal as logits) and NaN as 0, below every number, so it is picked only when nothing else is left.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+  uint32_t u = __float_as_uint(v);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return 0u;   // NaN
+  if ((u << 1) == 0u) u = 0u;                          // -0 as +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_logit(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 template <int NS>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
                                                    float* __restrict__ logits_out, int T, int E, int K,
@@ -81,182 +95,191 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     float a = part[0];
 #pragma unroll
     for (int q = 1; q < NS; ++q) a += part[q];     // slice order
-    v[j] = (j < per) ? a : -INFINITY;
+    v[j] = a;
   }
   if (logits_out) {
 #pragma unroll
     for (int j = 0; j < 8; ++j)
       if (j < per) logits_out[static_cast<size_t>(t) * E + lane + 32 * j] = v[j];
   }
-  unsigned taken = 0;              // bit j: element lane+32j already chosen
-  int my_id = 0x7FFFFFFF;          // lane k < K: the k-th pick
-  float my_l = 0.f;
-  for (int k = 0; k < K; ++k) {
-    // local best: highest logit, then lowest index
-    float bv = -INFINITY;
-    int bi = 0x7FFFFFFF;
+  uint32_t key[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int idx = lane + 32 * j;
-      const bool ok = (j < per) && !((taken >> j) & 1u);
-      if (ok && (v[j] > bv || (v[j] == bv && idx < bi))) { bv = v[j]; bi = idx; }
-    }
+  for (int j = 0; j < 8; ++j) key[j] = logit_key(v[j]);
+  unsigned live = (1u << per) - 1u;                // bit j: element lane+32j not yet chosen
+  // the picks are warp-uniform: every lane keeps all of them
+  int pid[kMaxTopK];
+  uint32_t pkey[kMaxTopK];
 #pragma unroll
-    for (int m = 16; m > 0; m >>= 1) {
-      const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, m);
-      const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, m);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+  for (int k = 0; k < kMaxTopK; ++k) {
+    pid[k] = 0x7FFFFFFF;           // unused slots sort last
+    pkey[k] = 0u;
+    if (k < K) {
+      uint32_t lk = 0u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if ((live >> j) & 1u) lk = max(lk, key[j]);
+      const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, lk);
+      uint32_t li = 0xFFFFFFFFu;
+#pragma unroll
+      for (int j = 7; j >= 0; --j)
+        if (((live >> j) & 1u) && key[j] == m) li = static_cast<uint32_t>(lane + 32 * j);
+      const uint32_t bi = __reduce_min_sync(0xFFFFFFFFu, li);
+      if (static_cast<int>(bi & 31u) == lane) live &= ~(1u << (bi >> 5));
+      pid[k] = static_cast<int>(bi);
+      pkey[k] = m;
     }
-    if (lane == k) {
-      my_id = bi;
-      my_l = bv;
-    }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
   }
-  // slot of the pick = its rank by expert id; lane r then takes the pick of rank r
-  int rank = 0;
-  for (int j = 0; j < K; ++j) rank += (__shfl_sync(0xFFFFFFFFu, my_id, j) < my_id);
-  const float my_s = 1.0f / (1.0f + expf(-my_l));
-  int id = 0;
-  float s = 0.f, sum = 0.f;
-  for (int r = 0; r < K; ++r) {
-    const unsigned who = __ballot_sync(0xFFFFFFFFu, lane < K && rank == r);
-    const int src = __ffs(who) - 1;
-    const int id_r = __shfl_sync(0xFFFFFFFFu, my_id, src);
-    const float s_r = __shfl_sync(0xFFFFFFFFu, my_s, src);
-    sum += s_r;                    // slot order
-    if (lane == r) {
-      id = id_r;
-      s = s_r;
+  // slots by ascending expert id (odd-even transposition network; the ids are distinct)
+#pragma unroll
+  for (int r = 0; r < kMaxTopK; ++r) {
+#pragma unroll
+    for (int i = r & 1; i + 1 < kMaxTopK; i += 2) {
+      if (pid[i] > pid[i + 1]) {
+        const int ti = pid[i];
+        pid[i] = pid[i + 1];
+        pid[i + 1] = ti;
+        const uint32_t tk = pkey[i];
+        pkey[i] = pkey[i + 1];
+        pkey[i + 1] = tk;
+      }
     }
+  }
+  float s[kMaxTopK];
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < kMaxTopK; ++k) {
+    s[k] = 1.0f / (1.0f + expf(-key_logit(pkey[k])));
+    if (k < K) sum += s[k];        // slot order
   }
   const float denom = fmaxf(sum, floor_);
+  int id = 0;
+  float sk = 0.f;
+#pragma unroll
+  for (int k = 0; k < kMaxTopK; ++k)
+    if (lane == k) {
+      id = pid[k];
+      sk = s[k];
+    }
   if (lane < K) {
     if ((flags & 1u) && (id < 0 || id >= E)) atomicOr(err, kErrBadId);
     ids[t * K + lane] = id;
-    wts[t * K + lane] = s / denom;
+    wts[t * K + lane] = sk / denom;
   }
 }
 
 // ---------------------------------------------------------------------------------------------
-// Expert-major permutation of the (token, slot) pairs: one CTA per two experts.
+// Expert-major permutation of the (token, slot) pairs, a counting sort that keeps pair order.
 // counts[e] = number of pairs routed to e; offsets = exclusive prefix (E+1 entries);
 // position p in [offsets[e], offsets[e+1]) lists the pairs of expert e by ascending token:
-// perm[p] = t*K+k and inv[t*K+k] = p. Every CTA reads all P = T*K expert ids (L2-resident):
-// pass 1 counts the pairs routed below e (its offset) and to e; a block scan over the threads'
-// contiguous shares gives each thread its first position; pass 2 writes the pairs of e in pair
-// order (a token routes to e at most once, so pair order is token order). No atomics decide an
-// order, so the result is deterministic. Invalid ids count as expert 0 (and are flagged).
-constexpr int kPermThreads = 1024;
+// perm[p] = t*K+k and inv[t*K+k] = p. CTA c owns the 1024 pairs [1024c, 1024c + 1024), one per
+// thread. It counts, in shared memory, every expert over all P pairs and over the pairs before its
+// range (the ids are L2-resident), which gives the first position of each expert in its range; a
+// pair's place among the equal ids of its range is its rank in its warp (match.any) plus the
+// counts of the warps before it. Counts do not depend on the order of the shared-memory atomics, so
+// the result is deterministic. A token routes to e at most once, so pair order is token order.
+// Invalid ids count as expert 0 (and are flagged).
+constexpr int kPermThreads = 1024;               // = pairs per CTA
 constexpr int kPermWarps = kPermThreads / 32;
-constexpr int kPermChunk = 16;                   // ids a thread holds in registers per round
-constexpr int kPermExperts = 2;                  // experts per CTA
+constexpr int kPermUnroll = 4;                   // 16-byte id loads in flight per thread
 
 __device__ __forceinline__ int clamp_id(int v, int E) { return (v < 0 || v >= E) ? 0 : v; }
-
-// Loads ids [i0, i0 + 16) as four 16-byte vectors (entries past P are not read); i0 is a multiple of 16.
-__device__ __forceinline__ void load_ids16(int (&v)[kPermChunk], const int* ids, int i0, int P) {
-  if (i0 + kPermChunk <= P) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int4 w = __ldg(reinterpret_cast<const int4*>(ids + i0) + q);
-      v[4 * q] = w.x;
-      v[4 * q + 1] = w.y;
-      v[4 * q + 2] = w.z;
-      v[4 * q + 3] = w.w;
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < kPermChunk; ++j) v[j] = (i0 + j < P) ? __ldg(ids + i0 + j) : 0;
-  }
-}
-
-// Counts the first `nv` of the thread's ids that are below e and equal to e.
-__device__ __forceinline__ void count_ids(const int (&v)[kPermChunk], int nv, int e, int E, int& lt, int& eq,
-                                          bool& bad) {
-#pragma unroll
-  for (int j = 0; j < kPermChunk; ++j) {
-    if (j >= nv) continue;
-    bad |= v[j] < 0 || v[j] >= E;
-    const int c = clamp_id(v[j], E);
-    lt += c < e;
-    eq += c == e;
-  }
-}
 
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __restrict__ ids, int P, int E,
                                                                int* __restrict__ counts, int* __restrict__ offsets,
                                                                int* __restrict__ perm, int* __restrict__ inv,
                                                                unsigned flags, unsigned* __restrict__ err) {
-  __shared__ int w_sum[kPermWarps], w_base[kPermWarps];
-  __shared__ int s_total;
+  __shared__ int h_total[kMaxE], h_before[kMaxE], first[kMaxE];
+  __shared__ int wcnt[kPermWarps * kMaxE];        // [warp][expert]: pairs of the expert in the warp
+  __shared__ int scan_w[kMaxE / 32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  constexpr int kRound = kPermThreads * kPermChunk;
-  // warp-order exclusive scan of one value per thread over the CTA; returns the exclusive prefix and
-  // leaves the CTA total in s_total
-  auto block_scan = [&](int x) -> int {
-    int incl = x;
+  const int c0 = blockIdx.x * kPermThreads;
+  const int i = c0 + tid;
+  const int raw = i < P ? __ldg(ids + i) : 0;
+  for (int q = tid; q < E; q += kPermThreads) {
+    h_total[q] = 0;
+    h_before[q] = 0;
+  }
+  for (int q = tid; q < kPermWarps * E; q += kPermThreads) wcnt[q] = 0;
+  __syncthreads();
+  // histograms of all pairs and of the pairs before this range (ids + 4j is 16-byte aligned)
+  bool bad = false;
+  for (int r0 = 0; r0 < P; r0 += 4 * kPermThreads * kPermUnroll) {
+    int v[4 * kPermUnroll];
+#pragma unroll
+    for (int u = 0; u < kPermUnroll; ++u) {
+      const int j0 = r0 + 4 * (tid + u * kPermThreads);
+      if (j0 + 4 <= P) {
+        const int4 w = __ldg(reinterpret_cast<const int4*>(ids + j0));
+        v[4 * u] = w.x;
+        v[4 * u + 1] = w.y;
+        v[4 * u + 2] = w.z;
+        v[4 * u + 3] = w.w;
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[4 * u + q] = (j0 + q < P) ? __ldg(ids + j0 + q) : 0;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPermUnroll; ++u) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = r0 + 4 * (tid + u * kPermThreads) + q;
+        if (j < P) {
+          bad |= v[4 * u + q] < 0 || v[4 * u + q] >= E;
+          const int e = clamp_id(v[4 * u + q], E);
+          atomicAdd(&h_total[e], 1);
+          if (j < c0) atomicAdd(&h_before[e], 1);
+        }
+      }
+    }
+  }
+  if (bad && (flags & 1u) && blockIdx.x == 0) atomicOr(err, kErrBadId);
+  // this thread's pair: its rank among the equal ids of its warp
+  const int e = i < P ? clamp_id(raw, E) : -1;
+  const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+  const int rank_w = __popc(peers & ((1u << lane) - 1u));
+  if (i < P && rank_w == 0) wcnt[warp * E + e] = __popc(peers);
+  __syncthreads();
+  // offsets: exclusive scan of the totals over the experts; per expert, exclusive scan of the warp
+  // counts over the warps
+  int incl = 0, tot = 0;
+  if (tid < kMaxE) {
+    tot = tid < E ? h_total[tid] : 0;
+    incl = tot;
 #pragma unroll
     for (int m = 1; m < 32; m <<= 1) {
       const int o = __shfl_up_sync(0xFFFFFFFFu, incl, m);
       if (lane >= m) incl += o;
     }
-    __syncthreads();                               // w_sum / s_total of a previous scan are consumed
-    if (lane == 31) w_sum[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      const int c = w_sum[lane];
-      int s = c;
+    if (lane == 31) scan_w[warp] = incl;
+    if (tid < E) {
+      int c[kPermWarps];
 #pragma unroll
-      for (int m = 1; m < 32; m <<= 1) {
-        const int o = __shfl_up_sync(0xFFFFFFFFu, s, m);
-        if (lane >= m) s += o;
-      }
-      w_base[lane] = s - c;
-      if (lane == 31) s_total = s;
-    }
-    __syncthreads();
-    return w_base[warp] + incl - x;
-  };
-  // the CTA's experts share the ids it loads (all of them in registers when P fits one round)
-  int v[kPermChunk];
-  for (int e = blockIdx.x * kPermExperts; e < min(E, blockIdx.x * kPermExperts + kPermExperts); ++e) {
-    // pass 1: pairs routed below e (the offset of e)
-    int lt = 0, eq_unused = 0;
-    bool bad = false;
-    for (int r0 = 0; r0 < P; r0 += kRound) {
-      const int i0 = r0 + kPermChunk * tid;
-      if (P > kRound || e == blockIdx.x * kPermExperts) load_ids16(v, ids, i0, P);
-      count_ids(v, min(max(P - i0, 0), kPermChunk), e, E, lt, eq_unused, bad);
-    }
-    if (bad && (flags & 1u) && e == 0) atomicOr(err, kErrBadId);
-    block_scan(lt);
-    const int off = s_total;
-    // pass 2: the pairs of e in pair order at off, off + 1, ...
-    int run = 0;
-    for (int r0 = 0; r0 < P; r0 += kRound) {
-      const int i0 = r0 + kPermChunk * tid;
-      const int nv = min(max(P - i0, 0), kPermChunk);
-      if (P > kRound) load_ids16(v, ids, i0, P);   // one round: the ids are still in registers
-      int l2 = 0, eq = 0;
-      bool b2 = false;
-      count_ids(v, nv, e, E, l2, eq, b2);
-      int pos = off + run + block_scan(eq);
-      run += s_total;
+      for (int w = 0; w < kPermWarps; ++w) c[w] = wcnt[w * E + tid];
+      int run = 0;
 #pragma unroll
-      for (int j = 0; j < kPermChunk; ++j) {
-        if (j < nv && clamp_id(v[j], E) == e) {
-          perm[pos] = i0 + j;
-          inv[i0 + j] = pos;
-          ++pos;
-        }
+      for (int w = 0; w < kPermWarps; ++w) {
+        wcnt[w * E + tid] = run;
+        run += c[w];
       }
     }
-    if (tid == 0) {
-      counts[e] = run;
-      offsets[e] = off;
-      if (e == E - 1) offsets[E] = off + run;
+  }
+  __syncthreads();
+  if (tid < E) {
+    int off = incl - tot;
+    for (int w = 0; w < warp; ++w) off += scan_w[w];
+    first[tid] = off + h_before[tid];
+    if (blockIdx.x == 0) {
+      counts[tid] = tot;
+      offsets[tid] = off;
+      if (tid == E - 1) offsets[E] = off + tot;
     }
+  }
+  __syncthreads();
+  if (i < P) {
+    const int pos = first[e] + wcnt[warp * E + e] + rank_w;
+    perm[pos] = i;
+    inv[i] = pos;
   }
 }
 
@@ -305,8 +328,9 @@ cudaError_t launch_topk(const float* logits, int nsplit, float* logits_out, int 
 
 cudaError_t launch_permute(const int* ids, int T, int K, int E, int* counts, int* offsets, int* perm, int* inv,
                            unsigned flags, unsigned* err, cudaStream_t s) {
-  permute_kernel<<<(E + kPermExperts - 1) / kPermExperts, kPermThreads, 0, s>>>(ids, T * K, E, counts, offsets, perm, inv,
-                                                                                  flags, err);
+  const int P = T * K;
+  const int grid = P > 0 ? (P + kPermThreads - 1) / kPermThreads : 1;
+  permute_kernel<<<grid, kPermThreads, 0, s>>>(ids, P, E, counts, offsets, perm, inv, flags, err);
   return cudaGetLastError();
 }
 
