@@ -329,6 +329,9 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   // expert's kernels (which leave SMs free) run on `s`. With instrumentation everything runs on `s`
   // in stage order.
   const bool fork = h->n_events == 0 && h->side != nullptr;
+  // routed down and combine start as programmatic dependents of their predecessor (not between
+  // instrumentation events, which serialise the stages anyway)
+  const bool pdl = h->n_events == 0;
   cudaStream_t rs = fork ? h->side : s;
   if (fork) {
     FLINT_TRY(cudaEventRecord(h->ev_fork, s));
@@ -361,13 +364,13 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   pp.tm_act = h->tm_pf_xg;
   pp.scales = h->w.gu_scales;
   pp.tscale = h->w.gu_tscale;
-  FLINT_TRY(launch_prefill_routed(pp, fmt, kPhaseGateUp, h->n_sm, s));
+  FLINT_TRY(launch_prefill_routed(pp, fmt, kPhaseGateUp, h->n_sm, false, s));
   FLINT_TRY(m.mark());
   pp.tm_codes = h->tm_pf_dn;
   pp.tm_act = h->tm_pf_hq;
   pp.scales = h->w.dn_scales;
   pp.tscale = h->w.dn_tscale;
-  FLINT_TRY(launch_prefill_routed(pp, fmt, kPhaseDown, h->n_sm, s));
+  FLINT_TRY(launch_prefill_routed(pp, fmt, kPhaseDown, h->n_sm, pdl, s));
   FLINT_TRY(m.mark());
   if (!fork) {
     pp.tm_a = h->tm_pf_sh_dn;
@@ -376,7 +379,7 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
     FLINT_TRY(launch_prefill_shared(pp, kPhaseDown, h->n_sm, s));
     FLINT_TRY(m.mark());
   }
-  FLINT_TRY(launch_prefill_combine(reinterpret_cast<const __half*>(h->o), h->ys, h->wts, h->inv, T, K, c.routed_scale, y, s));
+  FLINT_TRY(launch_prefill_combine(reinterpret_cast<const __half*>(h->o), h->ys, h->wts, h->inv, T, K, c.routed_scale, y, pdl, s));
   FLINT_TRY(m.mark());
   return FLINT_OK;
 }

@@ -91,7 +91,9 @@ struct PrefillParams {
   unsigned* err;
 };
 
-cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, int n_sm, cudaStream_t s);
+// pdl: launched as a programmatic dependent of the previous kernel in the stream (the routed down
+// kernel streams its weights while the gate|up kernel finishes; it waits for it before reading h).
+cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, int n_sm, bool pdl, cudaStream_t s);
 cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, cudaStream_t s);
 
 // Residual stream of a layer stack: x (f32 [T][H]) += y (bf16, when not null); then, when z is not
@@ -107,6 +109,6 @@ cudaError_t launch_permute(const int* ids, int T, int K, int E, int* counts, int
 cudaError_t launch_xg(const uint16_t* x, int T, int K, const int* inv, int rotate, __half* xg, cudaStream_t s);
 
 cudaError_t launch_prefill_combine(const __half* o, const float* ys, const float* w, const int* inv, int T, int K,
-                                   float routed_scale, uint16_t* y, cudaStream_t s);
+                                   float routed_scale, uint16_t* y, bool pdl, cudaStream_t s);
 
 }  // namespace flint

@@ -62,6 +62,12 @@ constexpr uint32_t kColA = 256;
 // ---------------------------------------------------------------------------------------------
 // tcgen05 / TMA primitives
 
+// Programmatic dependent launch: the next kernel of the stream may be scheduled once every CTA of this
+// one has called launch_dependents (or exited); wait blocks until the previous kernel has completed
+// and its writes are visible (a no-op without a programmatic predecessor).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -343,6 +349,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
   tc_fence_after();
   const uint32_t tmem = bb.tmem;
   const int total = tt.total;
+  pdl_trigger();   // the next kernel's CTAs take the SMs this grid leaves (it is resident in full)
 
   if (warp == 0) {
     // ---- codes: two TMA boxes (128 rows x 64 bytes) per stage
@@ -368,6 +375,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
     // chunk's rows rounded up to 16 in boxes of 16 rows x 64 fp16 (128-byte swizzled, 2 KB each);
     // rows past the chunk only feed unused accumulator columns
     if (lane == 0) {
+      pdl_wait();     // the activation rows are the previous kernel's output
       int it = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
         const PfTile tl = tile_at(tt, t);
@@ -790,6 +798,7 @@ __global__ void __launch_bounds__(256) pf_combine_kernel(const __half* __restric
                                                          int K, float routed_scale, uint16_t* __restrict__ y) {
   const int t = blockIdx.x;
   const int n = threadIdx.x * 8;
+  pdl_wait();      // o is the previous kernel's output
   // every slot's row index and weight first, then all rows' loads in flight together
   int row[KMAX];
   float wk[KMAX];
@@ -835,7 +844,22 @@ cudaError_t allow_smem(Kern kernel, int bytes) {
 
 }  // namespace
 
-cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, int n_sm, cudaStream_t s) {
+template <typename Kern, typename... Args>
+cudaError_t launch_maybe_pdl(Kern kernel, int grid, int threads, int smem, bool pdl, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, int n_sm, bool pdl, cudaStream_t s) {
   static bool smem_set = false;
   if (!smem_set) {
     cudaError_t e;
@@ -846,15 +870,17 @@ cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, in
     smem_set = true;
   }
   if (fmt == kInt4) {
-    if (phase == kPhaseGateUp)
-      pf_routed_kernel<kInt4, kPhaseGateUp><<<n_sm, PfRoles<kInt4, kPhaseGateUp>::kThreads, kPfSmem, s>>>(p);
-    else
-      pf_routed_kernel<kInt4, kPhaseDown><<<n_sm, PfRoles<kInt4, kPhaseDown>::kThreads, kPfSmem, s>>>(p);
+    return phase == kPhaseGateUp
+               ? launch_maybe_pdl(pf_routed_kernel<kInt4, kPhaseGateUp>, n_sm, PfRoles<kInt4, kPhaseGateUp>::kThreads,
+                                  kPfSmem, pdl, s, p)
+               : launch_maybe_pdl(pf_routed_kernel<kInt4, kPhaseDown>, n_sm, PfRoles<kInt4, kPhaseDown>::kThreads,
+                                  kPfSmem, pdl, s, p);
   } else {
-    if (phase == kPhaseGateUp)
-      pf_routed_kernel<kNvfp4, kPhaseGateUp><<<n_sm, PfRoles<kNvfp4, kPhaseGateUp>::kThreads, kPfSmem, s>>>(p);
-    else
-      pf_routed_kernel<kNvfp4, kPhaseDown><<<n_sm, PfRoles<kNvfp4, kPhaseDown>::kThreads, kPfSmem, s>>>(p);
+    return phase == kPhaseGateUp
+               ? launch_maybe_pdl(pf_routed_kernel<kNvfp4, kPhaseGateUp>, n_sm, PfRoles<kNvfp4, kPhaseGateUp>::kThreads,
+                                  kPfSmem, pdl, s, p)
+               : launch_maybe_pdl(pf_routed_kernel<kNvfp4, kPhaseDown>, n_sm, PfRoles<kNvfp4, kPhaseDown>::kThreads,
+                                  kPfSmem, pdl, s, p);
   }
   return cudaGetLastError();
 }
@@ -880,10 +906,9 @@ cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, c
 }
 
 cudaError_t launch_prefill_combine(const __half* o, const float* ys, const float* w, const int* inv, int T, int K,
-                                   float routed_scale, uint16_t* y, cudaStream_t s) {
+                                   float routed_scale, uint16_t* y, bool pdl, cudaStream_t s) {
   static_assert(kH == 256 * 8, "one CTA of 256 threads x 8 columns per token");
-  pf_combine_kernel<kMaxTopK><<<T, 256, 0, s>>>(o, ys, w, inv, K, routed_scale, y);
-  return cudaGetLastError();
+  return launch_maybe_pdl(pf_combine_kernel<kMaxTopK>, T, 256, 0, pdl, s, o, ys, w, inv, K, routed_scale, y);
 }
 
 }  // namespace flint
