@@ -93,8 +93,9 @@ def test_prefill_nvfp4_full_size():
 
 
 def test_permutation_spans_rounds():
-    # T*K = 18000 (token, slot) pairs: more than one round of the permutation kernel's register
-    # blocking (16384 pairs); the permutation is rebuilt from the device's ids by the oracle
+    # T*K = 18000 (token, slot) pairs: 18 CTAs of the counting sort (1024 pairs each, the last one
+    # ragged) and more than one round (16384 ids) of its histogram loop; the permutation is rebuilt
+    # from the device's ids by the oracle
     L = layer(32, "int4")
     T = 3000
     x = S.make_workload_x(T, 32)
@@ -128,6 +129,32 @@ def test_all_tokens_on_six_experts():
     x = S.make_x(64, skew=True)                                 # x[:, 0] = 1
     dev, xd, y, ref, st = full_check(L, x)
     np.testing.assert_array_equal(np.diff(ref["offsets"])[:6], 64)
+
+
+@pytest.mark.parametrize("T", [8, 64])
+def test_exact_tie_goes_to_lower_id(T):
+    # router rows 9 and 12 are identical, so their logits are equal bit for bit on every path; with
+    # experts 0..4 far above and the rest far below, the sixth pick is a tie between 9 and 12 for
+    # every token and must go to the lower id (T = 8: decode kernels; T = 64: tensor-core router and
+    # the top-k kernel of the prefill path)
+    L = dict(layer(32, "int4"))
+    rw = L["router_w"].copy()
+    rw[12] = rw[9]
+    col = np.full(32, -16.0, np.float32)
+    col[:5] = 16.0
+    col[9] = col[12] = 4.0
+    rw[:, 0] = S.f32_to_bf16_bits(col)
+    L["router_w"] = rw
+    x = S.make_x(T, skew=True)                                  # x[:, 0] = 1
+    ref = R.moe_forward(L, x)
+    expect = np.tile(np.array([0, 1, 2, 3, 4, 9], np.int32), (T, 1))
+    np.testing.assert_array_equal(ref["ids"], expect)
+    assert np.all(ref["gap"] == 0.0)                            # the tie is exact in the oracle too
+    dev, xd, y = run(L, x)
+    np.testing.assert_array_equal(dev.routing(T)["ids"].cpu().numpy(), expect)
+    st = PT.compare_y(y_to_host_bits(y), ref["y"])
+    assert st["finite"] and st["violations"] == 0, st
+    assert dev.error_word() == 0
 
 
 def test_intermediates_router_logits_and_rotation():
