@@ -35,6 +35,7 @@ EXPORTS = (
     "flint_moe_routing", "flint_moe_intermediate", "flint_moe_error_word", "flint_moe_destroy",
     "flint_moe_status_string", "flint_moe_set_stage_events", "flint_moe_stage_count", "flint_moe_stage_name",
     "flint_moe_route_noalloc", "flint_residual_rmsnorm", "flint_moe_stack_forward",
+    "flint_quantize_int4_g128", "flint_quantize_nvfp4",
 )
 
 
@@ -78,6 +79,8 @@ def _load():
         "flint_moe_route_noalloc": (I, [V, V, I, I, I, ctypes.c_float, V, V, V]),
         "flint_residual_rmsnorm": (I, [V, V, I, ctypes.c_float, V, V]),
         "flint_moe_stack_forward": (I, [P(V), I, V, I, ctypes.c_float, V, V, V]),
+        "flint_quantize_int4_g128": (I, [V, ctypes.c_longlong, I, I, V, V, V]),
+        "flint_quantize_nvfp4": (I, [V, I, I, I, V, V, V, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -146,6 +149,20 @@ def flint_moe_stack_forward(handles, x: int, T: int, eps: float, z: int, y: int,
     _check(_lib.flint_moe_stack_forward(arr, len(handles), ctypes.c_void_p(x), int(T), ctypes.c_float(eps),
                                         ctypes.c_void_p(z), ctypes.c_void_p(y), ctypes.c_void_p(stream)),
            "flint_moe_stack_forward")
+
+
+def flint_quantize_int4_g128(w: int, rows: int, cols: int, rotate: bool, codes: int, scales: int,
+                             stream: int = 0) -> None:
+    _check(_lib.flint_quantize_int4_g128(ctypes.c_void_p(w), int(rows), int(cols), 1 if rotate else 0,
+                                         ctypes.c_void_p(codes), ctypes.c_void_p(scales), ctypes.c_void_p(stream)),
+           "flint_quantize_int4_g128")
+
+
+def flint_quantize_nvfp4(w: int, n_mats: int, rows: int, cols: int, codes: int, scales: int, tscale: int,
+                         stream: int = 0) -> None:
+    _check(_lib.flint_quantize_nvfp4(ctypes.c_void_p(w), int(n_mats), int(rows), int(cols), ctypes.c_void_p(codes),
+                                     ctypes.c_void_p(scales), ctypes.c_void_p(tscale), ctypes.c_void_p(stream)),
+           "flint_quantize_nvfp4")
 
 
 def flint_moe_destroy(h: int) -> None:

@@ -8,7 +8,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libflint_moe.so")
-SOURCES = ["api.cu", "route.cu", "decode.cu", "prefill.cu", "stack.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "route.cu", "decode.cu", "prefill.cu", "stack.cu", "noalloc.cu", "quant.cu"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
               "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]
 
@@ -33,7 +33,7 @@ def up_to_date() -> bool:
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(ROOT, "include", "flint_moe.h")]
+    deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(ROOT, "include", f) for f in ("flint_moe.h", "flint_quant.h")]
     return all(os.path.getmtime(d) <= t for d in deps)
 
 

@@ -54,6 +54,7 @@ FMT_NVFP4 = "nvfp4"
 
 # stream tags, one per component
 _TAG_ROUTER, _TAG_GU_CODES, _TAG_GU_SCALES, _TAG_DN_CODES, _TAG_DN_SCALES, _TAG_SH_GU, _TAG_SH_DN = range(7)
+_TAG_MASTER_GU, _TAG_MASTER_DN, _TAG_MASTER_OUT = range(7, 10)
 
 
 def _rng(*key: int) -> np.random.Generator:
@@ -120,6 +121,23 @@ def make_layer(E: int, fmt: str = FMT_INT4, *, H: int = H_DEFAULT, I: int = I_DE
     L["sh_gu"] = _bf16_normal(_rng(seed, _TAG_SH_GU), (2 * Is, H), W_STD)
     L["sh_dn"] = _bf16_normal(_rng(seed, _TAG_SH_DN), (H, Is), W_STD)
     return L
+
+
+def make_master_weights(E: int, *, H: int = H_DEFAULT, I: int = I_DEFAULT, seed: int = SEED_WEIGHTS,
+                        outliers: int = 0) -> dict:
+    """bf16 expert weights before quantisation (the input of the weight-preparation entry points):
+    gu u16 [E][2I][H] (gate rows then up rows) and dn u16 [E][H][I], normal with std W_STD; with
+    `outliers` > 0 that many entries per row are set to +-30 W_STD (heavy-tailed rows)."""
+    out = {}
+    for name, tag, shape in (("gu", _TAG_MASTER_GU, (E, 2 * I, H)), ("dn", _TAG_MASTER_DN, (E, H, I))):
+        w = _rng(seed, tag).standard_normal(size=shape, dtype=np.float32) * np.float32(W_STD)
+        if outliers:
+            r = _rng(seed, _TAG_MASTER_OUT, tag)
+            idx = r.integers(0, shape[-1], size=shape[:-1] + (outliers,))
+            val = r.choice(np.float32([-30.0, 30.0]), size=idx.shape) * np.float32(W_STD)
+            np.put_along_axis(w, idx, val, axis=-1)
+        out[name] = f32_to_bf16_bits(w)
+    return out
 
 
 def x_row(r: int, d: int, H: int = H_DEFAULT, skew: bool = False) -> np.ndarray:

@@ -110,3 +110,32 @@ def test_status_strings():
     for s in range(7):
         assert B.flint_moe_status_string(s)
     assert "unknown" in B.flint_moe_status_string(99)
+
+
+def test_quantiser_entry_points_check_arguments_on_the_host():
+    V, LL = ctypes.c_void_p, ctypes.c_longlong
+    q4 = "flint_quantize_int4_g128"
+    bad = [
+        (V(0x1000), LL(4), 200, 1, V(0x2000), V(0x3000), V(0)),        # cols not a multiple of 128
+        (V(0x1000), LL(-1), 256, 1, V(0x2000), V(0x3000), V(0)),       # negative rows
+        (V(0x1000), LL(4), 256, 2, V(0x2000), V(0x3000), V(0)),        # rotate is 0 or 1
+        (V(0x1008), LL(4), 256, 1, V(0x2000), V(0x3000), V(0)),        # w not 16-byte aligned
+        (V(0x1000), LL(4), 256, 1, V(0x2001), V(0x3000), V(0)),        # codes not 2-byte aligned
+        (V(0), LL(4), 256, 1, V(0x2000), V(0x3000), V(0)),             # null input
+    ]
+    for args in bad:
+        assert B.raw_status(q4, *args) == B.FLINT_ERR_INVALID_ARG, args
+    assert B.raw_status(q4, V(0), LL(0), 256, 1, V(0), V(0), V(0)) == B.FLINT_OK       # rows = 0: no-op
+    nv = "flint_quantize_nvfp4"
+    bad = [
+        (V(0x1000), 2, 4, 24, V(0x2000), V(0x3000), V(0x4000), V(0)),  # cols not a multiple of 16
+        (V(0x1000), -1, 4, 32, V(0x2000), V(0x3000), V(0x4000), V(0)), # negative count
+        (V(0x1000), 70000, 4, 32, V(0x2000), V(0x3000), V(0x4000), V(0)),  # more Linears than one grid row holds
+        (V(0x1000), 2, 0, 32, V(0x2000), V(0x3000), V(0x4000), V(0)),  # empty Linears
+        (V(0x1000), 2, 4, 32, V(0x2004), V(0x3000), V(0x4000), V(0)),  # codes not 8-byte aligned
+        (V(0x1000), 2, 4, 32, V(0x2000), V(0x3000), V(0x4002), V(0)),  # tscale not 4-byte aligned
+        (V(0x1000), 2, 4, 32, V(0x2000), V(0x3000), V(0), V(0)),       # no tscale
+    ]
+    for args in bad:
+        assert B.raw_status(nv, *args) == B.FLINT_ERR_INVALID_ARG, args
+    assert B.raw_status(nv, V(0), 0, 4, 32, V(0), V(0), V(0), V(0)) == B.FLINT_OK     # no Linears: no-op
