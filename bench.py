@@ -48,6 +48,9 @@ WORKLOADS = {
 }
 # stacks: layers of the workload (layer l drawn with seed 1000 + l); T tokens decode through all of them
 STACK_LAYERS = {"stack47_int4": 47}
+# weight preparation: the bf16 gate|up and down banks of all E experts quantised once per step
+QUANT_WORKLOADS = {"quant_int4": (256, "int4"), "quant_nvfp4": (256, "nvfp4")}
+QUANT_SEED = 7
 STACK_EPS = 1e-6
 
 
@@ -56,10 +59,12 @@ def parse_args():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=2000)
     p.add_argument("--warmup", type=int, default=20)
-    p.add_argument("--workload", default="decode_int4", choices=sorted(WORKLOADS))
+    p.add_argument("--workload", default="decode_int4", choices=sorted(WORKLOADS) + sorted(QUANT_WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-extras", action="store_true", help="skip the per-T decode and prefill side measurements")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU-oracle baseline sample")
+    p.add_argument("--quant-experts", type=int, default=0,
+                   help="quant_* workloads: experts per step (default: all of the workload's); for small profiles")
     return p.parse_args()
 
 
@@ -139,7 +144,7 @@ def ncu_traffic(kernel: str, workload: str):
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
-    cur = source_hash()
+    cur = source_hash(TRAFFIC_SOURCES.get(kernel))
     for line in open(path):
         line = line.split("#")[0].strip()
         if not line:
@@ -150,11 +155,21 @@ def ncu_traffic(kernel: str, workload: str):
     return None
 
 
-def source_hash() -> str:
+# the translation unit of each kernel whose DRAM traffic is recorded (profiles/ncu_traffic.txt): a
+# recorded figure stands while these files are unchanged
+TRAFFIC_SOURCES = {
+    "gate_up": ("common.cuh", "decode.cu", "frag.cuh", "kernels.cuh"),
+    "gu_routed": ("common.cuh", "kernels.cuh", "prefill.cu"),
+    "quant": ("quant.cu",),
+}
+
+
+def source_hash(files=None) -> str:
+    """sha256 (first 12 hex digits) over the named kernel sources (default: all of csrc), in name order."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_routed_expert_sigmoid_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in sorted(files if files is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:12]
@@ -434,6 +449,18 @@ def cpu_baseline(args, L, x_bits, E) -> dict:
 def run_reference(args) -> dict:
     from bit_routed_expert_sigmoid_b200 import synthetic as S
     from oracle import flint_moe_ref as R
+    if args.workload in QUANT_WORKLOADS:
+        E, fmt = QUANT_WORKLOADS[args.workload]
+        bps, nbytes = quant_reference_sample(fmt, min(args.cpu_seconds, 30.0))
+        v = round(bps / 1e9, 6)
+        return {"impl": "reference", "metric": "weight preparation: bf16 GB/s quantised (all experts' gate|up "
+                "and down banks)", "value": v, "unit": "GB/s", "n_gpus": 1, "steps": 1, "warmup": 0,
+                "ms_per_step": round(nbytes / bps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32 decisions", "data": "synthetic",
+                "config": {"workload": f"{args.workload}: E={E} experts bf16 -> {fmt}", "E": E, "fmt": fmt},
+                "cpu_baseline": {"value": v, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                                 "sample": f"oracle quantiser on 64 rows x {H}, {nbytes / 1e6:.1f} MB"},
+                "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     E, fmt, T, skew = WORKLOADS[args.workload]
     if args.workload in STACK_LAYERS:
         # bounded sample: whole oracle stack steps on the first layers, the per-layer time scaled
@@ -479,6 +506,148 @@ def run_reference(args) -> dict:
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def quant_bytes_per_weight(fmt: str) -> float:
+    """Algorithmic bytes per weight of the weight preparation: the bf16 read, the 4-bit code and the
+    scale share (int4: a bf16 per 128; NVFP4: an E4M3 per 16, its amax pass re-reads the input)."""
+    return 2.0 + 0.5 + (2.0 / 128 if fmt == "int4" else 1.0 / 16 + 2.0)
+
+
+def quant_reference_sample(fmt: str, seconds: float):
+    """The oracle quantiser on whole rows of one bank, for about `seconds`: bf16 bytes per second."""
+    from oracle import quant_ref as Q
+    rng = np.random.default_rng(QUANT_SEED)
+    w = (rng.standard_normal((64, H)) * 0.02).astype(np.float32)
+    wb = ((w.view(np.uint32).astype(np.uint64) + 0x7FFF + ((w.view(np.uint32) >> 16) & 1)) >> 16).astype(np.uint16)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        if fmt == "int4":
+            Q.quantize_int4_g128(wb, rotate=True)
+        else:
+            Q.quantize_nvfp4(wb)
+        done += wb.nbytes
+        if time.perf_counter() - t0 >= seconds:
+            break
+    return done / (time.perf_counter() - t0), done
+
+
+def run_quant(args) -> dict:
+    """Weight preparation of every expert of a layer: bf16 gate|up [E][2I][H] and down [E][H][I]
+    (normal, std 0.02, drawn on the device from a seeded generator) into the layer's format."""
+    import torch
+
+    from bit_routed_expert_sigmoid_b200 import binding as B
+
+    E, fmt = QUANT_WORKLOADS[args.workload]
+    if args.quant_experts > 0:
+        E = min(E, args.quant_experts)
+    I = 512
+    dev = "cuda:0"
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(QUANT_SEED)
+    gu = (torch.randn((E, 2 * I, H), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    dn = (torch.randn((E, H, I), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    n_w = gu.numel() + dn.numel()
+    if fmt == "int4":
+        gc = torch.empty((E, 2 * I, H // 2), dtype=torch.uint8, device=dev)
+        gs = torch.empty((E, 2 * I, H // 128), dtype=torch.int16, device=dev)
+        dc = torch.empty((E, H, I // 2), dtype=torch.uint8, device=dev)
+        ds = torch.empty((E, H, I // 128), dtype=torch.int16, device=dev)
+
+        def step(w_gu=gu, w_dn=dn, e=E):
+            B.flint_quantize_int4_g128(w_gu.data_ptr(), e * 2 * I, H, True, gc.data_ptr(), gs.data_ptr(), 0)
+            B.flint_quantize_int4_g128(w_dn.data_ptr(), e * H, I, True, dc.data_ptr(), ds.data_ptr(), 0)
+        launches = 2
+    else:
+        gc = torch.empty((2 * E, I, H // 2), dtype=torch.uint8, device=dev)
+        gs = torch.empty((2 * E, I, H // 16), dtype=torch.uint8, device=dev)
+        gt = torch.empty((2 * E,), dtype=torch.float32, device=dev)
+        dc = torch.empty((E, H, I // 2), dtype=torch.uint8, device=dev)
+        ds = torch.empty((E, H, I // 16), dtype=torch.uint8, device=dev)
+        dt = torch.empty((E,), dtype=torch.float32, device=dev)
+
+        def step(w_gu=gu, w_dn=dn, e=E):
+            B.flint_quantize_nvfp4(w_gu.data_ptr(), 2 * e, I, H, gc.data_ptr(), gs.data_ptr(), gt.data_ptr(), 0)
+            B.flint_quantize_nvfp4(w_dn.data_ptr(), e, H, I, dc.data_ptr(), ds.data_ptr(), dt.data_ptr(), 0)
+        launches = 6
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.perf_counter()
+    ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    ms_per_step = float(np.mean(ms))
+    in_bytes = 2 * n_w
+    value = in_bytes / (ms_per_step * 1e-3) / 1e9
+    peaks = measured_peaks()
+    ab = quant_bytes_per_weight(fmt) * n_w
+    achieved = ab / (ms_per_step * 1e-3) / 1e9
+    kern = "quant_int4_kernel" if fmt == "int4" else "quant_amax_kernel + quant_nvfp4_kernel"
+    roofline = {"bound": "hbm", "kernel": kern, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": ncu_traffic("quant", args.workload),
+                "algorithmic_bytes": int(ab), "peak_source": peaks["source"] + " (burst copy)"}
+
+    # end to end through the public API on a 16-expert slice: pinned host bf16 in, codes and scales out
+    Ee = min(16, E)
+    h_gu = gu[:Ee].cpu().pin_memory()
+    h_dn = dn[:Ee].cpu().pin_memory()
+    d_gu, d_dn = torch.empty_like(gu[:Ee]), torch.empty_like(dn[:Ee])
+    outs = [t[: (2 * Ee if (fmt == "nvfp4" and t is gc) else Ee)] for t in (gc, dc)]
+    h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+
+    def e2e_step():
+        d_gu.copy_(h_gu, non_blocking=True)
+        d_dn.copy_(h_dn, non_blocking=True)
+        step(d_gu, d_dn, Ee)
+        for o, ho in zip(outs, h_out):
+            ho.copy_(o, non_blocking=True)
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    k = max(3, min(args.steps, 20))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(k):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / k
+    e_in = 2 * (h_gu.numel() + h_dn.numel())
+    e2e = {"value": round(e_in / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": int(e_in),
+           "d2h_bytes_per_step": int(sum(o.numel() * o.element_size() for o in outs)),
+           "ms_per_step": round(e2e_ms, 4), "slice": f"{Ee} of the {E} experts (codes read back, scales not)"}
+    clk = clocks.stop()
+    cpu_bps, cpu_bytes = quant_reference_sample(fmt, args.cpu_seconds)
+    return {
+        "metric": "weight preparation: bf16 GB/s quantised (all experts' gate|up and down banks)",
+        "value": round(value, 1), "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 decisions (IEEE, fixed order) from bf16 input" + (", 128-wide Hadamard rotation" if fmt == "int4" else ""),
+        "data": "synthetic (seeded normal bf16 weights, std 0.02, drawn on the device)",
+        "config": {"workload": f"{args.workload}: E={E} experts x (gate|up {2 * I}x{H}, down {H}x{I}) bf16 -> {fmt}",
+                   "E": E, "fmt": fmt, "weights": int(n_w),
+                   "l2": f"not flushed: {in_bytes / 1e9:.2f} GB of input per step, larger than the 126 MB L2",
+                   "parallelism": "single GPU"},
+        "roofline": roofline, "e2e": e2e, "gpu_launches": launches * args.steps, "clocks": clk,
+        "cpu_baseline": {"value": round(cpu_bps / 1e9, 6), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"fp32-decision oracle quantiser on 64 rows x {H} bf16, {cpu_bytes / 1e6:.1f} MB "
+                                   f"in {args.cpu_seconds:.0f} s"},
+        "wall_s_timed_region": round(wall1 - wall0, 4),
+    }
 
 
 def run_stack(args) -> dict:
@@ -625,6 +794,10 @@ def main():
     if args.workload in STACK_LAYERS:
         if rank == 0:
             print(json.dumps(run_stack(args)), flush=True)
+        return
+    if args.workload in QUANT_WORKLOADS:
+        if rank == 0:
+            print(json.dumps(run_quant(args)), flush=True)
         return
     res = run_ours(args, rank, world, local_rank)
     if rank == 0:

@@ -28,18 +28,13 @@ __device__ __forceinline__ uint32_t f32_to_bf16_rne(float x) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// int4 g128: one warp per (row, 128-group); lane l holds elements 4l .. 4l+3 of the group.
-__global__ void __launch_bounds__(256) quant_int4_kernel(const uint16_t* __restrict__ w, long long rows, int cols,
-                                                          int rotate, uint8_t* __restrict__ codes,
-                                                          uint16_t* __restrict__ scales) {
-  const int lane = threadIdx.x & 31;
-  const long long gw = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int ngrp = cols / 128;
-  if (gw >= rows * ngrp) return;
-  const long long row = gw / ngrp;
-  const int g = static_cast<int>(gw - row * ngrp);
-  const uint2 raw = *reinterpret_cast<const uint2*>(w + row * cols + g * 128 + 4 * lane);
-  float v[4] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y)};
+// int4 g128: a warp takes kGroupsPerWarp consecutive (row, 128-group) units, all of whose loads it
+// issues before any arithmetic (HBM needs several KB in flight per SM); lane l holds elements
+// 4l .. 4l+3 of a group.
+constexpr int kGroupsPerWarp = 4;
+
+__device__ __forceinline__ void quant_int4_group(float (&v)[4], int lane, bool rotate, uint32_t& sb_out,
+                                                 uint32_t& packed) {
   if (rotate) {
     // Sylvester butterfly, stages h = 1, 2 (inside the lane) then 4 .. 64 (partner lane l ^ h/4):
     // the pair (i, i + h), i & h = 0, becomes (v_i + v_i+h, v_i - v_i+h)
@@ -72,15 +67,46 @@ __global__ void __launch_bounds__(256) quant_int4_kernel(const uint16_t* __restr
   for (int m = 16; m > 0; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
   const uint32_t sb = f32_to_bf16_rne(__fdiv_rn(mx, 7.0f));
   const float s = __uint_as_float(sb << 16);
-  uint32_t packed = 0;
+  const float rs = s > 0.f ? __frcp_rn(s) : 0.f;            // correctly rounded reciprocal
+  packed = 0;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    int q = 0;
-    if (s > 0.f) q = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(v[j], s)), -8.f), 7.f));
+    const int q = static_cast<int>(fminf(fmaxf(rintf(__fmul_rn(v[j], rs)), -8.f), 7.f));
     packed |= (static_cast<uint32_t>(q) & 0xFu) << (4 * j);
   }
-  *reinterpret_cast<uint16_t*>(codes + row * (cols / 2) + g * 64 + 2 * lane) = static_cast<uint16_t>(packed);
-  if (lane == 0) scales[row * ngrp + g] = static_cast<uint16_t>(sb);
+  sb_out = sb;
+}
+
+__global__ void __launch_bounds__(256) quant_int4_kernel(const uint16_t* __restrict__ w, long long rows, int cols,
+                                                          int rotate, uint8_t* __restrict__ codes,
+                                                          uint16_t* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const long long u0 = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kGroupsPerWarp;
+  const int ngrp = cols / 128;
+  const long long units = rows * ngrp;
+  if (u0 >= units) return;
+  uint2 raw[kGroupsPerWarp];
+#pragma unroll
+  for (int k = 0; k < kGroupsPerWarp; ++k) {
+    const long long u = u0 + k;
+    if (u < units) {
+      const long long row = u / ngrp;
+      const int g = static_cast<int>(u - row * ngrp);
+      raw[k] = __ldg(reinterpret_cast<const uint2*>(w + row * cols + g * 128 + 4 * lane));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kGroupsPerWarp; ++k) {
+    const long long u = u0 + k;
+    if (u >= units) break;                                // warp-uniform
+    const long long row = u / ngrp;
+    const int g = static_cast<int>(u - row * ngrp);
+    float v[4] = {bf16_lo(raw[k].x), bf16_hi(raw[k].x), bf16_lo(raw[k].y), bf16_hi(raw[k].y)};
+    uint32_t sb, packed;
+    quant_int4_group(v, lane, rotate != 0, sb, packed);
+    *reinterpret_cast<uint16_t*>(codes + row * (cols / 2) + g * 64 + 2 * lane) = static_cast<uint16_t>(packed);
+    if (lane == 0) scales[row * ngrp + g] = static_cast<uint16_t>(sb);
+  }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -93,15 +119,20 @@ __global__ void __launch_bounds__(256) quant_amax_kernel(const uint16_t* __restr
   const int mat = blockIdx.y;
   const uint4* src = reinterpret_cast<const uint4*>(w + static_cast<long long>(mat) * per_mat);
   const long long units = per_mat / 8;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   uint32_t m = 0;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < units;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const uint4 q = __ldg(src + i);
-    const uint32_t ws[4] = {q.x, q.y, q.z, q.w};
+  for (long long i0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < units; i0 += 4 * stride) {
+    uint4 q[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      m = max(m, (ws[k] << 16) & 0x7FFFFFFFu);
-      m = max(m, ws[k] & 0x7FFF0000u);
+    for (int r = 0; r < 4; ++r) q[r] = i0 + r * stride < units ? __ldg(src + i0 + r * stride) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const uint32_t ws[4] = {q[r].x, q[r].y, q[r].z, q[r].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        m = max(m, (ws[k] << 16) & 0x7FFFFFFFu);
+        m = max(m, ws[k] & 0x7FFF0000u);
+      }
     }
   }
 #pragma unroll
@@ -164,10 +195,11 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(const uint16_t* __rest
   }
   const uint32_t sb = e4m3_rne_pos(__fdiv_rn(bm, __fmul_rn(6.0f, ts)));
   const float d = __fmul_rn(e4m3_value(sb), ts);
+  const float rd = d > 0.f ? __frcp_rn(d) : 0.f;            // correctly rounded reciprocal
   uint32_t lo = 0, hi = 0;
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
-    const uint32_t c = d > 0.f ? e2m1_rne(__fdiv_rn(v[k], d)) : 0u;
+    const uint32_t c = d > 0.f ? e2m1_rne(__fmul_rn(v[k], rd)) : 0u;
     if (k < 8) lo |= c << (4 * k);
     else hi |= c << (4 * (k - 8));
   }
@@ -193,7 +225,7 @@ extern "C" flint_status flint_quantize_int4_g128(const void* w, long long rows, 
   if (rows == 0) return FLINT_OK;
   if (!w || !codes || !scales || !aligned(w, 16) || !aligned(codes, 2) || !aligned(scales, 2))
     return FLINT_ERR_INVALID_ARG;
-  const long long warps = rows * (cols / 128);
+  const long long warps = (rows * (cols / 128) + kGroupsPerWarp - 1) / kGroupsPerWarp;
   const long long grid = (warps + 7) / 8;
   if (grid > 0x7FFFFFFFLL) return FLINT_ERR_INVALID_ARG;
   quant_int4_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
@@ -216,7 +248,7 @@ extern "C" flint_status flint_quantize_nvfp4(const void* w, int n_mats, int rows
   uint32_t* amax = reinterpret_cast<uint32_t*>(tscale);        // scratch until quant_tscale_kernel
   if (cudaMemsetAsync(amax, 0, sizeof(uint32_t) * n_mats, s) != cudaSuccess) return FLINT_ERR_CUDA;
   const long long units = per_mat / 8;
-  const long long gx = (units + 1023) / 1024;
+  const long long gx = (units + 4095) / 4096;
   quant_amax_kernel<<<dim3(static_cast<unsigned>(gx < 4096 ? gx : 4096), n_mats), 256, 0, s>>>(
       static_cast<const uint16_t*>(w), per_mat, amax);
   quant_nvfp4_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(

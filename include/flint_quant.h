@@ -4,14 +4,15 @@
  * int4 g128 with rotation (Aijuus/flint-w4exp, summary table, weights row: codes i4, group 128, bf16
  * scale, 128-wide Hadamard rotation; the container is converted from the bf16 checkpoint, same page,
  * "Serving it"). The stored matrix is W blockdiag(Hn), Hn = H_128 / sqrt(128), so every 128-segment
- * of a row is rotated and then rounded: per segment s = bf16(max|r| / 7) and code = clamp(rint(r / s),
- * -8, 7).
+ * of a row is rotated and then rounded: per segment s = bf16(max|r| / 7) and code = clamp(rint(r * (1/s)),
+ * -8, 7), 1/s the correctly rounded fp32 reciprocal.
  *
  * NVFP4 (kekzle/Flint-NVFP4, "What is in the files": E2M1 codes two per byte, E4M3 scale per 16
  * columns, F32 tensor scale per Linear; value = code x block scale x tensor scale): tensor scale =
  * amax / (6 * 448) (1 for an all-zero Linear); block scale = E4M3(block amax / (6 * tensor scale)),
- * nearest even, saturated at 448; code = E2M1(w / (block scale * tensor scale)), nearest grid value,
- * ties to the even code, saturated at 6, sign from the sign bit of the quotient.
+ * nearest even, saturated at 448; code = E2M1(w * (1 / (block scale * tensor scale))), the reciprocal
+ * correctly rounded in fp32; nearest grid value, ties to the even code, saturated at 6, sign from the
+ * sign bit of the product.
  *
  * Every step is IEEE fp32 with one rounding per operation, in a fixed order (the rotation is the
  * Sylvester butterfly by stages 1, 2, 4, ..., 64 followed by one multiplication by the fp32 nearest

@@ -13,14 +13,15 @@ What the pages fix, and the readings taken where they are silent:
   round-to-nearest conversion, same page, "Serving it" and the 11.7 % error paragraph). The stored
   matrix is the rotated one, W_q = W blockdiag(Hn) with Hn = H_128 / sqrt(128), so the quantiser
   rotates every 128-segment of a row and rounds the result. Readings: the scale is symmetric,
-  s = bf16(max |r| / 7) (codes -7..7, -8 unused), and a code is rint(r / s) clamped to [-8, 7].
+  s = bf16(max |r| / 7) (codes -7..7, -8 unused), and a code is rint(r * (1/s)) clamped to [-8, 7],
+  with 1/s the correctly rounded fp32 reciprocal (the quotient formed as one multiplication).
 * NVFP4 (kekzle/Flint-NVFP4, "What is in the files": E2M1 codes two per byte, an E4M3 scale per 16
   columns, an F32 tensor scale per Linear; value = code x block scale x tensor scale). Readings:
   tensor scale = amax / (6 * 448), the largest magnitude of the Linear over the largest products of
   the two formats; block scale = E4M3(block amax / (6 * tensor scale)), rounded to nearest even and
-  saturated at 448; code = E2M1(w / (block scale * tensor scale)), nearest grid value, ties to the
-  even code, saturated at 6, sign from the sign bit of the quotient. An all-zero Linear gets tensor
-  scale 1.
+  saturated at 448; code = E2M1(w * (1 / (block scale * tensor scale))), nearest grid value, ties
+  to the even code, saturated at 6, sign from the sign bit of the product (the reciprocal correctly
+  rounded in fp32, so the quotient is one multiplication). An all-zero Linear gets tensor scale 1.
 
 Precision. A quantiser decides integers (codes) from floating point, so this oracle takes every
 decision in the precision the kernels use, IEEE fp32 with round-to-nearest for each operation, and
@@ -81,7 +82,7 @@ def fwht128_f32(v: np.ndarray) -> np.ndarray:
 def quantize_int4_g128(w_bf16, rotate: bool = True) -> dict:
     """bf16 matrix [N][K] (bit patterns) -> {codes u8 [N][K/2], scales bf16 bits [N][K/128]}.
     r = the rotated row (or the row itself); per 128-group: s = bf16(max|r| / 7) and
-    c = clamp(rint(r / s), -8, 7), two's complement, low nibble = even K index; s = 0 gives c = 0."""
+    c = clamp(rint(r * fp32(1/s)), -8, 7), two's complement, low nibble = even K index; s = 0 gives c = 0."""
     w = bf16_to_f32(w_bf16)
     N, K = w.shape
     assert K % GROUP == 0
@@ -91,7 +92,8 @@ def quantize_int4_g128(w_bf16, rotate: bool = True) -> dict:
     sb = f32_to_bf16_rne(m / np.float32(7.0))                        # fp32 division, then bf16
     s = bf16_to_f32(sb)
     with np.errstate(divide="ignore", invalid="ignore"):
-        q = np.rint(g / s[..., None])                                # fp32 division, ties to even
+        rs = np.float32(1.0) / s                                     # correctly rounded reciprocal
+        q = np.rint(g * rs[..., None])                               # fp32 product, ties to even
     q = np.where(s[..., None] > 0, q, 0.0)
     q = np.clip(q, -8, 7).astype(np.int64).reshape(N, K)
     nib = (q & 0xF).astype(np.uint8)
@@ -146,7 +148,7 @@ def e4m3_rne_pos(x) -> np.ndarray:
 def quantize_nvfp4(w_bf16) -> dict:
     """bf16 Linear [N][K] (bit patterns) -> {codes u8 [N][K/2], scales e4m3 [N][K/16], tscale f32}.
     fp32 throughout: ts = amax / 2688 (1 for an all-zero Linear); per 16-block sb = E4M3(bm / (6 ts))
-    with 6 ts one fp32 product; d = value(sb) * ts; code = E2M1(w / d) (0 where d = 0)."""
+    with 6 ts one fp32 product; d = value(sb) * ts; code = E2M1(w * fp32(1/d)) (0 where d = 0)."""
     w = bf16_to_f32(w_bf16)
     N, K = w.shape
     assert K % BLOCK == 0
@@ -159,7 +161,8 @@ def quantize_nvfp4(w_bf16) -> dict:
     sv = R.e4m3fn_to_f64(sb).astype(np.float32)                       # exact
     d = (sv * ts).astype(np.float32)                                  # fp32 product
     with np.errstate(divide="ignore", invalid="ignore"):
-        x = blk / d[..., None]                                        # fp32 division
+        rd = np.float32(1.0) / d                                      # correctly rounded reciprocal
+        x = blk * rd[..., None]                                       # fp32 product
     x = np.where(d[..., None] > 0, x, np.float32(0.0)).astype(np.float32)
     nib = e2m1_rne(x).reshape(N, K)
     codes = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
