@@ -233,6 +233,28 @@ class ClockSampler:
                 "samples": len(sm), "power_w_max": max(power) if power else None}
 
 
+# --------------------------------------------------------------------------------------------- ranks
+
+def rank_first_row(rank: int, T: int) -> int:
+    """Weak scaling: rank r decodes its own T token rows, [r*T, (r+1)*T) of the seeded stream."""
+    return rank * T
+
+
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The largest of the ranks' values (every rank takes part; returns the input with one rank)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, T: int, steps: int, max_total_ms: float) -> float:
+    """Whole-job throughput: the tokens of every rank over the slowest rank's timed region."""
+    return world * T * steps / (max_total_ms / 1e3)
+
+
 # --------------------------------------------------------------------------------------------- ours
 
 def run_ours(args, rank: int, world: int, local_rank: int):
@@ -257,7 +279,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     layer = FlintMoELayer(L, t_max=max(t_max, 2048 if not args.no_extras else t_max), device=dev_name)
     # each rank takes its own batch of token rows (weak scaling: T tokens per GPU)
     redraws = S.redraw_table(E, skew=skew)
-    x_bits = S.make_x(T, skew=skew, redraws=redraws, first_row=0 if world == 1 else 0)
+    x_bits = S.make_x(T, skew=skew, redraws=redraws, first_row=rank_first_row(rank, T))
     x = x_to_device(x_bits, dev_name)
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev_name)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev_name)
@@ -293,13 +315,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     step_ms = timed_steps(fwd, args.steps)
     barrier()
     wall1 = time.perf_counter()
-    total_ms = float(sum(step_ms))
-    if dist is not None:
-        tt = torch.tensor([total_ms], device=dev_name)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(float(sum(step_ms)), dist, dev_name)
     ms_per_step = total_ms / args.steps
-    value = world * T * args.steps / (total_ms / 1e3)
+    value = job_tokens_per_s(world, T, args.steps, total_ms)
 
     # per-kernel times of the same forward (instrumented pass)
     n_st = B.flint_moe_stage_count(layer.handle, T)
