@@ -105,7 +105,7 @@ def stage_bytes(name: str, E: int, fmt: str, T: int, K: int, n_active: int) -> i
                 + T * H * 2,
         # larger T: one kernel per step (tensor-core path)
         "router_logits": E * H * 2 + T * H * 2 + T * E * 4,
-        "topk": T * E * 4 + P * 8,
+        "topk": 4 * T * E * 4 + T * E * 4 + P * 8,              # 4 partial-logit slices in, logits out
         "permute": P * 4 * 3 + (E + 1) * 4,
         "xq": T * H * 2 + P * H * 2 + P * 4,
         "gu_routed": n_active * eb_gu + P * H * 2 + P * I * 2,
