@@ -164,14 +164,23 @@ TRAFFIC_SOURCES = {
 }
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without comments and with whitespace runs collapsed: what compiles."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_hash(files=None) -> str:
-    """sha256 (first 12 hex digits) over the named kernel sources (default: all of csrc), in name order."""
+    """sha256 (first 12 hex digits) over the code of the named kernel sources (default: all of csrc), in
+    name order; comments and layout do not count, so a figure survives edits that change no code."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_routed_expert_sigmoid_b200", "csrc")
     for fn in sorted(files if files is not None else os.listdir(csrc)):
-        with open(os.path.join(csrc, fn), "rb") as f:
-            h.update(fn.encode() + f.read())
+        with open(os.path.join(csrc, fn), encoding="utf-8") as f:
+            h.update(fn.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:12]
 
 

@@ -2,23 +2,27 @@
 // cores (tcgen05.mma, fp32 accumulators in tensor memory).
 //
 // Routed experts (pf_routed_kernel). The permuted rows of one expert are its tokens; a tile is
-// (expert, a chunk of up to 128 of those rows, a pair of 128-row weight blocks): for gate|up the
+// (expert, a chunk of up to 64 of those rows, a pair of 128-row weight blocks): for gate|up the
 // gate rows [128r, 128r+128) and the matching up rows, for down the output rows [256r, 256r+128)
 // and [256r+128, 256r+256). One persistent CTA per SM walks the tiles; its warps specialise:
 //   warp 0       TMA copies of the 4-bit codes, 128 K per stage, into a shared-memory ring
 //   warp 3       TMA copies of the chunk's activation rows (fp16, stored per permuted row so that
 //                an expert's rows are contiguous; 128-byte swizzled K-major, 16-row boxes) into a ring
 //   warps 4..    dequantisation (8 or 16 warps): a thread owns one weight row of one block and both
-//                64-code halves of the stage, or one of them, turns those codes into exact fp16 (int4: code x bf16 group scale; NVFP4: E2M1 x E4M3) and
-//                writes them to tensor memory with tcgen05.st, where the MMA reads its A operand.
-//                A in tensor memory costs no shared-memory bandwidth, which a 128 x 48 MMA with A
-//                in shared memory would exhaust.
-//   warps 1, 2   one MMA-issuing thread per block (an MMA instruction takes ~45 cycles to issue, so
-//                two issuers keep N = 48 tiles near the tensor-core rate); D[128 x N] per block
+//                64-code halves of the stage, or one of them, turns those codes into exact fp16
+//                (int4: code x bf16 group scale; NVFP4: E2M1 x E4M3) and writes them to tensor
+//                memory with tcgen05.st, where the MMA reads its A operand. A in tensor memory costs
+//                no shared-memory bandwidth, which a 128 x 48 MMA with A in shared memory would
+//                exhaust.
+//   warps 1, 2   MMA issue, one warp per block with an elected lane issuing (an MMA instruction
+//                takes ~45 cycles to issue, so two issuers keep N = 48 tiles near the tensor-core
+//                rate); D[128 x N] per block, double-buffered
 //   last 4 warps epilogue: gate|up -> h = silu(g) u, int4: rotated per 128-segment by the Hadamard
 //                butterfly, stored fp16 in the order of the down operand; down -> o in fp16.
-// Every dependency is an mbarrier: TMA transaction counts, cp.async arrivals, tcgen05.commit
-// arrivals and thread arrivals; every wait is bounded and sets a timeout bit on expiry.
+// Every dependency is an mbarrier: TMA transaction counts, tcgen05.commit arrivals and thread
+// arrivals; every wait is bounded and sets a timeout bit on expiry. The routed down kernel is a
+// programmatic dependent of the gate|up kernel: its code copies start as soon as it has an SM, its
+// activation copies after griddepcontrol.wait.
 //
 // The shared expert (pf_shared_kernel) is a dense bf16 GEMM of the same shape of pipeline with the
 // weights and activations brought by TMA in the 128-byte swizzled layout and read by the MMA from
