@@ -342,3 +342,57 @@ def test_f64_to_bf16_rounding_matches_torch():
                         [0.0, -0.0, 1.0, 1.00390625, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -9]])
     ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     np.testing.assert_array_equal(R.f64_to_bf16_bits(x), ref)
+
+
+@pytest.mark.parametrize("top_k", [2, 3])
+def test_combine_pairs_each_weight_with_its_own_expert(top_k):
+    """The weighted combine, recomputed without the oracle's routing, permutation or rotation: a toy
+    int4 layer (E = 4, H = 256, I = 128) whose four experts differ, routed by brute force over every
+    k-subset, weighted through an explicit [T][E] routing matrix and summed by einsum. A weight paired
+    with the wrong slot (for example weights left in score order while the ids are sorted by id)
+    changes y here, because the experts and the weights all differ (midagedev/bloomery issue #632:
+    unbiased sigmoid top-k with the SelectedSumFloor; NInfer README, "What is inside": scores
+    renormalised)."""
+    scipy_linalg = pytest.importorskip("scipy.linalg")
+    E, H, I, Is, T = 4, 256, 128, 64, 24
+    L = S.make_layer(E, "int4", H=H, I=I, Is=Is, seed=21)
+    x_bits = S.make_x(T, H=H)
+    out = R.moe_forward(L, x_bits, top_k=top_k)
+
+    x = (x_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    # unrotated fp64 weights: the stored W_q times blockdiag(Hs), Hs from scipy's Sylvester matrix
+    Hs = scipy_linalg.hadamard(128) / math.sqrt(128)
+
+    def unrotate(Wq):
+        return np.concatenate([Wq[:, 128 * j:128 * (j + 1)] @ Hs for j in range(Wq.shape[1] // 128)], axis=1)
+
+    Wg = np.stack([unrotate(R.dequant_int4(L["gu_codes"][e, :I], L["gu_scales"][e, :I])) for e in range(E)])
+    Wu = np.stack([unrotate(R.dequant_int4(L["gu_codes"][e, I:], L["gu_scales"][e, I:])) for e in range(E)])
+    Wd = np.stack([unrotate(R.dequant_int4(L["dn_codes"][e], L["dn_scales"][e])) for e in range(E)])
+
+    # brute-force routing: the k-subset whose every score beats every score outside it
+    logits = x @ ((L["router_w"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)).T
+    s = 1.0 / (1.0 + np.exp(-logits))
+    Rm = np.zeros((T, E))
+    for t in range(T):
+        sel = [c for c in itertools.combinations(range(E), top_k)
+               if min(s[t, list(c)]) > max(s[t, [e for e in range(E) if e not in c]])]
+        assert len(sel) == 1
+        c = list(sel[0])
+        Rm[t, c] = s[t, c] / max(s[t, c].sum(), 2.0 ** -14)
+        # the oracle's slot k carries the weight of the expert in slot k
+        np.testing.assert_array_equal(out["ids"][t], sorted(c))
+        np.testing.assert_allclose(out["w"][t], Rm[t, out["ids"][t]], rtol=1e-14)
+    assert np.all(np.abs(np.diff(np.sort(Rm, axis=1), axis=1))[:, -top_k + 1:] > 1e-6)   # weights differ
+
+    silu = lambda z: z / (1.0 + np.exp(-z))  # noqa: E731
+    G = np.einsum("eih,th->eti", Wg, x)
+    U = np.einsum("eih,th->eti", Wu, x)
+    O = np.einsum("ehi,eti->eth", Wd, silu(G) * U)
+    routed = np.einsum("te,eth->th", Rm, O)
+    Sgu = (L["sh_gu"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    Sdn = (L["sh_dn"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    shared = (silu(x @ Sgu[:Is].T) * (x @ Sgu[Is:].T)) @ Sdn.T
+    np.testing.assert_allclose(out["y"], routed + shared, rtol=1e-11, atol=1e-13)
+    # the experts differ enough that pairing a weight with a neighbouring slot is visible
+    assert np.abs(O[0] - O[1]).max() > 1e-3
