@@ -18,26 +18,48 @@ def bf16(x):
     return S.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
 
 
-def test_inv_sqrt128_is_nearest_f32():
-    c = float(Q.F32_INV_SQRT128)
-    exact = 1.0 / math.sqrt(128.0)
-    up = float(np.nextafter(Q.F32_INV_SQRT128, np.float32(1)))
-    dn = float(np.nextafter(Q.F32_INV_SQRT128, np.float32(0)))
-    assert abs(c - exact) < abs(up - exact) and abs(c - exact) < abs(dn - exact)
-
-
-def test_butterfly_matches_dense_hadamard():
+def test_int4_brute_force_nearest_code():
+    # every code is the integer c in [-8, 7] nearest to r / s (ties to the even c), found by trying all 16
     rng = np.random.default_rng(1)
-    v = rng.standard_normal((7, 512)).astype(np.float32)
-    got = Q.fwht128_f32(v).astype(np.float64)
-    ref = R.rotate_segments(v.astype(np.float64))
-    # 7 butterfly stages and one multiplication, each rounding by at most half an fp32 ulp of a
-    # partial sum bounded by the segment's L1 norm
-    l1 = np.abs(v.reshape(7, 4, 128)).sum(-1, keepdims=True)
-    bound = np.repeat(l1, 128, axis=-1).reshape(7, 512) * 8 * 2.0 ** -24 / math.sqrt(128) + 1e-30
-    assert np.all(np.abs(got - ref) <= bound)
-    # the normalised transform is its own inverse
-    np.testing.assert_allclose(Q.fwht128_f32(Q.fwht128_f32(v)), v, rtol=0, atol=1e-5)
+    w = bf16(rng.standard_normal((9, 256)) * 0.03)
+    for rotate in (True, False):
+        out = Q.quantize_int4_g128(w, rotate=rotate)
+        r = R.rotate_segments(R.bf16_to_f64(w)) if rotate else R.bf16_to_f64(w)
+        s = np.repeat(R.bf16_to_f64(out["scales"]), 128, axis=1)
+        cands = np.arange(-8, 8)
+        dist = np.abs(r[..., None] - cands * s[..., None])
+        best = dist.min(-1, keepdims=True)
+        tie = np.where(dist == best, cands, 99)
+        even = np.where(tie % 2 == 0, tie, 99).min(-1)
+        want = np.where((tie < 99).sum(-1) > 1, even, np.where(tie < 99, tie, 99).min(-1))
+        np.testing.assert_array_equal(R.int4_values(out["codes"]), want)
+
+
+def test_int4_scale_is_bf16_of_max_over_7():
+    rng = np.random.default_rng(9)
+    w = bf16(rng.standard_normal((4, 512)) * 0.05)
+    out = Q.quantize_int4_g128(w, rotate=True)
+    r = R.rotate_segments(R.bf16_to_f64(w)).reshape(4, 4, 128)
+    m = np.abs(r).max(-1) / 7.0
+    want = torch.from_numpy(m).to(torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    # torch rounds through fp32 first; the two roundings agree unless m/7 sits within 2^-24 of a
+    # bf16 midpoint, which these draws do not
+    assert np.all(Q.int4_margins(w, True)["scale"] > 2.0 ** -20)
+    np.testing.assert_array_equal(out["scales"], want)
+
+
+def test_int4_margins_mark_the_rounding_boundaries():
+    # a group with max 7 * 2^-4 (scale 2^-4 exactly) and values at, near and far from half-steps
+    vals = np.zeros((1, 128))
+    vals[0, 0] = 7 * 2.0 ** -4
+    vals[0, 1] = 2.5 * 2.0 ** -4                      # exactly half-way: margin 0, ties to even (2)
+    vals[0, 2] = 3.0 * 2.0 ** -4                      # an integer: margin 0.5
+    vals[0, 3] = -1.5 * 2.0 ** -4                     # half-way, negative: ties to even (-2)
+    w = bf16(vals)
+    mg = Q.int4_margins(w, rotate=False)
+    np.testing.assert_allclose(mg["code"][0, :4], [0.5, 0.0, 0.5, 0.0])
+    out = Q.quantize_int4_g128(w, rotate=False)
+    assert R.int4_values(out["codes"])[0, :4].tolist() == [7, 2, 3, -2]
 
 
 def test_int4_fixed_points_unrotated():
@@ -63,8 +85,8 @@ def test_int4_round_to_nearest_bound(rotate):
     deq = R.dequant_int4(out["codes"], out["scales"])                     # the layer's decoder
     s = np.repeat(R.bf16_to_f64(out["scales"]), 128, axis=1)
     m = np.repeat(np.abs(target).reshape(6, 8, 128).max(-1), 128, axis=1)
-    # half a step, plus the fp32 rotation and division errors (a few ulp of the group maximum)
-    assert np.all(np.abs(deq - target) <= s / 2 + 2.0 ** -18 * m)
+    # half a step, up to the fp64 rounding of r / s
+    assert np.all(np.abs(deq - target) <= s / 2 * (1 + 2.0 ** -50) + 2.0 ** -60 * m)
     assert np.all(np.abs(R.int4_values(out["codes"])) <= 7)
 
 
@@ -109,7 +131,7 @@ def test_e2m1_rounding_brute_force():
     even = np.where(cand % 2 == 0, cand, 99).min(1)
     want = np.where((cand < 99).sum(1) > 1, even, cand.min(1))
     np.testing.assert_array_equal(got & 0x7, want)
-    np.testing.assert_array_equal(got >> 3, (x.view(np.uint32) >> 31).astype(np.uint8))
+    np.testing.assert_array_equal(got >> 3, np.signbit(x).astype(np.uint8))
 
 
 def test_e4m3_rounding_matches_torch():
@@ -161,3 +183,19 @@ def test_nvfp4_zero_linear():
     out = Q.quantize_nvfp4(np.zeros((2, 32), np.uint16))
     assert float(out["tscale"]) == 1.0
     assert np.all(out["scales"] == 0) and np.all(out["codes"] == 0)
+
+
+def test_nvfp4_margins_mark_the_rounding_boundaries():
+    # ts = 2^-10 (amax 6 * 448 * 2^-10); block 0 has scale 448 -> d = 448 * 2^-10; 1.25 d is an E2M1
+    # midpoint (margin 0, rounds to the even code 1.0), 1.5 d a grid value
+    d = 448 * 2.0 ** -10
+    w = np.zeros((1, 32))
+    w[0, 0] = 6 * d
+    w[0, 1] = 1.25 * d
+    w[0, 2] = 1.5 * d
+    wb = bf16(w)
+    mg = Q.nvfp4_margins(wb)
+    assert mg["code"][0, 1] == 0.0 and mg["code"][0, 2] > 0.1
+    out = Q.quantize_nvfp4(wb)
+    assert R.e2m1_to_f64(R.unpack_nibbles(out["codes"]))[0, :3].tolist() == [6.0, 1.0, 1.5]
+    assert mg["scale"][0, 0] > 0.01                 # 448 is an E4M3 value, far from a midpoint
