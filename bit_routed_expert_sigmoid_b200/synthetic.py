@@ -32,7 +32,7 @@ Every component draws from its own counter-keyed PCG64 stream, so the router
 and shared expert are identical across weight formats. Token row r of x comes
 from stream (SEED_X, r, d) where d is that row's redraw count; the redraw
 table (rows whose 6th/7th sigmoid-score gap is under 1e-4 are redrawn) is
-passed in by the caller, which reads it from a committed file.
+data shipped with this package (redraws.json).
 """
 
 from __future__ import annotations
@@ -182,12 +182,11 @@ def expert_nbytes(L: dict) -> int:
 
 
 def redraw_table(E: int, seed: int = SEED_WEIGHTS, skew: bool = False) -> dict:
-    """Redraw counts per token row for the router drawn with (E, seed, skew), from the committed
-    table tests/golden/redraws.json (written by tests/golden/make_redraws.py)."""
+    """Redraw counts per token row for the router drawn with (E, seed, skew), from the table shipped
+    with this package (redraws.json beside this module; written by tests/golden/make_redraws.py)."""
     import json
     import os
-    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "tests", "golden",
-                        "redraws.json")
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "redraws.json")
     with open(path) as f:
         tab = json.load(f)["tables"]
     key = f"E{E}_seed{seed}" + ("_skew" if skew else "")

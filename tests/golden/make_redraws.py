@@ -1,4 +1,4 @@
-"""Writes tests/golden/redraws.json: for each synthetic router, how many times each token row of
+"""Writes bit_routed_expert_sigmoid_b200/redraws.json (the synthetic generator's package data): for each synthetic router, how many times each token row of
 x is redrawn so that the gap between its 6th and 7th sigmoid scores is at least 1e-4.
 
 The workload definition asks for that resampling; the gap is computed by the fp64 oracle only.
@@ -55,7 +55,7 @@ def main():
         red = table(E, seed, skew, rows)
         out["tables"][key(E, seed, skew)] = {"rows": rows, "redraws": {str(k): v for k, v in sorted(red.items())}}
         print(key(E, seed, skew), len(red), "rows redrawn of", rows)
-    with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "redraws.json"), "w") as f:
+    with open(os.path.join(ROOT, "bit_routed_expert_sigmoid_b200", "redraws.json"), "w") as f:
         json.dump(out, f, indent=1, sort_keys=True)
 
 
