@@ -97,12 +97,8 @@ def stage_bytes(name: str, E: int, fmt: str, T: int, K: int, n_active: int) -> i
     sc_x = T * (H // 128) * 4 if fmt == "int4" else 0          # units of the 16-bit activation limbs
     sc_h = P * (I // 128) * 4 if fmt == "int4" else 0
     return {
-        # decode path (T <= 8): three kernels
-        "route": E * H * 2 + T * H * 2 + T * E * 4 + T * H * 2 * (2 if fmt == "int4" else 1) + sc_x,
-        "gate_up": n_active * eb_gu + 2 * IS * H * 2 + T * H * 2 + T * H * 2 + sc_x + P * I * 4 + P * I * 2 + sc_h
-                   + 2 * T * IS * 2,
-        "down": n_active * eb_dn + H * IS * 2 + P * I * 2 + sc_h + 2 * T * IS * 2 + P * H * 4 * 2 + T * H * 4 * 2
-                + T * H * 2,
+        # decode path (T <= 8): one kernel moves the whole layer
+        "layer": algorithmic_bytes(E, fmt, T, n_active),
         # larger T: one kernel per step (tensor-core path)
         "router_logits": E * H * 2 + T * H * 2 + T * E * 4,
         "topk": 4 * T * E * 4 + T * E * 4 + P * 8,              # 4 partial-logit slices in, logits out
@@ -158,7 +154,7 @@ def ncu_traffic(kernel: str, workload: str):
 # the translation unit of each kernel whose DRAM traffic is recorded (profiles/ncu_traffic.txt): a
 # recorded figure stands while these files are unchanged
 TRAFFIC_SOURCES = {
-    "gate_up": ("common.cuh", "decode.cu", "frag.cuh", "kernels.cuh"),
+    "layer": ("common.cuh", "decode.cu", "frag.cuh", "kernels.cuh"),
     "gu_routed": ("common.cuh", "kernels.cuh", "prefill.cu"),
     "quant": ("quant.cu",),
 }
@@ -724,7 +720,7 @@ def run_stack(args) -> dict:
     glue = (n + 1) * T * H * (4 + 4 + 2 + 2)          # residual read + write, y read, z write per boundary
     ab = sum(algorithmic_bytes(E, fmt, T, a) for a in n_active) + glue
 
-    # gate|up of every layer, timed with the library's stage events (instrumented pass)
+    # the layer kernel of every layer, timed with the library's stage events (instrumented pass)
     n_st = B.flint_moe_stage_count(stack.layers[0].handle, T)
     names = [B.flint_moe_stage_name(stack.layers[0].handle, T, i) for i in range(n_st)]
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)] for _ in stack.layers]
@@ -743,12 +739,12 @@ def run_stack(args) -> dict:
     for layer in stack.layers:
         B.flint_moe_set_stage_events(layer.handle, None)
     stage_ms = acc / n_prof
-    gi = names.index("gate_up")
-    gu_bytes = sum(stage_bytes("gate_up", E, fmt, T, 6, a) for a in n_active)
+    gi = names.index("layer")
+    gu_bytes = sum(stage_bytes("layer", E, fmt, T, 6, a) for a in n_active)
     gu_ms = float(stage_ms[:, gi].sum())
     peaks = measured_peaks()
     achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "gate_up (every layer)", "achieved": round(achieved, 1),
+    roofline = {"bound": "hbm", "kernel": "layer (every layer)", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": None, "algorithmic_bytes": gu_bytes, "peak_source": peaks["source"] + " (burst copy)"}
 

@@ -46,7 +46,7 @@ struct flint_moe_ctx {
   uint16_t* y_stage;
   int last_T;
   int n_sm;
-  CUtensorMap tm_gu, tm_sh_gu, tm_sh_dn;  // tensor maps of the decode kernels' weight copies
+  CUtensorMap tm_gu, tm_gu_sc, tm_sh_gu, tm_sh_dn;  // tensor maps of the decode kernel's weight copies
   CUtensorMap tm_pf_gu, tm_pf_dn;          // prefill: routed codes, 16-word x 128-row boxes, 64-byte swizzle
   CUtensorMap tm_pf_sh_gu, tm_pf_sh_dn;    // prefill: shared-expert weights, 64 x 128 bf16 boxes
   CUtensorMap tm_pf_router;                // prefill: router rows [E][H], 64 x 128 bf16 boxes
@@ -217,8 +217,8 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
   return off;
 }
 
-// T <= kDecodeMaxT: three kernels chained by programmatic dependent launch; larger T: one kernel per step.
-const char* const kDecodeStages[] = {"route", "gate_up", "down"};
+// T <= kDecodeMaxT: one kernel; larger T: one kernel per step.
+const char* const kDecodeStages[] = {"layer"};
 const char* const kGemvStages[] = {"router_logits", "topk", "permute", "xq", "gu_shared",
                                    "gu_routed", "dn_routed", "dn_shared", "combine"};
 
@@ -258,6 +258,7 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   if (T <= kDecodeMaxT) {
     DecodeParams d{};
     d.tm_gu = h->tm_gu;
+    d.tm_gu_sc = h->tm_gu_sc;
     d.tm_sh_gu = h->tm_sh_gu;
     d.tm_sh_dn = h->tm_sh_dn;
     d.fmt = fmt;
@@ -296,15 +297,10 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
     d.hsc = h->hsc;
     d.hs_hi = h->hs_hi;
     d.hs_lo = h->hs_lo;
-    d.o = h->o;
     d.ys = h->ys;
     d.err = h->err;
     d.cnt = h->cnt;
-    // with instrumentation events, one is recorded between consecutive kernels (which serialises them)
-    cudaEvent_t e1 = m.next < h->n_events ? h->events[m.next] : nullptr;
-    cudaEvent_t e2 = m.next + 1 < h->n_events ? h->events[m.next + 1] : nullptr;
-    m.next += (e1 ? 1 : 0) + (e2 ? 1 : 0);
-    FLINT_TRY(launch_decode(d, h->n_sm, s, e1, e2));
+    FLINT_TRY(launch_decode(d, h->n_sm, s));
     FLINT_TRY(m.mark());
     return FLINT_OK;
   }
@@ -424,8 +420,10 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
       cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       cudaMemset(h->err, 0, 16) != cudaSuccess || cudaMemset(h->cnt, 0, kCntInts * 4) != cudaSuccess ||
       !encode_rows(&h->tm_gu, w.gu_codes, static_cast<uint64_t>(cfg->n_experts) * 2 * kI, kH / 2, 64, 8) ||
+      (cfg->fmt == FLINT_W_NVFP4 &&
+       !encode_rows(&h->tm_gu_sc, w.gu_scales, static_cast<uint64_t>(cfg->n_experts) * 2 * kI, kH / 16, 8, 8)) ||
       !encode_rows(&h->tm_sh_gu, w.sh_gu, 2 * kIs, kH * 2, 256, 2) ||
-      !encode_rows(&h->tm_sh_dn, w.sh_dn, kH, kIs * 2, 128, 8) ||
+      !encode_rows(&h->tm_sh_dn, w.sh_dn, kH, kIs * 2, 64, 16) ||
       !encode_code_tiles(&h->tm_pf_gu, w.gu_codes, static_cast<uint64_t>(cfg->n_experts) * 2 * kI, kH / 2) ||
       !encode_code_tiles(&h->tm_pf_dn, w.dn_codes, static_cast<uint64_t>(cfg->n_experts) * kH, kI / 2) ||
       !encode_bf16_tiles(&h->tm_pf_sh_gu, w.sh_gu, 2 * kIs, kH) ||
@@ -438,6 +436,16 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
       !create_side_stream(h)) {
     delete h;
     return FLINT_ERR_CUDA;
+  }
+  // the decode kernel keeps every CTA resident (one per SM) and gives each at most 16 rows of y
+  int per_sm = 0;
+  if (decode_check_residency(cfg->fmt == FLINT_W_INT4_G128_FWHT128 ? kInt4 : kNvfp4, &per_sm) != cudaSuccess) {
+    delete h;
+    return FLINT_ERR_CUDA;
+  }
+  if (per_sm < 1 || h->n_sm < kH / 16) {
+    delete h;
+    return FLINT_ERR_UNSUPPORTED;
   }
   *out = h;
   return FLINT_OK;
@@ -535,8 +543,12 @@ flint_status flint_moe_intermediate(flint_moe_t h, int which, void* dst, size_t 
 
 flint_status flint_moe_error_word(flint_moe_t h, unsigned* out) {
   if (!h || !out) return FLINT_ERR_INVALID_ARG;
+  // the handle's own stream may still run part of a forward; the caller's stream must be idle
+  if (h->side) FLINT_TRY(cudaStreamSynchronize(h->side));
   FLINT_TRY(cudaMemcpy(out, h->err, sizeof(unsigned), cudaMemcpyDeviceToHost));
   FLINT_TRY(cudaMemset(h->err, 0, sizeof(unsigned)));
+  // a forward whose grid barrier gave up leaves its barrier words behind: start the next one clean
+  if (*out & kErrTimeout) FLINT_TRY(cudaMemset(h->cnt, 0, kCntInts * 4));
   return FLINT_OK;
 }
 

@@ -1,24 +1,28 @@
-// Whole-layer forward for small token counts (T <= 8): three kernels chained by programmatic
-// dependent launch (PDL), none of which ever waits for another CTA.
+// Whole-layer forward for small token counts (T <= 8): ONE persistent kernel, one CTA per SM,
+// launched cooperatively so that every CTA is resident at once.
 //
 // A decode forward streams 23-92 MB of weights through the chain router -> selection -> gate|up ->
-// down -> combine. Each arrow of that chain is a kernel boundary here, and PDL hides it: the next
-// kernel is resident and streaming weights that do not depend on the previous one before that one
-// has finished, and it calls griddepcontrol.wait only before it reads what the previous one wrote.
+// down -> combine. Each arrow that needs data from every SM is a grid barrier inside the kernel
+// (an arrival counter and a generation word in global memory, one bounded wait per CTA), not a
+// kernel boundary, and every SM keeps weight copies in flight across it.
 //
-//   route    CTAs split the router rows (fp32 logits) and the activation operand of gate|up; the
-//            last CTA to finish (atomic arrival counter) selects the top-k of every token and builds
-//            the routing tables. It lets the gate|up kernel launch at once.
-//   gate_up  persistent, one CTA per SM; every warp runs its own pipeline: its lanes bring 4 KB
-//            stages of weight rows from HBM into the warp's shared-memory ring with bulk copies
-//            (cp.async.bulk + mbarrier transaction counts) and the warp turns them into tensor-core
-//            products with the activations. Shared-expert tiles come first and need no routing, so
-//            they stream while the route kernel still runs; the routed tiles follow after
-//            griddepcontrol.wait. The warp that finishes the last of the 16 tiles of a 128-segment
-//            of h turns that segment into the down operand.
-//   down     same pipelines; the first weight stages are requested before griddepcontrol.wait, so
-//            HBM stays busy through the tail of gate_up. The warp that finishes the last tile of a
-//            64-row block of y combines that block: y = bf16(routed_scale * sum_k w_k o_k + ys).
+//   phase A  no dependencies. Warps 4-6 compute the router logits (a warp per router row, x staged
+//            by one bulk copy) and the routed experts' activation operand (a warp per 128-segment
+//            of a token); warps 0-3 start streaming the shared expert's gate|up tiles at once; one
+//            thread asks L2 for the shared expert's down rows.
+//   barrier 1
+//   phase B  every CTA selects the top-k of every token from the logits (a warp per token) and
+//            builds the routing tables in its own shared memory; then the routed gate|up tiles of
+//            the active experts (8 gate + 8 up rows, all of K, per tile). The warp that finishes
+//            the last of the 16 tiles of a 128-segment of h turns that segment into the down
+//            operand (last-arriver counter; nobody waits for it). Before the barrier every warp
+//            already requests its first down stages.
+//   barrier 2
+//   phase C  CTA c owns output rows [2048c/G, 2048(c+1)/G) of y (13-14 rows on 148 SMs), so the
+//            combine needs no other CTA: it streams those rows of every active expert's down
+//            matrix and of the shared expert's down matrix (eight K slices), keeps the partial
+//            results in shared memory and sums them in a fixed order:
+//            y = bf16(routed_scale * sum_k w_k o_k + ys).
 //
 // Arithmetic. Decode is bound by HBM, and at 6.5 TB/s an SM may spend only a few instructions per
 // weight byte, so the cost of turning 4-bit codes into MMA operands decides the speed.
@@ -32,8 +36,10 @@
 //   NVFP4    codes are converted by the hardware E2M1 -> fp16 conversion and multiplied by their
 //            E4M3 block scale in fp16 (exact), then fp16 MMA with fp32 accumulation.
 //   bf16     (shared expert) bf16 MMA with fp32 accumulation.
-// Every wait is either the hardware grid dependency or an mbarrier wait on the warp's own copies;
-// the latter is bounded and records a timeout bit in the error word when it expires.
+// Every wait is bounded: the mbarrier waits on a warp's own copies and the two grid barriers give
+// up after 1 s of %globaltimer and set the timeout bit of the error word; a grid wait that gives up
+// also sets an abort word that makes every later grid wait of the forward return at once, so a
+// forward always ends.
 #include "frag.cuh"
 #include "kernels.cuh"
 
@@ -47,13 +53,18 @@ namespace {
 constexpr uint64_t kWaitNs = FLINT_WAIT_NS;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
+constexpr int kWarps = 8;                    // warps per CTA
+constexpr int kThreads = kWarps * 32;
+constexpr int kRouteWarp0 = 4;               // warps 4..7: router rows, operand, top-k, tables
+constexpr int kRouteThreads = (kWarps - kRouteWarp0) * 32;
+constexpr int kBarRoute = 1;                 // named barrier of the routing warps
+constexpr int kMaxRowsPerCta = 16;           // phase C rows of y per CTA (one MMA tile)
+constexpr int kShDnSlices = kIs / kGroup;    // shared down K slices of 128 (8)
+
 // Asks L2 to fetch [ptr, ptr + bytes) from HBM (a hint; no completion to wait for).
 __device__ __forceinline__ void prefetch_l2(const void* ptr, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
 }
-
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Arrival of the calling thread on a counter with acquire-release semantics at GPU scope; returns
 // the previous value.
@@ -61,6 +72,10 @@ __device__ __forceinline__ int atom_add_acq_rel(int* ctr, int v) {
   int old;
   asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(ctr), "r"(v) : "memory");
   return old;
+}
+
+__device__ __forceinline__ void st_relaxed_gpu(int* p, int v) {
+  asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // A warp's arrival on a counter whose result is examined later: the warp barrier orders every
@@ -98,21 +113,60 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// ------------------------------------------------------------------------------------ grid barrier
+
+// Barrier words in global memory (zeroed at handle creation): an arrival count, a generation that
+// the last arriver advances, and an abort word. A CTA's thread 0 reads the generation at the start
+// of the forward (it cannot change before every CTA has arrived once), so barrier b of the forward
+// is passed when the generation equals start + b.
+struct GridBarrier {
+  int* count;
+  int* gen;
+  int* abort_;
+  // One thread per CTA, after the CTA's writes that must be visible are ordered before it by a
+  // CTA barrier: arrive, and if last, reset the count and advance the generation (release).
+  __device__ __forceinline__ void arrive(int nblocks, int target) const {
+    __threadfence();
+    const int old = atom_add_acq_rel(count, 1);
+    if (old == nblocks - 1) {
+      st_relaxed_gpu(count, 0);
+      st_release_gpu(gen, target);
+    }
+  }
+  // Bounded wait of one thread for generation `target`; false on timeout or abort.
+  __device__ __forceinline__ bool wait(int target, unsigned* err) const {
+    if (ld_acquire_gpu(gen) == target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    unsigned ns = 32;
+    for (;;) {
+      if (ld_acquire_gpu(gen) == target) return true;
+      if (ld_relaxed_gpu(abort_) != 0) return false;
+      if (globaltimer_ns() - t0 > kWaitNs) {
+        atomicOr(err, kErrTimeout);
+        atomicExch(abort_, 1);
+        return false;
+      }
+      __nanosleep(ns);
+      if (ns < 256) ns <<= 1;
+    }
+  }
+};
+
 // ------------------------------------------------------------------------ 16-bit fixed-point limbs
 
 // m16n8k32 integer MMA, A = int8 weights (16 rows), B = high (signed) or low (unsigned) limb bytes.
 __device__ __forceinline__ void imma_hi(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                         uint32_t b1) {
   asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-               : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ void imma_lo(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                         uint32_t b1) {
   asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-               : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // Stores the warp's 128-segment v (lane l holds the natural elements 4l..4l+3) as 16-bit fixed
@@ -168,7 +222,8 @@ __device__ __forceinline__ void int4_group(float (&acc)[4], const uint4& ra, con
 }
 
 // One 128-wide K group of a 16-row NVFP4 tile into two fp32 accumulator sets (steps alternate).
-// Codes x E4M3 block scale are exact in fp16; thread t's 32 codes span the blocks 8j+2t, 8j+2t+1.
+// Codes x E4M3 block scale are exact in fp16; thread t's 32 codes span the blocks 8j+2t, 8j+2t+1 of
+// the scale rows bs0 (row g) and bs1 (row g+8), whose block 0 is the group-0 block of j.
 __device__ __forceinline__ void nvfp4_group(float (&acc)[2][4], const uint4& ra, const uint4& rb, const RawB& B,
                                             const uint8_t* bs0, const uint8_t* bs1, int j, int t) {
   const int blk = j * 8 + 2 * t;
@@ -207,7 +262,7 @@ __device__ __forceinline__ void bf16_group(float (&acc)[2][4], const RawA<kBf16>
 __device__ __forceinline__ void load_a_bf16_rows(RawA<kBf16>& A, const uint8_t* st, int pitch, int nrows, int g, int jj,
                                                  int t) {
   if (g < nrows) {
-    load_a_bf16_smem(A, st + g * pitch, nullptr, jj, t);
+    load_a_bf16_smem(A, st + g * pitch, (g + 8 < nrows) ? st + (g + 8) * pitch : nullptr, jj, t);
   } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) A.r0[i] = A.r1[i] = make_uint4(0, 0, 0, 0);
@@ -215,8 +270,6 @@ __device__ __forceinline__ void load_a_bf16_rows(RawA<kBf16>& A, const uint8_t* 
 }
 
 // ============================================================================================ route
-
-constexpr int kRouteWarps = 8;
 
 // 8 bf16 x 8 bf16 dot product; the products are exact in fp32.
 __device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b, float acc) {
@@ -236,8 +289,9 @@ __device__ __forceinline__ void load_router_row(uint4 (&w)[8], const DecodeParam
 }
 
 // logits[t][e] for every token (one warp, router row in w; lane l covers elements 8l + 256i; x in
-// shared memory).
-__device__ void route_row(const DecodeParams& p, int e, const uint4 (&w)[8], const uint16_t* xs) {
+// shared memory, token rows `pitch` bytes apart). The lane order and the shuffle reduction are those
+// of the routing-only entry point's router kernel, so both produce the same fp32 logits.
+__device__ void route_row(const DecodeParams& p, int e, const uint4 (&w)[8], const uint8_t* xs, int pitch) {
   const int lane = threadIdx.x & 31;
   float acc[kDecodeMaxT];
 #pragma unroll
@@ -246,23 +300,23 @@ __device__ void route_row(const DecodeParams& p, int e, const uint4 (&w)[8], con
     if (t < p.T) {
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        acc[t] = dot8_bf16(w[i], *reinterpret_cast<const uint4*>(xs + t * kH + 8 * lane + 256 * i), acc[t]);
+        acc[t] = dot8_bf16(w[i], *reinterpret_cast<const uint4*>(xs + t * pitch + (8 * lane + 256 * i) * 2), acc[t]);
     }
   }
 #pragma unroll
   for (int t = 0; t < kDecodeMaxT; ++t) {
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) acc[t] += __shfl_xor_sync(kFull, acc[t], m);
-    if (lane == 0 && t < p.T) p.logits[t * p.E + e] = acc[t];
+    if (lane == 0 && t < p.T) __stcg(p.logits + t * p.E + e, acc[t]);
   }
 }
 
 // One 128-segment of the gate|up activation operand (x in shared memory), written to global memory:
 // fp16(Hn x) with every 8-block in the order 0,4,1,5,2,6,3,7 and the 16-bit limbs of Hn x with
 // their unit (int4), or fp16(x) (NVFP4).
-__device__ void xq_segment(const DecodeParams& p, int tok, int seg, const uint16_t* xs) {
+__device__ void xq_segment(const DecodeParams& p, int tok, int seg, const uint8_t* xs, int pitch) {
   const int lane = threadIdx.x & 31;
-  const uint2 raw = *reinterpret_cast<const uint2*>(xs + tok * kH + seg * kGroup + 4 * lane);
+  const uint2 raw = *reinterpret_cast<const uint2*>(xs + tok * pitch + (seg * kGroup + 4 * lane) * 2);
   float v[4] = {bf16lo_to_f32(raw.x), bf16hi_to_f32(raw.x), bf16lo_to_f32(raw.y), bf16hi_to_f32(raw.y)};
   if (p.fmt == kInt4) {
     fwht128_warp(v);
@@ -272,18 +326,19 @@ __device__ void xq_segment(const DecodeParams& p, int tok, int seg, const uint16
   store_seg_half(p.xq + static_cast<size_t>(tok) * kH + seg * kGroup, v, p.fmt == kInt4);
 }
 
-// Order-preserving map of a float (not NaN) to an unsigned integer; -0 maps like +0.
-__device__ __forceinline__ unsigned float_key(float f) {
+// Order-preserving map of a logit to an unsigned key: -0 as +0, NaN as 0 (below every number, so it
+// is picked only when nothing else is left); every other key is above 0.
+__device__ __forceinline__ unsigned logit_key(float f) {
   unsigned b = __float_as_uint(f);
-  if (b == 0x80000000u) b = 0u;
+  if ((b & 0x7FFFFFFFu) > 0x7F800000u) return 0u;
+  if ((b << 1) == 0u) b = 0u;
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
-__device__ __forceinline__ float key_float(unsigned k) {
+__device__ __forceinline__ float key_logit(unsigned k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// Routing of a forward in one CTA's shared memory. Every projection CTA derives it from the logits
-// (top-k and tables are a few microseconds of work for T <= 8): a CTA never waits for another.
+// Routing of a forward in one CTA's shared memory.
 struct RouteSmem {
   int ids[kMaxActive];                      // [T][K] selected experts, slots by ascending id
   float w[kMaxActive];                      // [T][K] routing weights
@@ -301,33 +356,28 @@ struct RouteSmem {
 __device__ __forceinline__ void topk_token(const DecodeParams& p, int tok, RouteSmem& rs, bool publish) {
   const int lane = threadIdx.x & 31;
   const int E = p.E, K = p.K, per = E >> 5;
-  const float floor_ = p.floor_;
-  const float* logits = p.logits;
-  int* g_ids = p.ids;
-  float* g_wts = p.wts;
-  // element j of lane l is expert l + 32j; key 0 marks an element that is absent or taken (every
-  // finite logit has a key above 0)
+  // element j of lane l is expert l + 32j; a taken or absent element has key 0 and index E+
   unsigned key[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) key[j] = (j < per) ? float_key(__ldcg(logits + tok * E + lane + 32 * j)) : 0u;
+  for (int j = 0; j < 8; ++j) key[j] = (j < per) ? logit_key(__ldcg(p.logits + tok * E + lane + 32 * j)) : 0u;
+  unsigned taken = 0u;                             // bit j: element j already chosen
   int my_id = 0;
   float my_l = 0.f;
   for (int k = 0; k < K; ++k) {
-    // largest logit: one warp max-reduction of the keys; then the lowest index holding it
+    // largest key among the elements not yet taken, then the lowest index holding it
     unsigned lm = 0u;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) lm = max(lm, key[j]);
+    for (int j = 0; j < 8; ++j)
+      if (j < per && !((taken >> j) & 1u)) lm = max(lm, key[j]);
     const unsigned gm = __reduce_max_sync(kFull, lm);
     unsigned cand = 0xFFFFFFFFu;
 #pragma unroll
     for (int j = 7; j >= 0; --j)
-      if (key[j] == gm) cand = static_cast<unsigned>(lane + 32 * j);
+      if (j < per && !((taken >> j) & 1u) && key[j] == gm) cand = static_cast<unsigned>(lane + 32 * j);
     unsigned win = __reduce_min_sync(kFull, cand);
-    if (win >= static_cast<unsigned>(E)) win = 0u;  // unreachable with finite logits
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (win == static_cast<unsigned>(lane + 32 * j)) key[j] = 0u;
-    if (lane == k) { my_id = static_cast<int>(win); my_l = key_float(gm); }
+    if (win >= static_cast<unsigned>(E)) win = 0u;   // unreachable: K <= E elements are never all taken
+    if ((win & 31u) == static_cast<unsigned>(lane)) taken |= 1u << (win >> 5);
+    if (lane == k) { my_id = static_cast<int>(win); my_l = key_logit(gm); }
   }
   int rank = 0;
   for (int k = 0; k < K; ++k) rank += (__shfl_sync(kFull, my_id, k) < my_id);
@@ -340,13 +390,13 @@ __device__ __forceinline__ void topk_token(const DecodeParams& p, int tok, Route
   }
   float sum = 0.f;
   for (int r = 0; r < K; ++r) sum += __shfl_sync(kFull, s_r, r);
-  const float denom = fmaxf(sum, floor_);
+  const float denom = fmaxf(sum, p.floor_);
   if (lane < K) {
     rs.ids[tok * K + rank] = my_id;
     rs.w[tok * K + rank] = s / denom;
     if (publish) {
-      g_ids[tok * K + rank] = my_id;
-      g_wts[tok * K + rank] = s / denom;
+      p.ids[tok * K + rank] = my_id;
+      p.wts[tok * K + rank] = s / denom;
     }
   }
 }
@@ -362,16 +412,8 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& r
   const int* s_ids = rs.ids;
   const int lane = threadIdx.x & 31;
   const int T = p.T, E = p.E, K = p.K, P = T * K;
-  // parameters in registers: the table stores below could otherwise force them to be reloaded
   const float* gu_ts = p.gu_ts;
   const float* dn_ts = p.dn_ts;
-  int* g_counts = p.counts;
-  int* g_offsets = p.offsets;
-  int* g_active = p.active;
-  int4* g_etab = p.etab;
-  int* g_n_active = p.n_active;
-  int* g_perm = p.perm;
-  int* g_inv = p.inv;
   for (int e = lane; e < kMaxE; e += 32) {
     scr_cnt[e] = 0;
     scr_mask[e] = 0u;
@@ -381,10 +423,9 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& r
   if (lane < P) { atomicAdd(&scr_cnt[id0], 1); atomicOr(&scr_mask[id0], 1u << (lane / K)); }
   if (lane + 32 < P) { atomicAdd(&scr_cnt[id1], 1); atomicOr(&scr_mask[id1], 1u << ((lane + 32) / K)); }
   __syncwarp();
-  // lane holds experts 8*lane .. 8*lane+7 (loops kept rolled: this code runs once per CTA, where
-  // instruction fetches dominate)
+  // lane holds experts 8*lane .. 8*lane+7
   int s = 0, a = 0;
-#pragma unroll 1
+#pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int e = 8 * lane + j;
     const int c = e < E ? scr_cnt[e] : 0;
@@ -405,8 +446,8 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& r
     if (e >= E) break;
     const int c = scr_cnt[e];
     if (publish) {
-      g_counts[e] = c;
-      g_offsets[e] = off;
+      p.counts[e] = c;
+      p.offsets[e] = off;
     }
     scr_cnt[e] = off;
     if (c > 0) {
@@ -424,9 +465,9 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& r
       rs.etab[slot][0] = t0;
       rs.etab[slot][1] = t1;
       if (publish) {
-        g_active[slot] = e;
-        g_etab[2 * slot] = t0;
-        g_etab[2 * slot + 1] = t1;
+        p.active[slot] = e;
+        p.etab[2 * slot] = t0;
+        p.etab[2 * slot + 1] = t1;
       }
       ++slot;
     }
@@ -435,8 +476,8 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& r
   if (lane == 31) {
     rs.na = ai;
     if (publish) {
-      g_offsets[E] = si;
-      *g_n_active = ai;
+      p.offsets[E] = si;
+      *p.n_active = ai;
     }
   }
   __syncwarp();
@@ -448,80 +489,10 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& r
       const int pos = scr_cnt[id] + __popc(scr_mask[id] & ((1u << tt) - 1u));
       rs.inv[q] = pos;
       if (publish) {
-        g_perm[pos] = q;
-        g_inv[q] = pos;
+        p.perm[pos] = q;
+        p.inv[q] = pos;
       }
     }
-  }
-}
-
-// A group of `nw` warps (group-relative warp index gw; named barrier `bar` over the group's
-// threads): top-k of every token (a token per warp), then the tables (the group's first warp).
-__device__ __noinline__ void route_group(const DecodeParams& p, RouteSmem& rs, bool publish, int gw, int nw,
-                                            int bar) {
-  for (int tok = gw; tok < p.T; tok += nw) topk_token(p, tok, rs, publish);
-  named_bar_sync(bar, nw * 32);
-  if (gw == 0) build_tables(p, rs, publish);
-  named_bar_sync(bar, nw * 32);
-}
-
-__global__ void __launch_bounds__(kRouteWarps * 32) decode_route_kernel(const __grid_constant__ DecodeParams p) {
-  pdl_trigger();                                   // the gate|up kernel may start its shared-expert tiles
-  __shared__ __align__(128) uint16_t xs[kDecodeMaxT * kH];
-  __shared__ uint64_t xbar;
-  const int warp = threadIdx.x >> 5;
-  const int gw = blockIdx.x * kRouteWarps + warp, nw = gridDim.x * kRouteWarps;
-  if (threadIdx.x == 0) {                          // x (T contiguous rows) by one bulk copy
-    mbar_init(&xbar, 1);
-    fence_mbar_init();
-    mbar_arrive_expect_tx(&xbar, p.T * kH * 2);
-    bulk_g2s(xs, p.x, p.T * kH * 2, &xbar);
-  }
-  uint4 w[8];
-  if (gw < p.E) load_router_row(w, p, gw);
-  __syncthreads();                                 // the barrier is initialised
-  if (!mbar_wait_bounded(&xbar, 0, kWaitNs) && threadIdx.x == 0) atomicOr(p.err, kErrTimeout);
-  for (int e = gw; e < p.E; e += nw) {
-    if (e != gw) load_router_row(w, p, e);
-    route_row(p, e, w, xs);
-  }
-  for (int sg = gw; sg < p.T * (kH / kGroup); sg += nw) xq_segment(p, sg / (kH / kGroup), sg % (kH / kGroup), xs);
-}
-
-// ================================================================================ weight pipelines
-
-constexpr int kShGuTiles = kIs / 2;         // shared gate|up tiles: 2 hs columns each
-constexpr int kShDnTiles = kH / 8;          // shared down tiles: 8 ys rows each, in 4 stages
-constexpr int kGuTilesPerExpert = kI / 8;   // 64 routed gate|up tiles: 8 h columns each
-constexpr int kDnTilesPerExpert = kH / 32;  // 64 routed down tiles: 32 o rows each
-
-
-constexpr int kDnStage = 4096 + 512;        // codes (16 rows x 256 B, or 8 bf16 rows x 512 B) + scales
-// int4 runs 16 warps with 2-stage rings (at most 128 registers), NVFP4 8 warps with 4 stages; about
-// 128 KB per SM in flight, and the rest of the SM's 256 KB holds L1 lines of the activation rows.
-template <int FMT>
-struct DnGeom {
-  static constexpr int kWarps = FMT == kInt4 ? 16 : 8;
-  static constexpr int kDepth = FMT == kInt4 ? 2 : 4;
-};
-template <int FMT>
-struct DnWarp {
-  alignas(128) uint8_t stage[DnGeom<FMT>::kDepth][kDnStage];
-  uint64_t full[DnGeom<FMT>::kDepth];
-};
-template <int FMT>
-struct DnShared {
-  DnWarp<FMT> w[DnGeom<FMT>::kWarps];
-  RouteSmem rs;
-  alignas(128) uint8_t hq[kMaxActive][2 * kI];        // down operand of every position: int4 limbs (hi, lo), NVFP4 fp16
-  float hsc[kMaxActive][kI / kGroup];                 // int4: unit / 16 of each segment of hq
-  uint64_t hqbar;                                     // completion of the operand copy
-};
-
-// Bounded wait for a stage (the barrier is the warp's own).
-__device__ __forceinline__ void wait_stage(const DecodeParams& p, uint64_t* bar, uint32_t parity) {
-  if (!mbar_wait_bounded(bar, parity, kWaitNs)) {
-    if ((threadIdx.x & 31) == 0) atomicOr(p.err, kErrTimeout);
   }
 }
 
@@ -533,7 +504,7 @@ struct ExpertInfo {
 };
 
 // The expert table held by one warp in registers (lane l keeps entries l and l + 32), loaded once;
-// an entry is then fetched by shuffles instead of a round trip to L2 per tile.
+// an entry is then fetched by shuffles instead of a shared-memory round trip per tile.
 struct WarpTable {
   int4 a[2], b[2];
   __device__ __forceinline__ void load(const RouteSmem& rs) {
@@ -569,57 +540,76 @@ __device__ __forceinline__ int active_count(const DecodeParams& p, const RouteSm
   return min(max(rs.na, 0), min(kMaxActive, p.T * p.K));
 }
 
-// ============================================================================================ gate|up
+// ===================================================================================== the kernel
 
-// gate|up shared memory: per warp a ring of 4 KB stages (16 rows x 256 B of codes, or 4 bf16 rows x
-// 1 KB) and the scales of its current and next tile; per CTA the token rows of x (bf16, for the
-// shared expert) and of the routed operand (int4: limbs, NVFP4: fp16), rows padded by 64 bytes so
-// that the 8-lane phases of the fragment loads of different tokens hit different banks.
-// Warps per CTA and stages per warp ring: int4 (at most 128 registers) runs 16 warps with 2 stages,
-// NVFP4 (more registers per thread) 8 warps with 3; about 128 / 96 KB per SM in flight. A ring holds
-// at most one tile's 4 stages, which keeps the scale double buffer safe.
-template <int FMT>
-struct GuGeom {
-  static constexpr int kWarps = FMT == kInt4 ? 16 : 8;
-  static constexpr int kDepth = FMT == kInt4 ? 2 : 3;
-};
-constexpr int kGuStage = 4096;
-constexpr int kTokPitch = 2 * kH + 64;      // bytes per token row of x or of the routed operand
+constexpr int kShGuTiles = kIs / 2;         // shared gate|up tiles: 2 hs columns (2 gate + 2 up rows) each
+constexpr int kGuTilesPerExpert = kI / 8;   // 64 routed gate|up tiles: 8 h columns (8 gate + 8 up rows) each
+constexpr int kTokPitch = 2 * kH + 64;      // bytes per staged token row of x or of the routed operand
 
+// Per-warp ring of weight stages. int4: 4 stages of 4096 B codes (+256 B for phase C's scales);
+// NVFP4: 3 stages of 4096 B codes + 512 B of block scales.
 template <int FMT>
-struct GuWarp {
-  alignas(128) uint8_t stage[GuGeom<FMT>::kDepth][kGuStage];
-  alignas(128) uint8_t scales[2][FMT == kInt4 ? 16 * (kH / kGroup) * 2 : 16 * (kH / 16)];
-  uint64_t full[GuGeom<FMT>::kDepth];
+struct Geom {
+  static constexpr int kDepth = FMT == kInt4 ? 4 : 3;
+  static constexpr int kStage = FMT == kInt4 ? 4096 + 256 : 4096 + 512;
 };
 
 template <int FMT>
-struct GuShared {
-  GuWarp<FMT> w[GuGeom<FMT>::kWarps];
-  alignas(128) uint8_t xs[kDecodeMaxT][kTokPitch];    // x, bf16
-  alignas(128) uint8_t xq[kDecodeMaxT][kTokPitch];    // int4: hi limbs, lo limbs; NVFP4: fp16 x
-  float xsc[kDecodeMaxT][kH / kGroup];                // int4: unit / 16 of each segment of xq
+struct DecShared {
+  alignas(128) uint8_t stage[kWarps][Geom<FMT>::kDepth][Geom<FMT>::kStage];
+  alignas(16) uint8_t gu_sc[FMT == kInt4 ? kWarps : 1][2][16 * (kH / kGroup) * 2];   // int4: tile scales, 2 tiles
+  union {
+    struct {                                          // phases A and B
+      alignas(128) uint8_t xs[kDecodeMaxT][kTokPitch];  // x, bf16
+      alignas(128) uint8_t xq[kDecodeMaxT][kTokPitch];  // int4: hi limbs, lo limbs; NVFP4: fp16 x
+      float xsc[kDecodeMaxT][kH / kGroup];              // int4: unit / 16 of each segment of xq
+    } ab;
+    struct {                                          // phase C
+      alignas(128) uint8_t hq[kMaxActive][2 * kI];      // down operand of every position: int4 limbs, NVFP4 fp16
+      float hsc[kMaxActive][kI / kGroup];               // int4: unit / 16 of each segment of hq
+      float opart[kMaxActive][kMaxRowsPerCta];          // routed down outputs of this CTA's rows, per position
+      float spart[kShDnSlices][kDecodeMaxT][kMaxRowsPerCta];   // shared down partial sums per K slice
+    } c;
+  } u;
   RouteSmem rs;
-  uint64_t xbar;                                      // completion of the x copies
-  uint64_t xqbar;                                     // completion of the operand copies
-  uint64_t route_ready;                               // the routing warps have filled rs
+  uint64_t full[kWarps][Geom<FMT>::kDepth];
+  uint64_t xbar, xqbar, hqbar, route_ready;
+  int gen0;
 };
 
-// Warps kRouteWarp0.. of a gate|up CTA derive the routing (they hold no shared-expert tile: tile
-// b + ncta * w is one only for w < 512 / ncta <= 4); the others wait for it on an mbarrier only when
-// they reach a routed tile, so their shared-expert tiles never stall.
-constexpr int kRouteWarp0 = 4;
-
-// Warp-collective: stage s (K groups 4q..4q+3, q = s mod 4) of tile `tile`, as few large copies (the
-// copy engine's cost is per copy more than per byte). Shared tile st: one tensor box with Sg rows
-// 2st, 2st+1 and one with Su rows 2st, 2st+1 (1 KB each). Routed tile (gi, i8): one box of gate rows
-// 8*i8 .. +8 and one of the matching up rows (256 B each); with q == 0 also the tile's scales.
+// A warp's ring position: stages are issued and consumed in one sequence across the three phases.
 template <int FMT>
-__device__ void gu_issue(const DecodeParams& p, GuWarp<FMT>& ws, int s, int tile, const ExpertInfo& ex) {
+struct Ring {
+  static constexpr int D = Geom<FMT>::kDepth;
+  uint8_t* base;               // stage[warp][0]
+  uint64_t* full;              // full[warp][0]
+  int issued = 0, consumed = 0;
+  __device__ __forceinline__ uint8_t* slot_ptr(int i) const { return base + (i % D) * Geom<FMT>::kStage; }
+  __device__ __forceinline__ uint64_t* bar(int i) const { return full + (i % D); }
+  __device__ __forceinline__ bool has_room() const { return issued - consumed < D; }
+};
+
+// Bounded wait for a stage (the barrier is the warp's own).
+__device__ __forceinline__ void wait_stage(const DecodeParams& p, uint64_t* bar, uint32_t parity) {
+  if (!mbar_wait_bounded(bar, parity, kWaitNs)) {
+    if ((threadIdx.x & 31) == 0) atomicOr(p.err, kErrTimeout);
+  }
+}
+
+// ---- phase B: gate|up
+
+// Warp-collective: stage q (K groups 4q..4q+3) of gate|up tile `tile` into ring slot i. Shared tile
+// st: one tensor box with Sg rows 2st, 2st+1 and one with Su rows 2st, 2st+1 (1 KB each). Routed
+// tile (gi, i8): one box of gate rows 8*i8 .. +8 and one of the matching up rows (256 B each); int4
+// with q == 0 also the tile's scales (bulk copies into the warp's scale buffer of the tile's
+// parity); NVFP4 the block scales of the stage's K quarter (two 8-row boxes of 32 B rows).
+template <int FMT>
+__device__ void gu_issue(const DecodeParams& p, DecShared<FMT>& sm, Ring<FMT>& ring, int warp, int q, int k, int tile,
+                         const ExpertInfo& ex) {
   const int lane = threadIdx.x & 31;
-  const int slot = s % GuGeom<FMT>::kDepth, q = s & 3;
-  uint8_t* st = ws.stage[slot];
-  uint64_t* bar = &ws.full[slot];
+  const int i = ring.issued++;
+  uint8_t* st = ring.slot_ptr(i);
+  uint64_t* bar = ring.bar(i);
   if (tile < kShGuTiles) {
     if (lane == 0) {
       mbar_arrive_expect_tx(bar, 4 * 1024);
@@ -630,41 +620,50 @@ __device__ void gu_issue(const DecodeParams& p, GuWarp<FMT>& ws, int s, int tile
   }
   const int i0 = 8 * ((tile - kShGuTiles) % kGuTilesPerExpert);
   const int erow = ex.e * (2 * kI);
-  // scale bytes per row: int4 16 bf16 group scales, NVFP4 128 E4M3 block scales
-  constexpr uint32_t row_sc = FMT == kInt4 ? (kH / kGroup) * 2 : kH / 16;
-  if (lane == 0) {
-    mbar_arrive_expect_tx(bar, 16 * 256 + (q == 0 ? 16 * row_sc : 0));
-    tma_load_2d(st, &p.tm_gu, q * 64, erow + i0, bar);
-    tma_load_2d(st + 2048, &p.tm_gu, q * 64, erow + kI + i0, bar);
-  }
-  __syncwarp();
-  if (q == 0 && (lane == 1 || lane == 2)) {        // gate rows' scales, then the up rows'
-    uint8_t* sc = ws.scales[(s >> 2) & 1] + (lane - 1) * 8 * row_sc;
-    bulk_g2s(sc, p.gu_scales + (static_cast<size_t>(erow) + (lane - 1) * kI + i0) * row_sc, 8 * row_sc, bar);
+  if constexpr (FMT == kInt4) {
+    constexpr uint32_t row_sc = (kH / kGroup) * 2;   // 16 bf16 group scales per row
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar, 16 * 256 + (q == 0 ? 16 * row_sc : 0));
+      tma_load_2d(st, &p.tm_gu, q * 64, erow + i0, bar);
+      tma_load_2d(st + 2048, &p.tm_gu, q * 64, erow + kI + i0, bar);
+    }
+    __syncwarp();
+    if (q == 0 && (lane == 1 || lane == 2)) {        // gate rows' scales, then the up rows'
+      uint8_t* sc = sm.gu_sc[warp][k & 1] + (lane - 1) * 8 * row_sc;
+      bulk_g2s(sc, p.gu_scales + (static_cast<size_t>(erow) + (lane - 1) * kI + i0) * row_sc, 8 * row_sc, bar);
+    }
+  } else {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar, 16 * 256 + 16 * 32);
+      tma_load_2d(st, &p.tm_gu, q * 64, erow + i0, bar);
+      tma_load_2d(st + 2048, &p.tm_gu, q * 64, erow + kI + i0, bar);
+      tma_load_2d(st + 4096, &p.tm_gu_sc, q * 8, erow + i0, bar);
+      tma_load_2d(st + 4096 + 256, &p.tm_gu_sc, q * 8, erow + kI + i0, bar);
+    }
   }
 }
 
 // B operand of one group for one thread from a staged token row (32 stored elements, 64 bytes).
 __device__ __forceinline__ void load_b_smem(RawB& B, const uint8_t* row, int j, int t, bool valid) {
   if (valid) {
-    const uint8_t* p = row + (j * 128 + 32 * t) * 2;
+    const uint8_t* q = row + (j * 128 + 32 * t) * 2;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) B.u[q] = *reinterpret_cast<const uint4*>(p + 16 * q);
+    for (int i = 0; i < 4; ++i) B.u[i] = *reinterpret_cast<const uint4*>(q + 16 * i);
   } else {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) B.u[q] = make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < 4; ++i) B.u[i] = make_uint4(0, 0, 0, 0);
   }
 }
 
-// Limbs (hi row at row, lo row at row + kH) of a staged token row for group j: the thread's 32 bytes.
-__device__ __forceinline__ void load_limbs_smem(uint4 (&bh)[2], uint4 (&bl)[2], const uint8_t* row, int j, int t,
-                                                bool valid) {
+// Limbs (hi row at row, lo row at row + lo_off) of a staged row for group j: the thread's 32 bytes.
+__device__ __forceinline__ void load_limbs_smem(uint4 (&bh)[2], uint4 (&bl)[2], const uint8_t* row, int lo_off, int j,
+                                                int t, bool valid) {
   if (valid) {
     const uint8_t* ph = row + j * 128 + 32 * t;
     bh[0] = *reinterpret_cast<const uint4*>(ph);
     bh[1] = *reinterpret_cast<const uint4*>(ph + 16);
-    bl[0] = *reinterpret_cast<const uint4*>(ph + kH);
-    bl[1] = *reinterpret_cast<const uint4*>(ph + kH + 16);
+    bl[0] = *reinterpret_cast<const uint4*>(ph + lo_off);
+    bl[1] = *reinterpret_cast<const uint4*>(ph + lo_off + 16);
   } else {
     bh[0] = bh[1] = bl[0] = bl[1] = make_uint4(0, 0, 0, 0);
   }
@@ -688,95 +687,156 @@ __device__ void finish_segment(const DecodeParams& p, const ExpertInfo& ex, int 
   }
 }
 
+// ---- phase C: down
+
+// This CTA's rows of y: [r0, r0 + nr).
+__device__ __forceinline__ void cta_rows(int& r0, int& nr) {
+  const int G = gridDim.x, c = blockIdx.x;
+  r0 = (c * kH) / G;
+  nr = ((c + 1) * kH) / G - r0;
+}
+
+// Warp-collective: phase C item `item` of this CTA into ring slot i. Items 0..7 are the shared
+// expert's down rows [r0, r0+16) over K slice 128*item (one 64-word x 16-row tensor box; rows past
+// r0+nr belong to the next CTA and are ignored, rows past H read as zero); item 8+gi is active
+// expert gi's down rows [r0, r0+nr) over all of K (nr * 256 contiguous bytes of codes) and their
+// scales (int4: from the even row at or below r0, an even row count, so that the copy is 16-byte
+// aligned; NVFP4: nr rows of 32 B).
 template <int FMT>
-__global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
-    decode_gate_up_kernel(const __grid_constant__ DecodeParams p) {
-  constexpr int kWarps = GuGeom<FMT>::kWarps, kDepth = GuGeom<FMT>::kDepth;
+__device__ void dn_issue(const DecodeParams& p, Ring<FMT>& ring, int item, int r0, int nr, const WarpTable& tab) {
+  const int lane = threadIdx.x & 31;
+  const int i = ring.issued++;
+  uint8_t* st = ring.slot_ptr(i);
+  uint64_t* bar = ring.bar(i);
+  if (item < kShDnSlices) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar, 16 * 256);
+      tma_load_2d(st, &p.tm_sh_dn, item * 64, r0, bar);
+    }
+    return;
+  }
+  const ExpertInfo ex = tab.get(p, item - kShDnSlices);
+  const size_t row0 = static_cast<size_t>(ex.e) * kH + r0;
+  if (lane == 0) {
+    if constexpr (FMT == kInt4) {
+      const size_t re = row0 & ~static_cast<size_t>(1);
+      const uint32_t nsc = static_cast<uint32_t>(((row0 + nr + 1) & ~static_cast<size_t>(1)) - re);   // even
+      mbar_arrive_expect_tx(bar, nr * 256 + nsc * 8);
+      bulk_g2s(st, p.dn_codes + row0 * (kI / 2), nr * 256, bar);
+      bulk_g2s(st + 4096, p.dn_scales + re * 8, nsc * 8, bar);
+    } else {
+      mbar_arrive_expect_tx(bar, nr * 256 + nr * 32);
+      bulk_g2s(st, p.dn_codes + row0 * (kI / 2), nr * 256, bar);
+      bulk_g2s(st + 4096, p.dn_scales + row0 * 32, nr * 32, bar);
+    }
+  }
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int D = Geom<FMT>::kDepth;
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  GuShared<FMT>& sm = *reinterpret_cast<GuShared<FMT>*>(smem_raw);
+  DecShared<FMT>& sm = *reinterpret_cast<DecShared<FMT>*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  GuWarp<FMT>& ws = sm.w[warp];
+  const int G = gridDim.x, c = blockIdx.x;
+  const GridBarrier gb{p.cnt + kCntBar, p.cnt + kCntBar + 1, p.cnt + kCntBar + 2};
+  Ring<FMT> ring;
+  ring.base = &sm.stage[warp][0][0];
+  ring.full = &sm.full[warp][0];
   if (lane == 0) {
 #pragma unroll
-    for (int i = 0; i < kDepth; ++i) mbar_init(&ws.full[i], 1);
-    fence_mbar_init();
+    for (int i = 0; i < D; ++i) mbar_init(&sm.full[warp][i], 1);
   }
-  __syncwarp();
-  const int ncta = gridDim.x;
-  auto tile_of = [&](int k) { return static_cast<int>(blockIdx.x) + ncta * (warp + kWarps * k); };
-  int na = -1;                                     // active experts; known after the grid dependency
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.xbar, 1);
+    mbar_init(&sm.xqbar, 1);
+    mbar_init(&sm.hqbar, 1);
+    mbar_init(&sm.route_ready, 1);
+    sm.gen0 = ld_acquire_gpu(gb.gen);
+  }
+  fence_mbar_init();
+  __syncthreads();
+  const int gen0 = sm.gen0;
+
+  // ---------------------------------------------------------------- phase A
+  // gate|up tile k of this warp (round robin over the CTAs first, then the warps)
+  auto tile_of = [&](int k) { return c + G * (warp + kWarps * k); };
+  if (threadIdx.x == 0) {                          // x (T token rows), one bulk copy per row
+    mbar_arrive_expect_tx(&sm.xbar, p.T * kH * 2);
+    for (int r = 0; r < p.T; ++r) bulk_g2s(sm.u.ab.xs[r], p.x + static_cast<size_t>(r) * kH, kH * 2, &sm.xbar);
+  } else if (threadIdx.x == 32) {                  // the shared expert's down rows into L2 for phase C
+    for (int ch = c; ch < kH * kIs * 2 / 32768; ch += G) prefetch_l2(p.sh_dn + static_cast<size_t>(ch) * 32768, 32768);
+  }
+  // shared-expert stages need no routing: the ring fills at once
+  int na = -1;                                     // active experts, once the routing is known
   WarpTable tab;
-  // Once per warp, the first time a routed tile is needed (or at the end). The routing warps wait
-  // for the route kernel and derive the routing from its logits (CTA 0 also publishes the tables);
-  // the first of them requests the operand rows and signals route_ready.
-  auto routing = [&]() {
-    if (na < 0) {
-      if (warp >= kRouteWarp0) {
-        pdl_wait();                                // the route kernel has finished and is visible
-        route_group(p, sm.rs, blockIdx.x == 0, warp - kRouteWarp0, kWarps - kRouteWarp0, 1);
-        // the down kernel reads CTA 0's published tables: they are visible before any trigger
-        if (blockIdx.x == 0) __threadfence();
-        pdl_trigger();
-        if (warp == kRouteWarp0) {
-          constexpr int kRow = 2 * kH;             // int4: hi + lo limbs; NVFP4: fp16
-          const uint8_t* src = FMT == kInt4 ? p.xq8 : reinterpret_cast<const uint8_t*>(p.xq);
-          if (lane == 0) mbar_arrive_expect_tx(&sm.xqbar, p.T * kRow + (FMT == kInt4 ? p.T * (kH / kGroup) * 4 : 0));
-          __syncwarp();
-          if (lane < p.T) bulk_g2s(sm.xq[lane], src + static_cast<size_t>(lane) * kRow, kRow, &sm.xqbar);
-          if (FMT == kInt4 && lane == 31) bulk_g2s(&sm.xsc[0][0], p.xsc, p.T * (kH / kGroup) * 4, &sm.xqbar);
-          if (lane == 0) mbar_arrive(&sm.route_ready);
-        }
-      } else {
-        pdl_wait();
-        wait_stage(p, &sm.route_ready, 0);
-        pdl_trigger();
+  int k_issue = 0;                                 // next gate|up stage to issue: tile k_issue >> 2, quarter & 3
+  while (ring.has_room() && tile_of(k_issue >> 2) < kShGuTiles) {
+    gu_issue<FMT>(p, sm, ring, warp, k_issue & 3, k_issue >> 2, tile_of(k_issue >> 2), ExpertInfo{});
+    ++k_issue;
+  }
+  if (warp >= kRouteWarp0) {
+    // router rows e = c + G*r (warps 4, 5) and the operand segments (warp 6)
+    const int rw = warp - kRouteWarp0;
+    uint4 w[8];
+    const int e = c + G * rw;
+    if (rw < 2 && e < p.E) load_router_row(w, p, e);
+    wait_stage(p, &sm.xbar, 0);
+    if (rw < 2) {
+      for (int ee = e; ee < p.E; ee += 2 * G) {
+        if (ee != e) load_router_row(w, p, ee);
+        route_row(p, ee, w, sm.u.ab.xs[0], kTokPitch);
       }
-      na = active_count(p, sm.rs);
-      tab.load(sm.rs);
+    } else if (rw == 2) {
+      for (int sg = c; sg < p.T * (kH / kGroup); sg += G)
+        xq_segment(p, sg / (kH / kGroup), sg % (kH / kGroup), sm.u.ab.xs[0], kTokPitch);
     }
-  };
-  auto valid = [&](int k) {                        // blocks until the routing is known if needed
-    const int tl = tile_of(k);
-    if (tl < kShGuTiles) return true;
-    routing();
-    return tl < kShGuTiles + kGuTilesPerExpert * na;
-  };
-  auto can_issue = [&](int k) {                    // as valid, but a shared-tile warp does not wait
-    if (na < 0 && warp < kRouteWarp0 && tile_of(k) >= kShGuTiles && !mbar_test_wait(&sm.route_ready, 0))
-      return false;
-    return valid(k);
+    // ------------------------------------------------------------ barrier 1: logits and operand
+    __threadfence();
+    named_bar_sync(kBarRoute, kRouteThreads);
+    if (threadIdx.x == kRouteWarp0 * 32) {
+      gb.arrive(G, gen0 + 1);
+      gb.wait(gen0 + 1, p.err);
+      fence_proxy_async_global();                  // the operand copy below reads other CTAs' writes
+      constexpr int kRow = 2 * kH;                 // int4: hi + lo limbs; NVFP4: fp16
+      const uint8_t* src = FMT == kInt4 ? p.xq8 : reinterpret_cast<const uint8_t*>(p.xq);
+      mbar_arrive_expect_tx(&sm.xqbar, p.T * kRow + (FMT == kInt4 ? p.T * (kH / kGroup) * 4 : 0));
+      for (int r = 0; r < p.T; ++r) bulk_g2s(sm.u.ab.xq[r], src + static_cast<size_t>(r) * kRow, kRow, &sm.xqbar);
+      if (FMT == kInt4) bulk_g2s(&sm.u.ab.xsc[0][0], p.xsc, p.T * (kH / kGroup) * 4, &sm.xqbar);
+    }
+    named_bar_sync(kBarRoute, kRouteThreads);
+    // ------------------------------------------------------------ phase B: routing
+    for (int tok = rw; tok < p.T; tok += kWarps - kRouteWarp0) topk_token(p, tok, sm.rs, c == 0);
+    named_bar_sync(kBarRoute, kRouteThreads);
+    if (rw == 0) build_tables(p, sm.rs, c == 0);
+    named_bar_sync(kBarRoute, kRouteThreads);
+    if (threadIdx.x == kRouteWarp0 * 32) mbar_arrive(&sm.route_ready);
+    na = active_count(p, sm.rs);
+    tab.load(sm.rs);
+  }
+  // ---------------------------------------------------------------- phase B: gate|up tiles
+  if (warp < kRouteWarp0) wait_stage(p, &sm.xbar, 0);   // the shared tiles read the staged x
+  auto routing_known = [&](bool block) {
+    if (na >= 0) return true;
+    if (!block && !mbar_test_wait(&sm.route_ready, 0)) return false;
+    wait_stage(p, &sm.route_ready, 0);
+    na = active_count(p, sm.rs);
+    tab.load(sm.rs);
+    return true;
   };
   auto info = [&](int tl) {
     ExpertInfo ex{};
     if (tl >= kShGuTiles) ex = tab.get(p, (tl - kShGuTiles) / kGuTilesPerExpert);
     return ex;
   };
-
-  // The shared expert's down weights need no routing either: into L2 now, in 32 KB chunks over the
-  // CTAs, for the down kernel.
-  if (threadIdx.x == 0)
-    for (int c = blockIdx.x; c < kH * kIs * 2 / 32768; c += gridDim.x) prefetch_l2(p.sh_dn + c * 32768, 32768);
-  // Shared-expert stages need no routing: request them first, then stage x and build the routed
-  // operand while the route kernel runs.
-  int s_issue = 0;
-  for (; s_issue < kDepth && tile_of(s_issue >> 2) < kShGuTiles; ++s_issue)
-    gu_issue(p, ws, s_issue, tile_of(s_issue >> 2), ExpertInfo{});
-  if (warp == 0) {                                 // the token rows of x, one bulk copy each
-    if (lane == 0) {
-      mbar_init(&sm.xbar, 1);
-      mbar_init(&sm.xqbar, 1);
-      mbar_init(&sm.route_ready, 1);
-      fence_mbar_init();
-      mbar_arrive_expect_tx(&sm.xbar, p.T * kH * 2);
-    }
-    __syncwarp();
-    if (lane < p.T) bulk_g2s(sm.xs[lane], p.x + static_cast<size_t>(lane) * kH, kH * 2, &sm.xbar);
-  }
-  __syncthreads();                                 // the barriers are initialised
-  wait_stage(p, &sm.xbar, 0);
+  // tile k exists (blocks for the routing when the tile is a routed one)
+  auto gu_valid = [&](int k) {
+    const int tl = tile_of(k);
+    if (tl < kShGuTiles) return true;
+    routing_known(true);
+    return tl < kShGuTiles + kGuTilesPerExpert * na;
+  };
   bool have_xq = false;
-
-  // the previous routed tile's segment arrival; the last arriver of a segment rotates it
   PendingArrival seg_arr;
   auto finish_last = [&](int key) {
     if (key < 0) return;
@@ -791,9 +851,17 @@ __global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
   const uint8_t* brow = nullptr;                   // this lane's activation row (column g)
   for (int s = 0;; ++s) {
     const int k = s >> 2, q = s & 3, tl = tile_of(k);
-    if (q == 0 && !valid(k)) break;
-    for (; s_issue < s + kDepth && can_issue(s_issue >> 2); ++s_issue)  // keep the ring full
-      gu_issue(p, ws, s_issue, tile_of(s_issue >> 2), info(tile_of(s_issue >> 2)));
+    if (q == 0 && !gu_valid(k)) break;
+    // keep the ring full; a shared-tile warp does not block on the routing to issue a routed stage
+    while (ring.has_room()) {
+      const int tk = tile_of(k_issue >> 2);
+      if (tk >= kShGuTiles) {
+        if (!routing_known(false)) break;
+        if (tk >= kShGuTiles + kGuTilesPerExpert * na) break;
+      }
+      gu_issue<FMT>(p, sm, ring, warp, k_issue & 3, k_issue >> 2, tk, info(tk));
+      ++k_issue;
+    }
     if (q == 0) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[0][i] = acc[1][i] = 0.f;
@@ -806,16 +874,16 @@ __global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
         bvalid = g < ex.n;
         tok0 = token_of(p, ex, 2 * t);
         tok1 = token_of(p, ex, 2 * t + 1);
-        brow = sm.xq[bvalid ? token_of(p, ex, g) : 0];
+        brow = sm.u.ab.xq[bvalid ? token_of(p, ex, g) : 0];
       }
     }
-    const int slot = s % kDepth;
-    wait_stage(p, &ws.full[slot], (s / kDepth) & 1);
-    const uint8_t* st = ws.stage[slot];
+    const int i = ring.consumed;
+    wait_stage(p, ring.bar(i), (i / D) & 1);
+    const uint8_t* st = ring.slot_ptr(i);
     if (tl < kShGuTiles) {
       // rows g = 0,1: gate 2tl, 2tl+1; g = 2,3: up 2tl, 2tl+1; MMA rows 4..15 are zero
       const bool xv = g < p.T;
-      const uint8_t* xr = sm.xs[xv ? g : 0];
+      const uint8_t* xr = sm.u.ab.xs[xv ? g : 0];
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         RawA<kBf16> A;
@@ -825,7 +893,7 @@ __global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
         bf16_group(acc, A, B, nullptr);
       }
     } else if constexpr (FMT == kInt4) {
-      const uint16_t* sc = reinterpret_cast<const uint16_t*>(ws.scales[k & 1]);
+      const uint16_t* sc = reinterpret_cast<const uint16_t*>(sm.gu_sc[warp][k & 1]);
       const bool v0 = 2 * t < ex.n, v1 = 2 * t + 1 < ex.n;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
@@ -833,14 +901,15 @@ __global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
         const uint4 ra = *reinterpret_cast<const uint4*>(st + g * 256 + jj * 64 + 16 * t);
         const uint4 rb = *reinterpret_cast<const uint4*>(st + (g + 8) * 256 + jj * 64 + 16 * t);
         uint4 bh[2], bl[2];
-        load_limbs_smem(bh, bl, brow, j, t, bvalid);
+        load_limbs_smem(bh, bl, brow, kH, j, t, bvalid);
         const float sg = bf16_bits_to_f32(sc[g * 16 + j]), su = bf16_bits_to_f32(sc[(8 + g) * 16 + j]);
-        const float x0 = v0 ? sm.xsc[tok0][j] : 0.f, x1 = v1 ? sm.xsc[tok1][j] : 0.f;
+        const float x0 = v0 ? sm.u.ab.xsc[tok0][j] : 0.f, x1 = v1 ? sm.u.ab.xsc[tok1][j] : 0.f;
         const float f[4] = {sg * x0, sg * x1, su * x0, su * x1};
         int4_group(acc[0], ra, rb, bh, bl, f);
       }
     } else {
-      const uint8_t* sc = ws.scales[k & 1];
+      // scales of the stage: gate rows 8 x 32 B at 4096, up rows at 4352 (blocks of this K quarter)
+      const uint8_t* sc = st + 4096;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const int j = 4 * q + jj;
@@ -848,24 +917,25 @@ __global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
         const uint4 rb = *reinterpret_cast<const uint4*>(st + (g + 8) * 256 + jj * 64 + 16 * t);
         RawB B;
         load_b_smem(B, brow, j, t, bvalid);
-        nvfp4_group(acc, ra, rb, B, sc + g * 128, sc + 1024 + g * 128, j, t);
+        nvfp4_group(acc, ra, rb, B, sc + g * 32, sc + 256 + g * 32, jj, t);
       }
     }
     __syncwarp();                                  // every lane's reads of the slot precede its refill
+    ring.consumed++;
     if (q != 3) continue;
     // ---- tile epilogue
-    float c[4];
+    float cc[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) c[i] = acc[0][i] + acc[1][i];
+    for (int i2 = 0; i2 < 4; ++i2) cc[i2] = acc[0][i2] + acc[1][i2];
     if (tl < kShGuTiles) {
-      const float u0 = __shfl_down_sync(kFull, c[0], 8), u1 = __shfl_down_sync(kFull, c[1], 8);
+      const float u0 = __shfl_down_sync(kFull, cc[0], 8), u1 = __shfl_down_sync(kFull, cc[1], 8);
       if (g < 2) {
         const float uv[2] = {u0, u1};
 #pragma unroll
         for (int qq = 0; qq < 2; ++qq) {
           const int tok = 2 * t + qq;
           if (tok < p.T) {
-            const float hs = silu(c[qq]) * uv[qq];
+            const float hs = silu(cc[qq]) * uv[qq];
             const uint16_t hi = f32_to_bf16_bits(hs);
             const uint16_t lo = f32_to_bf16_bits(hs - bf16_bits_to_f32(hi));
             p.hs_hi[tok * kIs + 2 * tl + g] = hi;
@@ -879,312 +949,153 @@ __global__ void __launch_bounds__(GuGeom<FMT>::kWarps * 32, 1)
       for (int qq = 0; qq < 2; ++qq) {
         const int col = 2 * t + qq;
         if (col < ex.n)
-          p.h32[static_cast<size_t>(ex.off + col) * kI + 8 * i8 + g] = silu(c[qq] * ex.tsg) * (c[2 + qq] * ex.tsu);
+          p.h32[static_cast<size_t>(ex.off + col) * kI + 8 * i8 + g] = silu(cc[qq] * ex.tsg) * (cc[2 + qq] * ex.tsu);
       }
       const int seg = i8 / (kGroup / 8);
       finish_last(seg_arr.settle());
       seg_arr.arrive(p.cnt, kCntSeg + 4 * gi + seg, kGroup / 8);
     }
   }
-  routing();                                       // every warp passes the grid dependency before it ends
+  routing_known(true);
   finish_last(seg_arr.settle());
-  if (!have_xq) wait_stage(p, &sm.xqbar, 0);       // no bulk copy may still write this CTA's memory
-}
+  if (warp == kRouteWarp0 && !have_xq) wait_stage(p, &sm.xqbar, 0);   // no copy may still write the operand rows
 
-// ============================================================================================ down
-
-// Warp-collective: stage q of tile `tile` (slot s mod depth). Shared tile sd: one tensor box with
-// Sd rows 8sd .. +8, K quarter q (512 B each). Routed tile (gi, b): 16 rows 32b + 16q .. +16 of the
-// expert's down rows, all of K (256 B each, contiguous), and their scales.
-template <int FMT>
-__device__ void dn_issue(const DecodeParams& p, DnWarp<FMT>& ws, int s, int q, int tile, const ExpertInfo& ex) {
-  const int lane = threadIdx.x & 31;
-  const int slot = s % DnGeom<FMT>::kDepth;
-  uint8_t* st = ws.stage[slot];
-  uint64_t* bar = &ws.full[slot];
-  if (tile < kShDnTiles) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar, 4096);
-      tma_load_2d(st, &p.tm_sh_dn, q * 128, 8 * tile, bar);
-    }
-    return;
+  // ---------------------------------------------------------------- phase C: first stages, barrier 2
+  int r0, nr;
+  cta_rows(r0, nr);
+  const int n_items = kShDnSlices + na;
+  int it_issue = warp;                             // this warp's items: warp, warp + 8, ...
+  while (ring.has_room() && it_issue < n_items) {
+    dn_issue<FMT>(p, ring, it_issue, r0, nr, tab);
+    it_issue += kWarps;
   }
-  const int n0 = 32 * ((tile - kShDnTiles) % kDnTilesPerExpert) + 16 * q;
-  const size_t row0 = static_cast<size_t>(ex.e) * kH + n0;
-  // scale bytes per row: int4 4 bf16 group scales, NVFP4 32 E4M3 block scales
-  const uint32_t row_sc = p.fmt == kInt4 ? (kI / kGroup) * 2 : kI / 16;
-  if (lane == 0) {
-    mbar_arrive_expect_tx(bar, 4096 + 16 * row_sc);
-    bulk_g2s(st, p.dn_codes + row0 * (kI / 2), 4096, bar);
-    bulk_g2s(st + 4096, p.dn_scales + row0 * row_sc, 16 * row_sc, bar);
-  }
-}
-
-__device__ __forceinline__ void prefetch_l1(const void* ptr) { asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr)); }
-
-// Warp: brings `bytes` bytes at base into this SM's L1, one 128-byte line per lane and step.
-__device__ __forceinline__ void prefetch_range(const void* base, size_t bytes) {
-  const uint8_t* b = static_cast<const uint8_t*>(base);
-  for (size_t o = static_cast<size_t>(threadIdx.x & 31) * 128; o < bytes; o += 32 * 128) prefetch_l1(b + o);
-}
-
-// Warp: L1 prefetch of the activation rows a shared down tile reads (hs of every token; call after
-// the grid dependency). Routed tiles read their operand from shared memory.
-__device__ void dn_prefetch(const DecodeParams& p, int tile, const ExpertInfo&) {
-  if (tile < kShDnTiles) {
-    prefetch_range(p.hs_hi, static_cast<size_t>(p.T) * kIs * 2);
-    prefetch_range(p.hs_lo, static_cast<size_t>(p.T) * kIs * 2);
-  }
-}
-
-// y rows nb*64 .. +64 of every token (one warp), slots in slot order. The (position, weight) of
-// every pair is fetched once (lane q holds pairs q and q + 32); lane l then owns rows 4(l mod 16)
-// .. +4 of token t0 + l/16, two tokens per round.
-__device__ void combine_block(const DecodeParams& p, const RouteSmem& rs, int nb) {
-  const int lane = threadIdx.x & 31;
-  const int n = nb * 64 + 4 * (lane & 15), K = p.K, P = p.T * K;
-  int pos[2];
-  float wt[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int q = lane + 32 * h;
-    pos[h] = q < P ? min(max(rs.inv[q], 0), P - 1) : 0;
-    wt[h] = q < P ? rs.w[q] : 0.f;
-  }
-#pragma unroll 1
-  for (int t0 = 0; t0 < p.T; t0 += 2) {
-    const int tok = t0 + (lane >> 4);
-    const bool tv = tok < p.T;
-    const float4 yv = tv ? __ldcg(reinterpret_cast<const float4*>(p.ys + tok * kH + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 ov[kMaxTopK];
-    float w[kMaxTopK];
-#pragma unroll
-    for (int k = 0; k < kMaxTopK; ++k) {
-      if (k < K) {
-        const int q = min(tok, p.T - 1) * K + k;         // per lane: read both halves of the table
-        const int p0 = __shfl_sync(kFull, pos[0], q & 31), p1 = __shfl_sync(kFull, pos[1], q & 31);
-        const float w0 = __shfl_sync(kFull, wt[0], q & 31), w1 = __shfl_sync(kFull, wt[1], q & 31);
-        w[k] = q < 32 ? w0 : w1;
-        ov[k] = tv ? __ldcg(reinterpret_cast<const float4*>(p.o + static_cast<size_t>(q < 32 ? p0 : p1) * kH + n))
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
-    if (tv) {
-      float a[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int k = 0; k < kMaxTopK; ++k)
-        if (k < K) {
-          a[0] = fmaf(w[k], ov[k].x, a[0]);
-          a[1] = fmaf(w[k], ov[k].y, a[1]);
-          a[2] = fmaf(w[k], ov[k].z, a[2]);
-          a[3] = fmaf(w[k], ov[k].w, a[3]);
-        }
-      uint2 out;
-      out.x = pack_bf162(fmaf(p.routed_scale, a[0], yv.x), fmaf(p.routed_scale, a[1], yv.y));
-      out.y = pack_bf162(fmaf(p.routed_scale, a[2], yv.z), fmaf(p.routed_scale, a[3], yv.w));
-      *reinterpret_cast<uint2*>(p.y + tok * kH + n) = out;
-    }
-  }
-}
-
-template <int FMT>
-__global__ void __launch_bounds__(DnGeom<FMT>::kWarps * 32, 1)
-    decode_down_kernel(const __grid_constant__ DecodeParams p) {
-  constexpr int kWarps = DnGeom<FMT>::kWarps, kDepth = DnGeom<FMT>::kDepth;
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  DnShared<FMT>& sm = *reinterpret_cast<DnShared<FMT>*>(smem_raw);
-  DnWarp<FMT>& ws = sm.w[warp];
-  if (lane == 0) {
-#pragma unroll
-    for (int i = 0; i < kDepth; ++i) mbar_init(&ws.full[i], 1);
-    if (warp == 0) mbar_init(&sm.hqbar, 1);
-    fence_mbar_init();
-  }
-  __syncwarp();
-  // This kernel starts only after every gate|up warp has triggered, and gate|up CTA 0 triggers only
-  // after publishing the routing tables (fenced): they are read here while gate|up still runs. The
-  // gate|up outputs are read only after pdl_wait below.
-  if (warp == 0) {
-    const int nact = min(max(__ldcg(p.n_active), 0), min(kMaxActive, p.T * p.K));
-    for (int gi = lane; gi < nact; gi += 32) {
-      sm.rs.etab[gi][0] = __ldcg(p.etab + 2 * gi);
-      sm.rs.etab[gi][1] = __ldcg(p.etab + 2 * gi + 1);
-    }
-    for (int q = lane; q < p.T * p.K; q += 32) {
-      sm.rs.inv[q] = __ldcg(p.inv + q);
-      sm.rs.w[q] = __ldcg(p.wts + q);
-    }
-    if (lane == 0) sm.rs.na = nact;
-  }
-  __syncthreads();
-  const int na = active_count(p, sm.rs);
-  WarpTable tab;
-  tab.load(sm.rs);
-  const int n_tiles = kShDnTiles + kDnTilesPerExpert * na;
-  const int ncta = gridDim.x;
-  auto tile_of = [&](int k) { return static_cast<int>(blockIdx.x) + ncta * (warp + kWarps * k); };
-  auto info = [&](int tl) {
-    ExpertInfo ex{};
-    if (tl >= kShDnTiles) ex = tab.get(p, (tl - kShDnTiles) / kDnTilesPerExpert);
-    return ex;
-  };
-  // Stage s of this warp -> (tile ordinal k, stage q in the tile): a shared tile has 4 stages and can
-  // only be a warp's first tile (ncta * kWarps > kShDnTiles), routed tiles have 2.
-  const int first_len = tile_of(0) < kShDnTiles ? 4 : 2;
-  auto stage_k = [&](int s) { return s < first_len ? 0 : 1 + (s - first_len) / 2; };
-  auto stage_q = [&](int s) { return s < first_len ? s : (s - first_len) % 2; };
-  auto issue = [&](int s) {
-    const int tl = tile_of(stage_k(s));
-    dn_issue<FMT>(p, ws, s, stage_q(s), tl, info(tl));
-  };
-  int s_issue = 0;
-  for (; s_issue < kDepth && tile_of(stage_k(s_issue)) < n_tiles; ++s_issue) issue(s_issue);
-  pdl_wait();                                      // h and hs of the gate|up kernel
-  if (warp == 0 && lane == 0) {                    // the down operand of every position, one copy
+  __syncthreads();                                 // every warp's h, hs and operand writes are done
+  if (threadIdx.x == 0) {
+    gb.arrive(G, gen0 + 2);
+    gb.wait(gen0 + 2, p.err);
+    fence_proxy_async_global();
     const int P = p.T * p.K;
+    const uint8_t* src = FMT == kInt4 ? p.hq8 : reinterpret_cast<const uint8_t*>(p.hq);
     mbar_arrive_expect_tx(&sm.hqbar, P * 2 * kI + (FMT == kInt4 ? P * (kI / kGroup) * 4 : 0));
-    bulk_g2s(&sm.hq[0][0], FMT == kInt4 ? p.hq8 : reinterpret_cast<const uint8_t*>(p.hq), P * 2 * kI, &sm.hqbar);
-    if (FMT == kInt4) bulk_g2s(&sm.hsc[0][0], p.hsc, P * (kI / kGroup) * 4, &sm.hqbar);
+    bulk_g2s(&sm.u.c.hq[0][0], src, P * 2 * kI, &sm.hqbar);
+    if (FMT == kInt4) bulk_g2s(&sm.u.c.hsc[0][0], p.hsc, P * (kI / kGroup) * 4, &sm.hqbar);
   }
-  bool have_hq = false;
-  if (tile_of(0) < n_tiles) dn_prefetch(p, tile_of(0), info(tile_of(0)));
+  __syncthreads();                                 // the grid barrier is passed for every thread
 
-  // the previous tile's block arrival; the last arriver of a 64-row block combines it
-  PendingArrival blk_arr;
-  auto combine_last = [&](int key) {
-    if (key < 0) return;
-    combine_block(p, sm.rs, key - kCntBlk);
-    if (lane == 0) p.cnt[key] = 0;
-  };
-  float acc[2][2][4];                              // [16-row half][accumulator set][fragment]
-  ExpertInfo ex{};
-  const int target = 2 * na + kShDnTiles / (kH / 64);
-  for (int s = 0;; ++s) {
-    const int k = stage_k(s), q = stage_q(s), tl = tile_of(k);
-    if (tl >= n_tiles) break;
-    if (q == 0) {
+  // ---------------------------------------------------------------- phase C: down items
+  bool have_hq = false;
+  for (int it = warp; it < n_items; it += kWarps) {
+    const int i = ring.consumed;
+    wait_stage(p, ring.bar(i), (i / D) & 1);
+    const uint8_t* st = ring.slot_ptr(i);
+    float dacc[2][4];
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
+    for (int a = 0; a < 2; ++a)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[h][0][i] = acc[h][1][i] = 0.f;
-      if (tl >= kShDnTiles) ex = info(tl);
-      if (tile_of(k + 1) < n_tiles) dn_prefetch(p, tile_of(k + 1), info(tile_of(k + 1)));
-    }
-    const int slot = s % kDepth;
-    wait_stage(p, &ws.full[slot], (s / kDepth) & 1);
-    const uint8_t* st = ws.stage[slot];
-    if (tl < kShDnTiles) {
-      // rows 8tl + g (g < 8) of Sd, K quarter q (groups 2q, 2q+1); hs as a bf16 pair (hi + lo)
+      for (int b = 0; b < 4; ++b) dacc[a][b] = 0.f;
+    if (it < kShDnSlices) {
+      // rows g, g+8 of the box (row r at r * 256: K elements 128j .. 128j + 127, bf16) against K
+      // slice j of hs (bf16 hi + lo pair, written by other CTAs: read through L2)
+      const int j = it;
       const bool bv = g < p.T;
       const size_t r = static_cast<size_t>(bv ? g : 0) * kIs;
+      RawA<kBf16> A;
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        RawA<kBf16> A;
-        load_a_bf16_rows(A, st, 512, 8, g, jj, t);
-        RawB Bh, Bl;
-        Bh.load(p.hs_hi + r, 2 * q + jj, t, bv);
-        Bl.load(p.hs_lo + r, 2 * q + jj, t, bv);
-        bf16_group(acc[0], A, Bh, &Bl);
+      for (int qd = 0; qd < 4; ++qd) {
+        A.r0[qd] = *reinterpret_cast<const uint4*>(st + g * 256 + (32 * t) * 2 + 16 * qd);
+        A.r1[qd] = *reinterpret_cast<const uint4*>(st + (g + 8) * 256 + (32 * t) * 2 + 16 * qd);
+      }
+      RawB Bh, Bl;
+      Bh.load_cg(p.hs_hi + r, j, t, bv);
+      Bl.load_cg(p.hs_lo + r, j, t, bv);
+      bf16_group(dacc, A, Bh, &Bl);
+      float cs[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) cs[b] = dacc[0][b] + dacc[1][b];
+      // {row g, tok 2t}, {g, 2t+1}, {g+8, 2t}, {g+8, 2t+1}
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int tok = 2 * t + (b & 1), row = g + 8 * (b >> 1);
+        if (tok < p.T) sm.u.c.spart[j][tok][row] = cs[b];
       }
     } else {
-      // 16 rows (half q of the 32-row tile), all of K = 4 groups
       if (!have_hq) {
         wait_stage(p, &sm.hqbar, 0);
         have_hq = true;
       }
-      const bool bv = g < ex.n;
-      const uint8_t* hrow = sm.hq[ex.off + (bv ? g : 0)];
-      const uint8_t* sc = st + 4096;
+      const ExpertInfo e2 = tab.get(p, it - kShDnSlices);
+      const bool bv = g < e2.n;
+      const uint8_t* hrow = sm.u.c.hq[e2.off + (bv ? g : 0)];
+      // rows g, g+8 of the stage (row r at r * 256); rows >= nr are the next expert's or beyond:
+      // they are read (inside the stage) but their results are dropped
+      const uint8_t* ra_p = st + g * 256;
+      const uint8_t* rb_p = st + (g + 8) * 256;
       if constexpr (FMT == kInt4) {
-        const uint16_t* s16 = reinterpret_cast<const uint16_t*>(sc);
-        const bool v0 = 2 * t < ex.n, v1 = 2 * t + 1 < ex.n;
-        const float* x0p = sm.hsc[ex.off + (v0 ? 2 * t : 0)];
-        const float* x1p = sm.hsc[ex.off + (v1 ? 2 * t + 1 : 0)];
+        // scales: row r's 4 bf16 at 4096 + (r + (r0 & 1)) * 8 (the copy starts at an even row)
+        const uint16_t* s16 = reinterpret_cast<const uint16_t*>(st + 4096) + (r0 & 1) * 4;
+        const bool v0 = 2 * t < e2.n, v1 = 2 * t + 1 < e2.n;
+        const float* x0p = sm.u.c.hsc[e2.off + (v0 ? 2 * t : 0)];
+        const float* x1p = sm.u.c.hsc[e2.off + (v1 ? 2 * t + 1 : 0)];
+        const int ga = min(g, nr - 1), gb2 = min(g + 8, nr - 1);
 #pragma unroll
         for (int j = 0; j < kI / kGroup; ++j) {
-          const uint4 ra = *reinterpret_cast<const uint4*>(st + g * 256 + j * 64 + 16 * t);
-          const uint4 rb = *reinterpret_cast<const uint4*>(st + (g + 8) * 256 + j * 64 + 16 * t);
+          const uint4 ra = *reinterpret_cast<const uint4*>(ra_p + j * 64 + 16 * t);
+          const uint4 rb = *reinterpret_cast<const uint4*>(rb_p + j * 64 + 16 * t);
           uint4 bh[2], bl[2];
-          if (bv) {
-            const uint8_t* ph = hrow + j * 128 + 32 * t;
-            bh[0] = *reinterpret_cast<const uint4*>(ph);
-            bh[1] = *reinterpret_cast<const uint4*>(ph + 16);
-            bl[0] = *reinterpret_cast<const uint4*>(ph + kI);
-            bl[1] = *reinterpret_cast<const uint4*>(ph + kI + 16);
-          } else {
-            bh[0] = bh[1] = bl[0] = bl[1] = make_uint4(0, 0, 0, 0);
-          }
-          const float s0 = bf16_bits_to_f32(s16[g * 4 + j]), s1 = bf16_bits_to_f32(s16[(g + 8) * 4 + j]);
+          load_limbs_smem(bh, bl, hrow, kI, j, t, bv);
+          const float s0 = bf16_bits_to_f32(s16[ga * 4 + j]), s1 = bf16_bits_to_f32(s16[gb2 * 4 + j]);
           const float x0 = v0 ? x0p[j] : 0.f, x1 = v1 ? x1p[j] : 0.f;
           const float f[4] = {s0 * x0, s0 * x1, s1 * x0, s1 * x1};
-          int4_group(acc[q][0], ra, rb, bh, bl, f);
+          int4_group(dacc[0], ra, rb, bh, bl, f);
         }
       } else {
+        const uint8_t* sc = st + 4096;
+        const int ga = min(g, nr - 1), gb2 = min(g + 8, nr - 1);
 #pragma unroll
         for (int j = 0; j < kI / kGroup; ++j) {
-          const uint4 ra = *reinterpret_cast<const uint4*>(st + g * 256 + j * 64 + 16 * t);
-          const uint4 rb = *reinterpret_cast<const uint4*>(st + (g + 8) * 256 + j * 64 + 16 * t);
+          const uint4 ra = *reinterpret_cast<const uint4*>(ra_p + j * 64 + 16 * t);
+          const uint4 rb = *reinterpret_cast<const uint4*>(rb_p + j * 64 + 16 * t);
           RawB B;
           load_b_smem(B, hrow, j, t, bv);
-          nvfp4_group(acc[q], ra, rb, B, sc + g * 32, sc + (g + 8) * 32, j, t);
+          nvfp4_group(dacc, ra, rb, B, sc + ga * 32, sc + gb2 * 32, j, t);
         }
       }
-    }
-    __syncwarp();                                  // every lane's reads of the slot precede its refill
-    if (tile_of(stage_k(s_issue)) < n_tiles) {     // s_issue == s + kDepth: refill this slot
-      issue(s_issue);
-      ++s_issue;
-    }
-    if (q != (tl < kShDnTiles ? 3 : 1)) continue;
-    // ---- tile epilogue
-    int nb;
-    if (tl < kShDnTiles) {
-      const int n0 = 8 * tl;
+      float cs[4];
 #pragma unroll
-      for (int qq = 0; qq < 2; ++qq) {
-        const int tok = 2 * t + qq;
-        if (tok < p.T) p.ys[tok * kH + n0 + g] = acc[0][0][qq] + acc[0][1][qq];
+      for (int b = 0; b < 4; ++b) cs[b] = dacc[0][b] + dacc[1][b];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int col = 2 * t + (b & 1), row = g + 8 * (b >> 1);
+        if (col < e2.n) sm.u.c.opart[e2.off + col][row] = cs[b] * e2.tsd;
       }
-      nb = n0 / 64;
-    } else {
-      const int b = (tl - kShDnTiles) % kDnTilesPerExpert;
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const int col = 2 * t + (qq & 1);
-          if (col < ex.n)
-            p.o[static_cast<size_t>(ex.off + col) * kH + 32 * b + 16 * h + g + 8 * (qq >> 1)] =
-                (acc[h][0][qq] + acc[h][1][qq]) * ex.tsd;
-        }
-      nb = b / 2;
     }
-    combine_last(blk_arr.settle());
-    blk_arr.arrive(p.cnt, kCntBlk + nb, target);
+    __syncwarp();
+    ring.consumed++;
+    if (it_issue < n_items) {                      // refill the slot just consumed
+      dn_issue<FMT>(p, ring, it_issue, r0, nr, tab);
+      it_issue += kWarps;
+    }
   }
-  combine_last(blk_arr.settle());
-  if (!have_hq) wait_stage(p, &sm.hqbar, 0);       // no bulk copy may still write this CTA's memory
+  if (warp == 0 && !have_hq) wait_stage(p, &sm.hqbar, 0);   // no copy may still write this CTA's memory
+  __syncthreads();
+  // ---------------------------------------------------------------- combine this CTA's rows
+  for (int idx = threadIdx.x; idx < p.T * nr; idx += kThreads) {
+    const int tok = idx / nr, rl = idx % nr, n = r0 + rl;
+    float ys = 0.f;
+#pragma unroll
+    for (int j = 0; j < kShDnSlices; ++j) ys += sm.u.c.spart[j][tok][rl];
+    float a = 0.f;
+    for (int k = 0; k < p.K; ++k) {
+      const int q = tok * p.K + k;
+      const int pos = min(max(sm.rs.inv[q], 0), p.T * p.K - 1);
+      a = fmaf(sm.rs.w[q], sm.u.c.opart[pos][rl], a);
+    }
+    p.ys[tok * kH + n] = ys;
+    p.y[tok * kH + n] = f32_to_bf16_bits(fmaf(p.routed_scale, a, ys));
+  }
 }
 
-template <typename Kern>
-cudaError_t launch_ex(Kern kernel, int grid, int threads, size_t smem, bool pdl, cudaStream_t s,
-                      const DecodeParams& p) {
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, p);
-}
-
-// Dynamic shared memory limit, and the same L1/shared split for every decode kernel so that an SM
-// need not be reconfigured between them.
+// Dynamic shared memory limit and the carve-out, once per kernel.
 template <typename Kern>
 cudaError_t allow_smem(Kern kernel, size_t bytes) {
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
@@ -1194,32 +1105,34 @@ cudaError_t allow_smem(Kern kernel, size_t bytes) {
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeParams& p, int n_sm, cudaStream_t s, cudaEvent_t ev_after_route,
-                          cudaEvent_t ev_after_gate_up) {
-  constexpr size_t kGuSmem4 = sizeof(GuShared<kInt4>), kGuSmemF = sizeof(GuShared<kNvfp4>);
-  constexpr size_t kDnSmem4 = sizeof(DnShared<kInt4>), kDnSmemF = sizeof(DnShared<kNvfp4>);
-  static_assert(kGuSmem4 <= 227 * 1024 && kGuSmemF <= 227 * 1024 && kDnSmem4 <= 227 * 1024 && kDnSmemF <= 227 * 1024,
+size_t decode_smem_bytes(int fmt) { return fmt == kInt4 ? sizeof(DecShared<kInt4>) : sizeof(DecShared<kNvfp4>); }
+
+cudaError_t decode_check_residency(int fmt, int* blocks_per_sm) {
+  const size_t smem = decode_smem_bytes(fmt);
+  cudaError_t e = fmt == kInt4 ? allow_smem(decode_layer_kernel<kInt4>, smem)
+                               : allow_smem(decode_layer_kernel<kNvfp4>, smem);
+  if (e != cudaSuccess) return e;
+  return fmt == kInt4
+             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, decode_layer_kernel<kInt4>, kThreads, smem)
+             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, decode_layer_kernel<kNvfp4>, kThreads, smem);
+}
+
+cudaError_t launch_decode(const DecodeParams& p, int n_sm, cudaStream_t s) {
+  static_assert(sizeof(DecShared<kInt4>) <= 227 * 1024 && sizeof(DecShared<kNvfp4>) <= 227 * 1024,
                 "shared memory per CTA");
-  static bool smem_set = false;                    // per process; the attribute is per function
-  if (!smem_set) {
-    cudaError_t e;
-    if ((e = allow_smem(decode_gate_up_kernel<kInt4>, kGuSmem4)) != cudaSuccess) return e;
-    if ((e = allow_smem(decode_gate_up_kernel<kNvfp4>, kGuSmemF)) != cudaSuccess) return e;
-    if ((e = allow_smem(decode_down_kernel<kInt4>, kDnSmem4)) != cudaSuccess) return e;
-    if ((e = allow_smem(decode_down_kernel<kNvfp4>, kDnSmemF)) != cudaSuccess) return e;
-    if ((e = allow_smem(decode_route_kernel, 0)) != cudaSuccess) return e;
-    smem_set = true;
-  }
-  cudaError_t e = launch_ex(decode_route_kernel, (p.E + kRouteWarps - 1) / kRouteWarps, kRouteWarps * 32, 0, false,
-                            s, p);
-  if (e != cudaSuccess) return e;
-  if (ev_after_route && (e = cudaEventRecord(ev_after_route, s)) != cudaSuccess) return e;
-  e = p.fmt == kInt4 ? launch_ex(decode_gate_up_kernel<kInt4>, n_sm, GuGeom<kInt4>::kWarps * 32, kGuSmem4, true, s, p)
-                     : launch_ex(decode_gate_up_kernel<kNvfp4>, n_sm, GuGeom<kNvfp4>::kWarps * 32, kGuSmemF, true, s, p);
-  if (e != cudaSuccess) return e;
-  if (ev_after_gate_up && (e = cudaEventRecord(ev_after_gate_up, s)) != cudaSuccess) return e;
-  return p.fmt == kInt4 ? launch_ex(decode_down_kernel<kInt4>, n_sm, DnGeom<kInt4>::kWarps * 32, kDnSmem4, true, s, p)
-                        : launch_ex(decode_down_kernel<kNvfp4>, n_sm, DnGeom<kNvfp4>::kWarps * 32, kDnSmemF, true, s, p);
+  const size_t smem = decode_smem_bytes(p.fmt);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(n_sm);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;     // every CTA resident at once: the grid barriers need it
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return p.fmt == kInt4 ? cudaLaunchKernelEx(&cfg, decode_layer_kernel<kInt4>, p)
+                        : cudaLaunchKernelEx(&cfg, decode_layer_kernel<kNvfp4>, p);
 }
 
 }  // namespace flint

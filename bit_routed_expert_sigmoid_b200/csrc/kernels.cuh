@@ -8,22 +8,23 @@
 
 namespace flint {
 
-// ---- decode path (T <= kDecodeMaxT): three kernels chained by programmatic dependent launch ----
+// ---- decode path (T <= kDecodeMaxT): one persistent kernel, launched cooperatively ----
 constexpr int kDecodeMaxT = 8;
 constexpr int kMaxActive = 64;                 // active experts of a decode forward (T * top_k <= 64)
-// Counters of the decode kernels (ints in the workspace, zero between forwards; each is reset by
-// the last arriver that reads it).
+// Words of the decode kernel in the workspace (zeroed at create): the grid barrier (arrival count,
+// generation, abort word) and the arrival counters of the 128-segments of h (each reset to zero by
+// its last arriver).
 enum : int {
-  kCntRoute = 0,                               // route CTAs finished
+  kCntBar = 0,                                 // [3]: count, generation, abort
   kCntSeg = 32,                                // [kMaxActive][4] gate|up tiles finished per 128-segment of h
-  kCntBlk = kCntSeg + 4 * kMaxActive,          // [H/64] down tiles finished per 64-row block of y
-  kCntInts = kCntBlk + kH / 64
+  kCntInts = kCntSeg + 4 * kMaxActive
 };
 
 struct DecodeParams {
   CUtensorMap tm_gu;              // gate|up codes as 32-bit words [E*2I][H/8], box 64 words x 8 rows
+  CUtensorMap tm_gu_sc;           // NVFP4 gate|up block scales as words [E*2I][H/64], box 8 words x 8 rows
   CUtensorMap tm_sh_gu;           // shared gate|up rows as 32-bit words [2Is][H/2], box 256 words x 2 rows
-  CUtensorMap tm_sh_dn;           // shared down rows as 32-bit words [H][Is/2], box 128 words x 8 rows
+  CUtensorMap tm_sh_dn;           // shared down rows as 32-bit words [H][Is/2], box 64 words x 16 rows
   int fmt, T, E, K;
   float floor_, routed_scale;
   const uint16_t* x;              // [T][H] bf16
@@ -56,16 +57,16 @@ struct DecodeParams {
   float* hsc;                     // int4: [P][I/128] unit of hq8, / 16
   uint16_t* hs_hi;                // [T][Is] shared-expert SwiGLU output, bf16 pair
   uint16_t* hs_lo;
-  float* o;                       // [P][H] routed down outputs
   float* ys;                      // [T][H] shared-expert output
   unsigned* err;
   int* cnt;                       // [kCntInts]
 };
 
-// Launches the three decode kernels on `s`; with `events` (n_events >= 2) an event is recorded
-// after the first and second kernel (which serialises them; for instrumentation only).
-cudaError_t launch_decode(const DecodeParams& p, int n_sm, cudaStream_t s, cudaEvent_t ev_after_route,
-                          cudaEvent_t ev_after_gate_up);
+// Launches the decode kernel on `s` (grid = n_sm CTAs, cooperative). The caller has checked with
+// decode_check_residency that one CTA fits per SM, and that n_sm >= kH / 16.
+cudaError_t launch_decode(const DecodeParams& p, int n_sm, cudaStream_t s);
+// Sets the kernel's shared-memory attributes and reports how many of its CTAs fit on one SM.
+cudaError_t decode_check_residency(int fmt, int* blocks_per_sm);
 
 // ---- prefill path (T > kDecodeMaxT): tcgen05 grouped GEMMs ----
 enum PfPhase : int { kPhaseGateUp = 0, kPhaseDown = 1, kPhaseRouter = 2 };

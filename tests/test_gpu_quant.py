@@ -81,31 +81,32 @@ def check_int4(w, rotate, codes, scales):
     assert np.all(cg[~amb_e] == cr[~amb_e])
     assert np.all(np.abs(cg - cr)[~np.repeat(amb_g, 128, axis=1)] <= 1)
     # exact ties (the exact quotient is a half-integer) may go either way under any fp32 arithmetic;
-    # the other ambiguous positions are counted and bounded (the test matrices hold rows of exact and
-    # near ties on purpose, so the bound is loose there; on random weights the count is ~1e-4)
+    # the other ambiguous positions are counted and bounded, so that the comparison covers at least
+    # 95 % of the codes (bf16 weights put many quotients within a few fp32 ulps of a boundary: the
+    # test matrices hold rows of ties on purpose, and random bf16 weights give ~1e-3 of them)
     ties = mg["code"] == 0
     n_near = int((amb_e & ~ties).sum())
-    assert n_near <= max(16, 0.02 * amb_e.size), n_near
+    assert n_near <= max(16, 0.05 * amb_e.size), n_near
     return {"exact_ties": int(ties.sum()), "near_boundary": n_near, "ambiguous_groups": int(amb_g.sum()),
             "differing_codes": int((cg != cr).sum())}
 
 
 def check_nvfp4(w, codes, scales, ts):
     """GPU NVFP4 codes, block scales and tensor scale against the fp64 oracle. The kernels form 6 ts,
-    the block quotient, d = sb ts and 1/d in fp32, a few 2^-24 relative each; decisions closer than
-    2^-20 (block scales) or 2^-19 (codes) to their boundary may go either way."""
+    the block quotient, d = sb ts and 1/d in fp32, each within 2^-24 relative; decisions closer than
+    2^-22 (block scales: two roundings) or 2^-21 (codes: three) to their boundary may go either way."""
     ref = Q.quantize_nvfp4(w)
     mg = Q.nvfp4_margins(w)
     assert ts == ref["tscale"]
-    amb_b = mg["scale"] < 2.0 ** -20
-    amb_e = (mg["code"] < 2.0 ** -19) | np.repeat(amb_b, 16, axis=1)
+    amb_b = mg["scale"] < 2.0 ** -22
+    amb_e = (mg["code"] < 2.0 ** -21) | np.repeat(amb_b, 16, axis=1)
     assert np.all(scales[~amb_b] == ref["scales"][~amb_b])
     vg = R.e2m1_to_f64(R.unpack_nibbles(codes))
     vr = R.e2m1_to_f64(R.unpack_nibbles(ref["codes"]))
     assert np.all(vg[~amb_e] == vr[~amb_e])
     ties = mg["code"] == 0
     n_near = int((amb_e & ~ties).sum())
-    assert n_near <= max(16, 0.02 * amb_e.size), n_near
+    assert n_near <= max(16, 0.05 * amb_e.size), n_near
     return {"exact_ties": int(ties.sum()), "near_boundary": n_near, "ambiguous_blocks": int(amb_b.sum()),
             "differing_codes": int((vg != vr).sum())}
 
