@@ -148,13 +148,15 @@ __device__ __forceinline__ void red_relaxed_add(int* p, int v) {
 constexpr uint32_t kWaitSleepNs = 20000;      // longest sleep of a bounded wait between clock checks
 
 // Waits for the barrier phase with the given parity; gives up after `limit_ns` and returns false.
+// The clock is read every 16th poll only, so that waiting warps take few issue slots from working
+// ones.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) {
-    if (globaltimer_ns() - t0 > limit_ns) return false;
+  for (unsigned i = 1;; ++i) {
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if ((i & 15u) == 0u && globaltimer_ns() - t0 > limit_ns) return false;
   }
-  return true;
 }
 
 // Bulk copy global -> this CTA's shared memory, completing `bytes` of transaction on `bar`.

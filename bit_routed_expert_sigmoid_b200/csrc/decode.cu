@@ -74,32 +74,42 @@ __device__ __forceinline__ int atom_add_acq_rel(int* ctr, int v) {
   return old;
 }
 
-__device__ __forceinline__ void st_relaxed_gpu(int* p, int v) {
-  asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// A warp's arrival on a counter whose result is examined later: the warp barrier orders every
-// lane's earlier global writes before lane 0's release; the returned value is only waited for when
-// settle() reads it (typically one tile later), so the atomic's latency overlaps the next tile.
-// settle() returns the counter index if this arrival brought the counter to `target` (the warp is
-// the last arriver, and lane 0's acquire precedes every lane's later reads), else -1.
-struct PendingArrival {
-  int key = -1;                             // counter index, -1 when nothing is pending
-  int target = 0;
-  int old = 0;                              // lane 0: value before the add
-  __device__ __forceinline__ void arrive(int* cnt, int k, int tgt) {
+// A warp's arrivals on segment counters whose results are examined only at the end of the phase:
+// the warp barrier orders every lane's earlier global writes before lane 0's acquire-release add,
+// and the add's return value is not read until settle(), so no tile waits for an atomic's round
+// trip. Up to four arrivals are held (a warp has at most four routed gate|up tiles at the shapes
+// this kernel runs; a fifth settles the first four early). settle() calls finish(counter index) for
+// each counter this warp's arrival completed (the returned value was target - 1: the warp was the
+// last arriver, and lane 0's acquire precedes every lane's later reads).
+struct PendingArrivals {
+  int key0 = -1, key1 = -1, key2 = -1, key3 = -1;   // counter indices, -1 when the slot is empty
+  int old0 = 0, old1 = 0, old2 = 0, old3 = 0;       // lane 0: value before the add
+  int n = 0;
+  __device__ __forceinline__ void arrive(int* cnt, int k) {
     __syncwarp();
-    if ((threadIdx.x & 31) == 0) old = atom_add_acq_rel(cnt + k, 1);
-    key = k;
-    target = tgt;
+    const bool l0 = (threadIdx.x & 31) == 0;
+    switch (n) {
+      case 0: key0 = k; if (l0) old0 = atom_add_acq_rel(cnt + k, 1); break;
+      case 1: key1 = k; if (l0) old1 = atom_add_acq_rel(cnt + k, 1); break;
+      case 2: key2 = k; if (l0) old2 = atom_add_acq_rel(cnt + k, 1); break;
+      default: key3 = k; if (l0) old3 = atom_add_acq_rel(cnt + k, 1); break;
+    }
+    ++n;
   }
-  __device__ __forceinline__ int settle() {
-    if (key < 0) return -1;
-    const int o = __shfl_sync(kFull, old, 0);
-    const int k = key;
-    key = -1;
-    __syncwarp();
-    return o == target - 1 ? k : -1;
+  __device__ __forceinline__ bool full() const { return n >= 4; }
+  template <typename F>
+  __device__ __forceinline__ void settle(int target, F&& finish) {
+    const int keys[4] = {key0, key1, key2, key3};
+    const int olds[4] = {old0, old1, old2, old3};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (i < n) {
+        const int o = __shfl_sync(kFull, olds[i], 0);
+        __syncwarp();
+        if (o == target - 1) finish(keys[i]);
+      }
+    }
+    n = 0;
   }
 };
 
@@ -115,39 +125,42 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 
 // ------------------------------------------------------------------------------------ grid barrier
 
-// Barrier words in global memory (zeroed at handle creation): an arrival count, a generation that
-// the last arriver advances, and an abort word. A CTA's thread 0 reads the generation at the start
-// of the forward (it cannot change before every CTA has arrived once), so barrier b of the forward
-// is passed when the generation equals start + b.
+// A 64-bit arrival counter in global memory (zeroed at handle creation) that only ever grows: every
+// CTA adds 1 at each of the forward's two barriers, so a forward adds 2G. At its start a CTA reads the
+// counter; no barrier of this forward can have completed yet (this CTA has not arrived), so the value
+// lies in [base, base + G) and base = value - value mod 2G. Barrier b is passed once the counter
+// reaches base + b*G. An arrival is one fire-and-forget reduction with release semantics; a wait polls
+// with acquire loads and gives up after 1 s (setting the timeout bit and the abort word, which makes
+// every later wait of the forward return at once).
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
 struct GridBarrier {
-  int* count;
-  int* gen;
+  unsigned long long* count;
   int* abort_;
-  // One thread per CTA, after the CTA's writes that must be visible are ordered before it by a
-  // CTA barrier: arrive, and if last, reset the count and advance the generation (release).
-  __device__ __forceinline__ void arrive(int nblocks, int target) const {
+  // One thread per CTA, after the CTA's writes that must be visible are ordered before it by a CTA
+  // barrier.
+  __device__ __forceinline__ void arrive() const {
     __threadfence();
-    const int old = atom_add_acq_rel(count, 1);
-    if (old == nblocks - 1) {
-      st_relaxed_gpu(count, 0);
-      st_release_gpu(gen, target);
-    }
+    asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(count) : "memory");
   }
-  // Bounded wait of one thread for generation `target`; false on timeout or abort.
-  __device__ __forceinline__ bool wait(int target, unsigned* err) const {
-    if (ld_acquire_gpu(gen) == target) return true;
+  // Bounded wait of one thread until the counter reaches `target`; false on timeout or abort.
+  __device__ __forceinline__ bool wait(unsigned long long target, unsigned* err) const {
+    if (ld_acquire_u64(count) >= target) return true;
     const uint64_t t0 = globaltimer_ns();
-    unsigned ns = 32;
-    for (;;) {
-      if (ld_acquire_gpu(gen) == target) return true;
+    for (unsigned i = 1;; ++i) {
+      __nanosleep(32);
+      if (ld_acquire_u64(count) >= target) return true;
+      if ((i & 15u) != 0u) continue;               // abort word and clock every 16th poll
       if (ld_relaxed_gpu(abort_) != 0) return false;
       if (globaltimer_ns() - t0 > kWaitNs) {
         atomicOr(err, kErrTimeout);
         atomicExch(abort_, 1);
         return false;
       }
-      __nanosleep(ns);
-      if (ns < 256) ns <<= 1;
     }
   }
 };
@@ -221,28 +234,26 @@ __device__ __forceinline__ void int4_group(float (&acc)[4], const uint4& ra, con
     acc[q] = fmaf(static_cast<float>((dh[0][q] + dh[1][q]) * 256 + dl[0][q] + dl[1][q]), f[q], acc[q]);
 }
 
-// One 128-wide K group of a 16-row NVFP4 tile into two fp32 accumulator sets (steps alternate).
-// Codes x E4M3 block scale are exact in fp16; thread t's 32 codes span the blocks 8j+2t, 8j+2t+1 of
-// the scale rows bs0 (row g) and bs1 (row g+8), whose block 0 is the group-0 block of j.
-__device__ __forceinline__ void nvfp4_group(float (&acc)[2][4], const uint4& ra, const uint4& rb, const RawB& B,
-                                            const uint8_t* bs0, const uint8_t* bs1, int j, int t) {
-  const int blk = j * 8 + 2 * t;
-  uint32_t s0[2], s1[2];
+// One 128-wide K group j of a 16-row NVFP4 tile into two fp32 accumulator sets (steps alternate).
+// Codes x E4M3 block scale are exact in fp16; thread t's 32 codes span the blocks 8j+2t and 8j+2t+1,
+// whose scales it holds in registers (s0: row g, s1: row g+8; low byte = block 8j+2t).
+__device__ __forceinline__ void nvfp4_group_r(float (&acc)[2][4], const uint4& ra, const uint4& rb, const RawB& B,
+                                              uint32_t s0, uint32_t s1) {
+  uint32_t h0[2], h1[2];
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
-    const uint32_t h0 = e4m3_to_half_bits(bs0[blk + q]);
-    const uint32_t h1 = e4m3_to_half_bits(bs1[blk + q]);
-    s0[q] = h0 | (h0 << 16);
-    s1[q] = h1 | (h1 << 16);
+    const uint32_t a = e4m3_to_half_bits(s0 >> (8 * q)), b = e4m3_to_half_bits(s1 >> (8 * q));
+    h0[q] = a | (a << 16);
+    h1[q] = b | (b << 16);
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t w0 = u4_word(ra, i >> 1), w1 = u4_word(rb, i >> 1);
     const int sh = (i & 1) * 16;
-    const uint32_t a[4] = {hmul2_u32(e2m1x2_to_half2(w0 >> sh), s0[i >> 2]),
-                           hmul2_u32(e2m1x2_to_half2(w1 >> sh), s1[i >> 2]),
-                           hmul2_u32(e2m1x2_to_half2(w0 >> (sh + 8)), s0[i >> 2]),
-                           hmul2_u32(e2m1x2_to_half2(w1 >> (sh + 8)), s1[i >> 2])};
+    const uint32_t a[4] = {hmul2_u32(e2m1x2_to_half2(w0 >> sh), h0[i >> 2]),
+                           hmul2_u32(e2m1x2_to_half2(w1 >> sh), h1[i >> 2]),
+                           hmul2_u32(e2m1x2_to_half2(w0 >> (sh + 8)), h0[i >> 2]),
+                           hmul2_u32(e2m1x2_to_half2(w1 >> (sh + 8)), h1[i >> 2])};
     mma_f16_16816(acc[i & 1], a, B.b0(i), B.b1(i));
   }
 }
@@ -271,45 +282,49 @@ __device__ __forceinline__ void load_a_bf16_rows(RawA<kBf16>& A, const uint8_t* 
 
 // ============================================================================================ route
 
-// 8 bf16 x 8 bf16 dot product; the products are exact in fp32.
-__device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b, float acc) {
-  const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+// Router logits on the tensor cores: rows e0 = c and e1 = c + G of W_r for every token. Routing warp
+// rw takes K quarter rw (512 elements = 4 groups); MMA rows 0 and 1 are the two router rows (the
+// other 14 rows are zero), columns the tokens (x staged in shared memory). The bf16 products are
+// exact and accumulate in fp32 (the router rows are used widened to FP32 on the pages: NInfer
+// README, "What is inside"); the four quarters are added in order by routing warp 0.
+struct RouterRows {
+  uint4 a[4][4];                            // lanes with g < 2: 32 bf16 of row g per group, 4 groups
+  __device__ __forceinline__ void load(const DecodeParams& p, int rw, int row) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const bool v = g < 2 && row < p.E;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    acc = fmaf(bf16lo_to_f32(aw[q]), bf16lo_to_f32(bw[q]), acc);
-    acc = fmaf(bf16hi_to_f32(aw[q]), bf16hi_to_f32(bw[q]), acc);
+    for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        a[jj][q] = v ? ld_stream_v4(p.wr + static_cast<size_t>(row) * kH + (4 * rw + jj) * kGroup + 32 * t + 8 * q)
+                     : make_uint4(0, 0, 0, 0);
   }
-  return acc;
-}
-
-__device__ __forceinline__ void load_router_row(uint4 (&w)[8], const DecodeParams& p, int e) {
-  const int lane = threadIdx.x & 31;
+  // partial logits of this warp's quarter into rpart[rw][row 0/1][token]
+  __device__ __forceinline__ void mma(const DecodeParams& p, int rw, const uint8_t* xs, int pitch,
+                                      float (&rpart)[4][2][kDecodeMaxT]) const {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    const bool bv = g < p.T;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) w[i] = ld_stream_v4(p.wr + static_cast<size_t>(e) * kH + 8 * lane + 256 * i);
-}
-
-// logits[t][e] for every token (one warp, router row in w; lane l covers elements 8l + 256i; x in
-// shared memory, token rows `pitch` bytes apart). The lane order and the shuffle reduction are those
-// of the routing-only entry point's router kernel, so both produce the same fp32 logits.
-__device__ void route_row(const DecodeParams& p, int e, const uint4 (&w)[8], const uint8_t* xs, int pitch) {
-  const int lane = threadIdx.x & 31;
-  float acc[kDecodeMaxT];
+    for (int jj = 0; jj < 4; ++jj) {
+      RawA<kBf16> A;
 #pragma unroll
-  for (int t = 0; t < kDecodeMaxT; ++t) {
-    acc[t] = 0.f;
-    if (t < p.T) {
+      for (int q = 0; q < 4; ++q) {
+        A.r0[q] = a[jj][q];
+        A.r1[q] = make_uint4(0, 0, 0, 0);
+      }
+      RawB B;
+      const uint8_t* q0 = xs + (bv ? g : 0) * pitch + ((4 * rw + jj) * kGroup + 32 * t) * 2;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        acc[t] = dot8_bf16(w[i], *reinterpret_cast<const uint4*>(xs + t * pitch + (8 * lane + 256 * i) * 2), acc[t]);
+      for (int q = 0; q < 4; ++q) B.u[q] = bv ? *reinterpret_cast<const uint4*>(q0 + 16 * q) : make_uint4(0, 0, 0, 0);
+      bf16_group(acc, A, B, nullptr);
+    }
+    if (g < 2) {
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) rpart[rw][g][2 * t + qq] = acc[0][qq] + acc[1][qq];
     }
   }
-#pragma unroll
-  for (int t = 0; t < kDecodeMaxT; ++t) {
-#pragma unroll
-    for (int m = 16; m > 0; m >>= 1) acc[t] += __shfl_xor_sync(kFull, acc[t], m);
-    if (lane == 0 && t < p.T) __stcg(p.logits + t * p.E + e, acc[t]);
-  }
-}
+};
 
 // One 128-segment of the gate|up activation operand (x in shared memory), written to global memory:
 // fp16(Hn x) with every 8-block in the order 0,4,1,5,2,6,3,7 and the 16-bit limbs of Hn x with
@@ -347,19 +362,32 @@ struct RouteSmem {
   unsigned mask[kMaxE];                     // table scratch: token bit masks
   int4 etab[kMaxActive][2];                 // active experts: {e, offset, count, tokens}, {ts_g, ts_u, ts_d, 0}
   int na;                                   // number of active experts
+  int wsum[8];                              // table scan: per-warp sums
+  float rpart[4][2][kDecodeMaxT];           // router: partial logits of the CTA's two rows per K quarter
 };
+
+// Logits of one token (one warp): element j of lane l is expert l + 32j (through L2: other CTAs wrote
+// them); the keys are formed by make_keys once the loads are back, so that the loads of several
+// tokens are in flight together.
+__device__ __forceinline__ void load_logits(const DecodeParams& p, int tok, float (&v)[8]) {
+  const int lane = threadIdx.x & 31, per = p.E >> 5;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = (j < per) ? __ldcg(p.logits + tok * p.E + lane + 32 * j) : 0.f;
+}
+__device__ __forceinline__ void make_keys(const DecodeParams& p, const float (&v)[8], unsigned (&key)[8]) {
+  const int per = p.E >> 5;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) key[j] = (j < per) ? logit_key(v[j]) : 0u;
+}
 
 // Top-k of one token (one warp): K rounds of a warp argmax on the fp32 logits. The router is
 // unbiased and sigmoid increasing, so the largest logits are the largest scores; ties go to the
 // lower id. The slots are listed by ascending expert id and w_k = s_k / max(sum of the chosen s,
 // floor), the sum taken in slot order (midagedev/bloomery issue #632, host-policy comment).
-__device__ __forceinline__ void topk_token(const DecodeParams& p, int tok, RouteSmem& rs, bool publish) {
+__device__ __forceinline__ void topk_select(const DecodeParams& p, int tok, const unsigned (&key)[8], RouteSmem& rs,
+                                            bool publish) {
   const int lane = threadIdx.x & 31;
   const int E = p.E, K = p.K, per = E >> 5;
-  // element j of lane l is expert l + 32j; a taken or absent element has key 0 and index E+
-  unsigned key[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) key[j] = (j < per) ? logit_key(__ldcg(p.logits + tok * E + lane + 32 * j)) : 0u;
   unsigned taken = 0u;                             // bit j: element j already chosen
   int my_id = 0;
   float my_l = 0.f;
@@ -401,97 +429,88 @@ __device__ __forceinline__ void topk_token(const DecodeParams& p, int tok, Route
   }
 }
 
-// Routing tables from the selected ids (one warp): the experts with tokens (ascending) and their
-// table, and the expert-major permutation (pairs of one expert by ascending token): position p
-// holds t*K+k, inv[t*K+k] = p. Ranks come from bit masks and scans, so the result does not depend
-// on the order atomics run in. With `publish` the tables also go to global memory (counts,
-// offsets (E+1), perm, inv, active experts, their table) for inspection.
-__device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& rs, bool publish) {
-  int* scr_cnt = rs.cnt;
-  unsigned* scr_mask = rs.mask;
-  const int* s_ids = rs.ids;
-  const int lane = threadIdx.x & 31;
+// Routing tables from the selected ids, by all 256 threads of the CTA (tid; every thread calls it):
+// the P = T*K pairs count their experts and set their token bits with shared-memory atomics (sums
+// and ORs, so the result does not depend on the order they run in); thread e then holds expert e,
+// and one scan over the experts (two 16-bit sums packed in a word: counts and active flags, neither
+// above 64) gives every expert its offset and active slot; the active experts' table entries
+// {e, offset, count, tokens (4 bits each)}, {ts_g, ts_u, ts_d, 0}; then the expert-major permutation
+// (pairs of one expert by ascending token): position p holds t*K+k, inv[t*K+k] = p. With `publish`
+// the tables also go to global memory (counts, offsets (E+1), perm, inv, active experts, their
+// table) for inspection.
+__device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& rs, bool publish, int tid) {
+  const int lane = tid & 31, w = tid >> 5;
   const int T = p.T, E = p.E, K = p.K, P = T * K;
-  const float* gu_ts = p.gu_ts;
-  const float* dn_ts = p.dn_ts;
-  for (int e = lane; e < kMaxE; e += 32) {
-    scr_cnt[e] = 0;
-    scr_mask[e] = 0u;
+  rs.cnt[tid] = 0;
+  rs.mask[tid] = 0u;
+  __syncthreads();
+  if (tid < P) {
+    const int id = rs.ids[tid];
+    atomicAdd(&rs.cnt[id], 1);
+    atomicOr(&rs.mask[id], 1u << (tid / K));
   }
-  __syncwarp();
-  const int id0 = lane < P ? s_ids[lane] : 0, id1 = lane + 32 < P ? s_ids[lane + 32] : 0;
-  if (lane < P) { atomicAdd(&scr_cnt[id0], 1); atomicOr(&scr_mask[id0], 1u << (lane / K)); }
-  if (lane + 32 < P) { atomicAdd(&scr_cnt[id1], 1); atomicOr(&scr_mask[id1], 1u << ((lane + 32) / K)); }
-  __syncwarp();
-  // lane holds experts 8*lane .. 8*lane+7
-  int s = 0, a = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int e = 8 * lane + j;
-    const int c = e < E ? scr_cnt[e] : 0;
-    s += c;
-    a += c > 0;
-  }
-  int si = s, ai = a;
+  __syncthreads();
+  const int e = tid;
+  const int cnt = e < E ? rs.cnt[e] : 0;
+  const unsigned msk = rs.mask[e];
+  const unsigned own = static_cast<unsigned>(cnt) | (static_cast<unsigned>(cnt > 0) << 16);
+  unsigned inc = own;
 #pragma unroll
   for (int m = 1; m < 32; m <<= 1) {
-    const int os = __shfl_up_sync(kFull, si, m), oa = __shfl_up_sync(kFull, ai, m);
-    if (lane >= m) { si += os; ai += oa; }
+    const unsigned o = __shfl_up_sync(kFull, inc, m);
+    if (lane >= m) inc += o;
   }
-  int off = si - s, slot = ai - a;
-  __syncwarp();
-#pragma unroll 1
-  for (int j = 0; j < 8; ++j) {
-    const int e = 8 * lane + j;
-    if (e >= E) break;
-    const int c = scr_cnt[e];
-    if (publish) {
-      p.counts[e] = c;
-      p.offsets[e] = off;
-    }
-    scr_cnt[e] = off;
-    if (c > 0) {
-      const unsigned m = scr_mask[e];
-      unsigned toks = 0;
-      int n = 0;
-#pragma unroll 1
-      for (int tt = 0; tt < T; ++tt)
-        if ((m >> tt) & 1u) toks |= static_cast<unsigned>(tt) << (4 * n++);
-      const float tsg = gu_ts ? __ldg(gu_ts + 2 * e) : 1.f;
-      const float tsu = gu_ts ? __ldg(gu_ts + 2 * e + 1) : 1.f;
-      const float tsd = dn_ts ? __ldg(dn_ts + e) : 1.f;
-      const int4 t0 = make_int4(e, off, c, static_cast<int>(toks));
-      const int4 t1 = make_int4(__float_as_int(tsg), __float_as_int(tsu), __float_as_int(tsd), 0);
-      rs.etab[slot][0] = t0;
-      rs.etab[slot][1] = t1;
-      if (publish) {
-        p.active[slot] = e;
-        p.etab[2 * slot] = t0;
-        p.etab[2 * slot + 1] = t1;
-      }
-      ++slot;
-    }
-    off += c;
-  }
-  if (lane == 31) {
-    rs.na = ai;
-    if (publish) {
-      p.offsets[E] = si;
-      *p.n_active = ai;
-    }
-  }
-  __syncwarp();
+  if (lane == 31) rs.wsum[w] = static_cast<int>(inc);
+  __syncthreads();
+  unsigned before = 0u, total = 0u;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int q = lane + 32 * h;
-    if (q < P) {
-      const int id = h ? id1 : id0, tt = q / K;
-      const int pos = scr_cnt[id] + __popc(scr_mask[id] & ((1u << tt) - 1u));
-      rs.inv[q] = pos;
-      if (publish) {
-        p.perm[pos] = q;
-        p.inv[q] = pos;
-      }
+  for (int v = 0; v < kWarps; ++v) {
+    const unsigned x = static_cast<unsigned>(rs.wsum[v]);
+    if (v < w) before += x;
+    total += x;
+  }
+  const unsigned ex = before + inc - own;          // exclusive prefix (packed)
+  const int off = static_cast<int>(ex & 0xFFFF), slot = static_cast<int>(ex >> 16);
+  rs.cnt[e] = off;                                 // every count was read before the barrier above
+  if (e < E && publish) {
+    p.counts[e] = cnt;
+    p.offsets[e] = off;
+  }
+  if (e < E && cnt > 0) {
+    unsigned toks = 0u, m = msk;
+    for (int n = 0; m; ++n) {
+      const int tt = __ffs(m) - 1;
+      toks |= static_cast<unsigned>(tt) << (4 * n);
+      m &= m - 1;
+    }
+    const float tsg = p.gu_ts ? __ldg(p.gu_ts + 2 * e) : 1.f;
+    const float tsu = p.gu_ts ? __ldg(p.gu_ts + 2 * e + 1) : 1.f;
+    const float tsd = p.dn_ts ? __ldg(p.dn_ts + e) : 1.f;
+    const int4 t0 = make_int4(e, off, cnt, static_cast<int>(toks));
+    const int4 t1 = make_int4(__float_as_int(tsg), __float_as_int(tsu), __float_as_int(tsd), 0);
+    rs.etab[slot][0] = t0;
+    rs.etab[slot][1] = t1;
+    if (publish) {
+      p.active[slot] = e;
+      p.etab[2 * slot] = t0;
+      p.etab[2 * slot + 1] = t1;
+    }
+  }
+  if (tid == 0) {
+    rs.na = static_cast<int>(total >> 16);
+    if (publish) {
+      p.offsets[E] = static_cast<int>(total & 0xFFFF);
+      *p.n_active = rs.na;
+    }
+  }
+  __syncthreads();
+  if (tid < P) {
+    const int id = rs.ids[tid], tt = tid / K;
+    const int pos = rs.cnt[id] + __popc(rs.mask[id] & ((1u << tt) - 1u));
+    rs.inv[tid] = pos;
+    if (publish) {
+      p.perm[pos] = tid;
+      p.inv[tid] = pos;
     }
   }
 }
@@ -573,8 +592,8 @@ struct DecShared {
   } u;
   RouteSmem rs;
   uint64_t full[kWarps][Geom<FMT>::kDepth];
-  uint64_t xbar, xqbar, hqbar, route_ready;
-  int gen0;
+  uint64_t xbar, xqbar, hqbar, logits_ready;
+  unsigned long long bar_base;                        // the grid barriers' counter at the forward's start
 };
 
 // A warp's ring position: stages are issued and consumed in one sequence across the three phases.
@@ -739,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
   DecShared<FMT>& sm = *reinterpret_cast<DecShared<FMT>*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int G = gridDim.x, c = blockIdx.x;
-  const GridBarrier gb{p.cnt + kCntBar, p.cnt + kCntBar + 1, p.cnt + kCntBar + 2};
+  const GridBarrier gb{reinterpret_cast<unsigned long long*>(p.cnt + kCntBar), p.cnt + kCntBar + 2};
   Ring<FMT> ring;
   ring.base = &sm.stage[warp][0][0];
   ring.full = &sm.full[warp][0];
@@ -751,12 +770,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
     mbar_init(&sm.xbar, 1);
     mbar_init(&sm.xqbar, 1);
     mbar_init(&sm.hqbar, 1);
-    mbar_init(&sm.route_ready, 1);
-    sm.gen0 = ld_acquire_gpu(gb.gen);
+    mbar_init(&sm.logits_ready, 1);
+    const unsigned long long c0 = ld_acquire_u64(gb.count);
+    sm.bar_base = c0 - c0 % (2ull * G);
   }
   fence_mbar_init();
   __syncthreads();
-  const int gen0 = sm.gen0;
+  const unsigned long long bar_base = sm.bar_base;
 
   // ---------------------------------------------------------------- phase A
   // gate|up tile k of this warp (round robin over the CTAs first, then the warps)
@@ -764,82 +784,80 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
   if (threadIdx.x == 0) {                          // x (T token rows), one bulk copy per row
     mbar_arrive_expect_tx(&sm.xbar, p.T * kH * 2);
     for (int r = 0; r < p.T; ++r) bulk_g2s(sm.u.ab.xs[r], p.x + static_cast<size_t>(r) * kH, kH * 2, &sm.xbar);
-  } else if (threadIdx.x == 32) {                  // the shared expert's down rows into L2 for phase C
-    for (int ch = c; ch < kH * kIs * 2 / 32768; ch += G) prefetch_l2(p.sh_dn + static_cast<size_t>(ch) * 32768, 32768);
   }
-  // shared-expert stages need no routing: the ring fills at once
-  int na = -1;                                     // active experts, once the routing is known
-  WarpTable tab;
   int k_issue = 0;                                 // next gate|up stage to issue: tile k_issue >> 2, quarter & 3
-  while (ring.has_room() && tile_of(k_issue >> 2) < kShGuTiles) {
-    gu_issue<FMT>(p, sm, ring, warp, k_issue & 3, k_issue >> 2, tile_of(k_issue >> 2), ExpertInfo{});
-    ++k_issue;
-  }
   if (warp >= kRouteWarp0) {
-    // router rows e = c + G*r (warps 4, 5) and the operand segments (warp 6)
-    const int rw = warp - kRouteWarp0;
-    uint4 w[8];
-    const int e = c + G * rw;
-    if (rw < 2 && e < p.E) load_router_row(w, p, e);
+    // router rows c and c + G on the tensor cores (K quarter rw each), then the operand segments
+    const int rw = warp - kRouteWarp0, ri = threadIdx.x - kRouteWarp0 * 32;
+    RouterRows rr;
+    rr.load(p, rw, c + G * g);
     wait_stage(p, &sm.xbar, 0);
-    if (rw < 2) {
-      for (int ee = e; ee < p.E; ee += 2 * G) {
-        if (ee != e) load_router_row(w, p, ee);
-        route_row(p, ee, w, sm.u.ab.xs[0], kTokPitch);
-      }
-    } else if (rw == 2) {
+    rr.mma(p, rw, sm.u.ab.xs[0], kTokPitch, sm.rs.rpart);
+    if (rw == kWarps - kRouteWarp0 - 1)
       for (int sg = c; sg < p.T * (kH / kGroup); sg += G)
         xq_segment(p, sg / (kH / kGroup), sg % (kH / kGroup), sm.u.ab.xs[0], kTokPitch);
+    named_bar_sync(kBarRoute, kRouteThreads);
+    if (rw == 0) {                                 // quarters added in order: one logit per lane
+      const int r = lane >> 3, tok = lane & 7, e = c + G * r;
+      if (tok < p.T && e < p.E) {
+        const float* q = &sm.rs.rpart[0][r][tok];
+        const float v = ((q[0] + q[2 * kDecodeMaxT]) + q[4 * kDecodeMaxT]) + q[6 * kDecodeMaxT];
+        __stcg(p.logits + tok * p.E + e, v);
+      }
     }
     // ------------------------------------------------------------ barrier 1: logits and operand
-    __threadfence();
     named_bar_sync(kBarRoute, kRouteThreads);
-    if (threadIdx.x == kRouteWarp0 * 32) {
-      gb.arrive(G, gen0 + 1);
-      gb.wait(gen0 + 1, p.err);
+    if (ri == 0) {
+      gb.arrive();
+      gb.wait(bar_base + G, p.err);
       fence_proxy_async_global();                  // the operand copy below reads other CTAs' writes
       constexpr int kRow = 2 * kH;                 // int4: hi + lo limbs; NVFP4: fp16
       const uint8_t* src = FMT == kInt4 ? p.xq8 : reinterpret_cast<const uint8_t*>(p.xq);
       mbar_arrive_expect_tx(&sm.xqbar, p.T * kRow + (FMT == kInt4 ? p.T * (kH / kGroup) * 4 : 0));
       for (int r = 0; r < p.T; ++r) bulk_g2s(sm.u.ab.xq[r], src + static_cast<size_t>(r) * kRow, kRow, &sm.xqbar);
       if (FMT == kInt4) bulk_g2s(&sm.u.ab.xsc[0][0], p.xsc, p.T * (kH / kGroup) * 4, &sm.xqbar);
+      mbar_arrive(&sm.logits_ready);
     }
-    named_bar_sync(kBarRoute, kRouteThreads);
-    // ------------------------------------------------------------ phase B: routing
-    for (int tok = rw; tok < p.T; tok += kWarps - kRouteWarp0) topk_token(p, tok, sm.rs, c == 0);
-    named_bar_sync(kBarRoute, kRouteThreads);
-    if (rw == 0) build_tables(p, sm.rs, c == 0);
-    named_bar_sync(kBarRoute, kRouteThreads);
-    if (threadIdx.x == kRouteWarp0 * 32) mbar_arrive(&sm.route_ready);
-    na = active_count(p, sm.rs);
-    tab.load(sm.rs);
+  } else {
+    // the shared expert needs no routing, but x and the router rows go first: its gate|up stages
+    // (the ring holds the warp's whole shared tile) and the L2 fetch of its down rows start once x
+    // has landed
+    wait_stage(p, &sm.xbar, 0);
+    while (ring.has_room() && tile_of(k_issue >> 2) < kShGuTiles) {
+      gu_issue<FMT>(p, sm, ring, warp, k_issue & 3, k_issue >> 2, tile_of(k_issue >> 2), ExpertInfo{});
+      ++k_issue;
+    }
+    if (threadIdx.x == 32)
+      for (int ch = c; ch < kH * kIs * 2 / 32768; ch += G) prefetch_l2(p.sh_dn + static_cast<size_t>(ch) * 32768, 32768);
   }
-  // ---------------------------------------------------------------- phase B: gate|up tiles
-  if (warp < kRouteWarp0) wait_stage(p, &sm.xbar, 0);   // the shared tiles read the staged x
-  auto routing_known = [&](bool block) {
-    if (na >= 0) return true;
-    if (!block && !mbar_test_wait(&sm.route_ready, 0)) return false;
-    wait_stage(p, &sm.route_ready, 0);
-    na = active_count(p, sm.rs);
-    tab.load(sm.rs);
-    return true;
-  };
+  // ---------------------------------------------------------------- phase B: routing (every warp)
+  wait_stage(p, &sm.logits_ready, 0);              // barrier 1 is passed: every CTA's logits and operand are in
+  if (warp < p.T) {                                // token `warp`
+    float lv[8];
+    unsigned kv[8];
+    load_logits(p, warp, lv);
+    make_keys(p, lv, kv);
+    topk_select(p, warp, kv, sm.rs, c == 0);
+  }
+  __syncthreads();
+  build_tables(p, sm.rs, c == 0, threadIdx.x);
+  __syncthreads();
+  const int na = active_count(p, sm.rs);
+  WarpTable tab;
+  tab.load(sm.rs);
   auto info = [&](int tl) {
     ExpertInfo ex{};
     if (tl >= kShGuTiles) ex = tab.get(p, (tl - kShGuTiles) / kGuTilesPerExpert);
     return ex;
   };
-  // tile k exists (blocks for the routing when the tile is a routed one)
-  auto gu_valid = [&](int k) {
-    const int tl = tile_of(k);
-    if (tl < kShGuTiles) return true;
-    routing_known(true);
-    return tl < kShGuTiles + kGuTilesPerExpert * na;
-  };
+  const int n_gu = kShGuTiles + kGuTilesPerExpert * na;   // gate|up tiles of the forward
+  int r0, nr;
+  cta_rows(r0, nr);
+  const int n_items = kShDnSlices + na;            // phase C items of this CTA
+  // ---------------------------------------------------------------- phase B: gate|up tiles
   bool have_xq = false;
-  PendingArrival seg_arr;
-  auto finish_last = [&](int key) {
-    if (key < 0) return;
+  PendingArrivals seg_arr;
+  auto finish_last = [&](int key) {            // this warp completed the segment: rotate it
     const int gi = (key - kCntSeg) / 4, seg = (key - kCntSeg) % 4;
     finish_segment(p, tab.get(p, gi), seg);
     if (lane == 0) p.cnt[key] = 0;
@@ -849,19 +867,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
   bool bvalid = false;
   int tok0 = 0, tok1 = 0;                          // tokens of MMA columns 2t, 2t+1
   const uint8_t* brow = nullptr;                   // this lane's activation row (column g)
-  for (int s = 0;; ++s) {
-    const int k = s >> 2, q = s & 3, tl = tile_of(k);
-    if (q == 0 && !gu_valid(k)) break;
-    // keep the ring full; a shared-tile warp does not block on the routing to issue a routed stage
-    while (ring.has_room()) {
+  auto refill = [&]() {                            // keep the ring full
+    while (ring.has_room() && tile_of(k_issue >> 2) < n_gu) {
       const int tk = tile_of(k_issue >> 2);
-      if (tk >= kShGuTiles) {
-        if (!routing_known(false)) break;
-        if (tk >= kShGuTiles + kGuTilesPerExpert * na) break;
-      }
       gu_issue<FMT>(p, sm, ring, warp, k_issue & 3, k_issue >> 2, tk, info(tk));
       ++k_issue;
     }
+  };
+  for (int s = 0;; ++s) {
+    const int k = s >> 2, q = s & 3, tl = tile_of(k);
+    if (q == 0 && tl >= n_gu) break;
+    refill();
     if (q == 0) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[0][i] = acc[1][i] = 0.f;
@@ -892,36 +908,49 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
         load_b_smem(B, xr, 4 * q + jj, t, xv);
         bf16_group(acc, A, B, nullptr);
       }
-    } else if constexpr (FMT == kInt4) {
-      const uint16_t* sc = reinterpret_cast<const uint16_t*>(sm.gu_sc[warp][k & 1]);
-      const bool v0 = 2 * t < ex.n, v1 = 2 * t + 1 < ex.n;
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int j = 4 * q + jj;
-        const uint4 ra = *reinterpret_cast<const uint4*>(st + g * 256 + jj * 64 + 16 * t);
-        const uint4 rb = *reinterpret_cast<const uint4*>(st + (g + 8) * 256 + jj * 64 + 16 * t);
-        uint4 bh[2], bl[2];
-        load_limbs_smem(bh, bl, brow, kH, j, t, bvalid);
-        const float sg = bf16_bits_to_f32(sc[g * 16 + j]), su = bf16_bits_to_f32(sc[(8 + g) * 16 + j]);
-        const float x0 = v0 ? sm.u.ab.xsc[tok0][j] : 0.f, x1 = v1 ? sm.u.ab.xsc[tok1][j] : 0.f;
-        const float f[4] = {sg * x0, sg * x1, su * x0, su * x1};
-        int4_group(acc[0], ra, rb, bh, bl, f);
-      }
     } else {
-      // scales of the stage: gate rows 8 x 32 B at 4096, up rows at 4352 (blocks of this K quarter)
-      const uint8_t* sc = st + 4096;
+      // routed: the stage's codes (and NVFP4 block scales: gate rows 8 x 32 B at 4096, up rows at
+      // 4352, blocks of this K quarter) go to registers, and the slot is refilled before the MMAs
+      uint4 ra[4], rb[4];
+      uint32_t bs0[4], bs1[4];
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
-        const int j = 4 * q + jj;
-        const uint4 ra = *reinterpret_cast<const uint4*>(st + g * 256 + jj * 64 + 16 * t);
-        const uint4 rb = *reinterpret_cast<const uint4*>(st + (g + 8) * 256 + jj * 64 + 16 * t);
-        RawB B;
-        load_b_smem(B, brow, j, t, bvalid);
-        nvfp4_group(acc, ra, rb, B, sc + g * 32, sc + 256 + g * 32, jj, t);
+        ra[jj] = *reinterpret_cast<const uint4*>(st + g * 256 + jj * 64 + 16 * t);
+        rb[jj] = *reinterpret_cast<const uint4*>(st + (g + 8) * 256 + jj * 64 + 16 * t);
+        if constexpr (FMT != kInt4) {
+          bs0[jj] = *reinterpret_cast<const uint16_t*>(st + 4096 + g * 32 + jj * 8 + 2 * t);
+          bs1[jj] = *reinterpret_cast<const uint16_t*>(st + 4096 + 256 + g * 32 + jj * 8 + 2 * t);
+        }
+      }
+      __syncwarp();                                // every lane's reads of the slot precede its refill
+      ring.consumed++;
+      refill();
+      if constexpr (FMT == kInt4) {
+        const uint16_t* sc = reinterpret_cast<const uint16_t*>(sm.gu_sc[warp][k & 1]);
+        const bool v0 = 2 * t < ex.n, v1 = 2 * t + 1 < ex.n;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int j = 4 * q + jj;
+          uint4 bh[2], bl[2];
+          load_limbs_smem(bh, bl, brow, kH, j, t, bvalid);
+          const float sg = bf16_bits_to_f32(sc[g * 16 + j]), su = bf16_bits_to_f32(sc[(8 + g) * 16 + j]);
+          const float x0 = v0 ? sm.u.ab.xsc[tok0][j] : 0.f, x1 = v1 ? sm.u.ab.xsc[tok1][j] : 0.f;
+          const float f[4] = {sg * x0, sg * x1, su * x0, su * x1};
+          int4_group(acc[0], ra[jj], rb[jj], bh, bl, f);
+        }
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          RawB B;
+          load_b_smem(B, brow, 4 * q + jj, t, bvalid);
+          nvfp4_group_r(acc, ra[jj], rb[jj], B, bs0[jj], bs1[jj]);
+        }
       }
     }
-    __syncwarp();                                  // every lane's reads of the slot precede its refill
-    ring.consumed++;
+    if (tl < kShGuTiles) {
+      __syncwarp();                                // every lane's reads of the slot precede its refill
+      ring.consumed++;
+    }
     if (q != 3) continue;
     // ---- tile epilogue
     float cc[4];
@@ -952,18 +981,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
           p.h32[static_cast<size_t>(ex.off + col) * kI + 8 * i8 + g] = silu(cc[qq] * ex.tsg) * (cc[2 + qq] * ex.tsu);
       }
       const int seg = i8 / (kGroup / 8);
-      finish_last(seg_arr.settle());
-      seg_arr.arrive(p.cnt, kCntSeg + 4 * gi + seg, kGroup / 8);
+      if (seg_arr.full()) seg_arr.settle(kGroup / 8, finish_last);
+      seg_arr.arrive(p.cnt, kCntSeg + 4 * gi + seg);
     }
   }
-  routing_known(true);
-  finish_last(seg_arr.settle());
+  seg_arr.settle(kGroup / 8, finish_last);
   if (warp == kRouteWarp0 && !have_xq) wait_stage(p, &sm.xqbar, 0);   // no copy may still write the operand rows
 
   // ---------------------------------------------------------------- phase C: first stages, barrier 2
-  int r0, nr;
-  cta_rows(r0, nr);
-  const int n_items = kShDnSlices + na;
   int it_issue = warp;                             // this warp's items: warp, warp + 8, ...
   while (ring.has_room() && it_issue < n_items) {
     dn_issue<FMT>(p, ring, it_issue, r0, nr, tab);
@@ -971,8 +996,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
   }
   __syncthreads();                                 // every warp's h, hs and operand writes are done
   if (threadIdx.x == 0) {
-    gb.arrive(G, gen0 + 2);
-    gb.wait(gen0 + 2, p.err);
+    gb.arrive();
+    gb.wait(bar_base + 2ull * G, p.err);
     fence_proxy_async_global();
     const int P = p.T * p.K;
     const uint8_t* src = FMT == kInt4 ? p.hq8 : reinterpret_cast<const uint8_t*>(p.hq);
@@ -984,6 +1009,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
 
   // ---------------------------------------------------------------- phase C: down items
   bool have_hq = false;
+  auto release = [&]() {                           // the slot is read: refill it with the next item
+    __syncwarp();
+    ring.consumed++;
+    if (it_issue < n_items) {
+      dn_issue<FMT>(p, ring, it_issue, r0, nr, tab);
+      it_issue += kWarps;
+    }
+  };
   for (int it = warp; it < n_items; it += kWarps) {
     const int i = ring.consumed;
     wait_stage(p, ring.bar(i), (i / D) & 1);
@@ -999,15 +1032,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
       const int j = it;
       const bool bv = g < p.T;
       const size_t r = static_cast<size_t>(bv ? g : 0) * kIs;
+      RawB Bh, Bl;
+      Bh.load_cg(p.hs_hi + r, j, t, bv);
+      Bl.load_cg(p.hs_lo + r, j, t, bv);
       RawA<kBf16> A;
 #pragma unroll
       for (int qd = 0; qd < 4; ++qd) {
         A.r0[qd] = *reinterpret_cast<const uint4*>(st + g * 256 + (32 * t) * 2 + 16 * qd);
         A.r1[qd] = *reinterpret_cast<const uint4*>(st + (g + 8) * 256 + (32 * t) * 2 + 16 * qd);
       }
-      RawB Bh, Bl;
-      Bh.load_cg(p.hs_hi + r, j, t, bv);
-      Bl.load_cg(p.hs_lo + r, j, t, bv);
+      release();
       bf16_group(dacc, A, Bh, &Bl);
       float cs[4];
 #pragma unroll
@@ -1019,6 +1053,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
         if (tok < p.T) sm.u.c.spart[j][tok][row] = cs[b];
       }
     } else {
+      // rows g, g+8 of the stage (row r at r * 256); rows >= nr are the next expert's or beyond:
+      // they are read (inside the stage) but their results are dropped. Codes and scales go to
+      // registers and the slot is refilled before the MMAs.
+      const int ga = min(g, nr - 1), gb2 = min(g + 8, nr - 1);
+      uint4 ra[4], rb[4];
+      uint32_t sa[4], sb[4];                       // int4: f32 bits of the group scales; NVFP4: 2 E4M3 bytes
+#pragma unroll
+      for (int j = 0; j < kI / kGroup; ++j) {
+        ra[j] = *reinterpret_cast<const uint4*>(st + g * 256 + j * 64 + 16 * t);
+        rb[j] = *reinterpret_cast<const uint4*>(st + (g + 8) * 256 + j * 64 + 16 * t);
+        if constexpr (FMT == kInt4) {
+          // row r's 4 bf16 scales at 4096 + (r + (r0 & 1)) * 8 (the copy starts at an even row)
+          const uint16_t* s16 = reinterpret_cast<const uint16_t*>(st + 4096) + (r0 & 1) * 4;
+          sa[j] = static_cast<uint32_t>(s16[ga * 4 + j]) << 16;
+          sb[j] = static_cast<uint32_t>(s16[gb2 * 4 + j]) << 16;
+        } else {
+          sa[j] = *reinterpret_cast<const uint16_t*>(st + 4096 + ga * 32 + j * 8 + 2 * t);
+          sb[j] = *reinterpret_cast<const uint16_t*>(st + 4096 + gb2 * 32 + j * 8 + 2 * t);
+        }
+      }
+      release();
       if (!have_hq) {
         wait_stage(p, &sm.hqbar, 0);
         have_hq = true;
@@ -1026,38 +1081,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
       const ExpertInfo e2 = tab.get(p, it - kShDnSlices);
       const bool bv = g < e2.n;
       const uint8_t* hrow = sm.u.c.hq[e2.off + (bv ? g : 0)];
-      // rows g, g+8 of the stage (row r at r * 256); rows >= nr are the next expert's or beyond:
-      // they are read (inside the stage) but their results are dropped
-      const uint8_t* ra_p = st + g * 256;
-      const uint8_t* rb_p = st + (g + 8) * 256;
       if constexpr (FMT == kInt4) {
-        // scales: row r's 4 bf16 at 4096 + (r + (r0 & 1)) * 8 (the copy starts at an even row)
-        const uint16_t* s16 = reinterpret_cast<const uint16_t*>(st + 4096) + (r0 & 1) * 4;
         const bool v0 = 2 * t < e2.n, v1 = 2 * t + 1 < e2.n;
         const float* x0p = sm.u.c.hsc[e2.off + (v0 ? 2 * t : 0)];
         const float* x1p = sm.u.c.hsc[e2.off + (v1 ? 2 * t + 1 : 0)];
-        const int ga = min(g, nr - 1), gb2 = min(g + 8, nr - 1);
 #pragma unroll
         for (int j = 0; j < kI / kGroup; ++j) {
-          const uint4 ra = *reinterpret_cast<const uint4*>(ra_p + j * 64 + 16 * t);
-          const uint4 rb = *reinterpret_cast<const uint4*>(rb_p + j * 64 + 16 * t);
           uint4 bh[2], bl[2];
           load_limbs_smem(bh, bl, hrow, kI, j, t, bv);
-          const float s0 = bf16_bits_to_f32(s16[ga * 4 + j]), s1 = bf16_bits_to_f32(s16[gb2 * 4 + j]);
+          const float s0 = __uint_as_float(sa[j]), s1 = __uint_as_float(sb[j]);
           const float x0 = v0 ? x0p[j] : 0.f, x1 = v1 ? x1p[j] : 0.f;
           const float f[4] = {s0 * x0, s0 * x1, s1 * x0, s1 * x1};
-          int4_group(dacc[0], ra, rb, bh, bl, f);
+          int4_group(dacc[0], ra[j], rb[j], bh, bl, f);
         }
       } else {
-        const uint8_t* sc = st + 4096;
-        const int ga = min(g, nr - 1), gb2 = min(g + 8, nr - 1);
 #pragma unroll
         for (int j = 0; j < kI / kGroup; ++j) {
-          const uint4 ra = *reinterpret_cast<const uint4*>(ra_p + j * 64 + 16 * t);
-          const uint4 rb = *reinterpret_cast<const uint4*>(rb_p + j * 64 + 16 * t);
           RawB B;
           load_b_smem(B, hrow, j, t, bv);
-          nvfp4_group(dacc, ra, rb, B, sc + ga * 32, sc + gb2 * 32, j, t);
+          nvfp4_group_r(dacc, ra[j], rb[j], B, sa[j], sb[j]);
         }
       }
       float cs[4];
@@ -1068,12 +1110,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
         const int col = 2 * t + (b & 1), row = g + 8 * (b >> 1);
         if (col < e2.n) sm.u.c.opart[e2.off + col][row] = cs[b] * e2.tsd;
       }
-    }
-    __syncwarp();
-    ring.consumed++;
-    if (it_issue < n_items) {                      // refill the slot just consumed
-      dn_issue<FMT>(p, ring, it_issue, r0, nr, tab);
-      it_issue += kWarps;
     }
   }
   if (warp == 0 && !have_hq) wait_stage(p, &sm.hqbar, 0);   // no copy may still write this CTA's memory

@@ -10,6 +10,8 @@
 //
 // The array is part of the library image: every GPU on which the library is used holds it (64 KiB
 // plus a small tail) until the process exits. It bounds the sizes this entry point accepts.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "../../include/flint_moe.h"
@@ -28,21 +30,42 @@ static __device__ __align__(256) float g_route_scratch[kScratchFloats];
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 float* g_scratch_addr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
+
+// The driver's cuCtxGetCurrent, through the runtime (no link-time driver dependency).
+PFN_cuCtxGetCurrent_v4000 ctx_getter() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+  }
+  return fn;
+}
 
 // Device address of the scratch array for the current device. In host code the symbol itself is
-// only a host-side stand-in, so the address must come from cudaGetSymbolAddress, once per device,
-// with that device current.
+// only a host-side stand-in, so the address must come from cudaGetSymbolAddress, with that device
+// current. It is looked up once per device and context: the cached address is kept with the
+// context it belongs to, and a different current context (after cudaDeviceReset, say) looks it up
+// again.
 cudaError_t scratch_for_current_device(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  CUcontext ctx = nullptr;
+  PFN_cuCtxGetCurrent_v4000 get = ctx_getter();
+  if (!get || get(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_addr[dev]) {
+  if (!g_scratch_addr[dev] || !ctx || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    e = cudaGetSymbolAddress(&p, g_route_scratch);     // also makes the device's context current
     if (e != cudaSuccess) return e;
+    if (get(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
     g_scratch_addr[dev] = static_cast<float*>(p);
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_addr[dev];
   return cudaSuccess;

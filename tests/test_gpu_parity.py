@@ -208,3 +208,95 @@ def test_argument_errors_on_device():
         B.flint_moe_forward(dev.handle, xd.data_ptr() + 2, 4, y.data_ptr(), 0)
     B.flint_moe_forward(dev.handle, xd.data_ptr(), 0, y.data_ptr(), 0)      # T = 0 is a no-op
     torch.cuda.synchronize()
+
+
+def _logit_gap(L, x, top_k=6):
+    """fp64 gap between the top_k-th and next logit of every token (the selection is unique above the
+    fp32 error of the logits, ~1e-5 here)."""
+    lg = np.sort(R.bf16_to_f64(x) @ R.bf16_to_f64(L["router_w"]).T, axis=1)[:, ::-1]
+    return lg[:, top_k - 1] - lg[:, top_k]
+
+
+@pytest.mark.parametrize("T", [8, 40])
+def test_selected_sum_floor_is_applied(T):
+    # every logit near -20 (x[:, 0] = 1 carries a per-expert bias in router column 0), so the six
+    # selected sigmoid scores sum to ~1e-8, far below 2^-14: the weights are s / 2^-14, not s / sum
+    # (midagedev/bloomery issue #632, host-policy comment: SelectedSumFloor); T = 8 takes the decode
+    # kernel, T = 40 the tensor-core path
+    L = dict(layer(32, "int4"))
+    rw = L["router_w"].copy()
+    rw[:, 0] = S.f32_to_bf16_bits((-18.0 - 0.375 * np.arange(32)).astype(np.float32))
+    L["router_w"] = rw
+    x = S.make_x(T, skew=True)
+    ref = R.moe_forward(L, x)
+    s_sel = np.take_along_axis(ref["scores"], ref["ids"].astype(np.int64), axis=1)
+    assert np.all(s_sel.sum(axis=1) < 2.0 ** -14)
+    np.testing.assert_allclose(ref["w"], s_sel / 2.0 ** -14, rtol=1e-12)
+    keep = _logit_gap(L, x) >= 1e-3
+    assert keep.sum() >= T // 2
+    dev, xd, y = run(L, x)
+    r = dev.routing(T)
+    np.testing.assert_array_equal(r["ids"].cpu().numpy()[keep], ref["ids"][keep])
+    # w = s / 2^-14 with s = sigmoid(logit) ~ e^logit: its relative error is the absolute error of the
+    # fp32 logit (sums of 2048 exact products near -20, a few 2^-19)
+    np.testing.assert_allclose(r["w"].cpu().numpy()[keep], ref["w"][keep], rtol=1e-4)
+    assert float(r["w"].cpu().numpy().sum(axis=1).max()) < 0.1        # the floor, not a renormalisation to 1
+    st = PT.compare_y(y_to_host_bits(y), ref["y"])
+    assert st["finite"] and st["violations"] == 0, st
+    assert dev.error_word() == 0
+
+
+@pytest.mark.parametrize("fmt,T", [("int4", 8), ("nvfp4", 8), ("int4", 40), ("nvfp4", 40)])
+def test_routed_scale_half(fmt, T):
+    L = layer(32, fmt)
+    x = S.make_workload_x(T, 32)
+    ref = R.moe_forward(L, x, routed_scale=0.5)
+    dev = FlintMoELayer(L, t_max=T, routed_scale=0.5)
+    y = dev.forward(x_to_device(x))
+    torch.cuda.synchronize()
+    PT.check_routing(dev.routing(T), ref, T, 6)
+    st = PT.compare_y(y_to_host_bits(y), ref["y"])
+    assert st["finite"] and st["violations"] == 0, st
+    # and it is not the scale-1 layer
+    ref1 = R.moe_forward(L, x)
+    assert np.abs(ref1["y"] - ref["y"]).max() > 0.1
+    dev.close()
+
+
+@pytest.mark.parametrize("T", [8, 300])
+def test_debug_checks_stay_clear_on_a_valid_forward(T):
+    # FLINT_FLAG_DEBUG_CHECKS turns on the device-side range checks of ids and offsets; on a valid
+    # forward the error word stays 0 and the output is unchanged
+    L = layer(256, "int4")
+    x = S.make_workload_x(T, 256)
+    ref = R.moe_forward(L, x)
+    dev, xd, y = run(L, x, flags=B.FLINT_FLAG_DEBUG_CHECKS)
+    PT.check_routing(dev.routing(T), ref, T, 6)
+    st = PT.compare_y(y_to_host_bits(y), ref["y"])
+    assert st["finite"] and st["violations"] == 0, st
+    assert dev.error_word() == 0
+    dev2, _, y2 = run(L, x)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+def test_decode_top8_most_active_experts():
+    # top-8 at T = 8: 64 (token, slot) pairs, the most the decode kernel takes; ~57 distinct experts,
+    # so four routed gate|up tiles per warp and nine phase-C items per warp on 148 SMs
+    L = layer(256, "int4")
+    x = S.make_x(8, redraws=S.redraw_table(256))
+    ref = R.moe_forward(L, x, top_k=8)
+    keep = ref["gap"] >= 1e-4
+    dev, xd, y = run(L, x, top_k=8)
+    r = dev.routing(8)
+    np.testing.assert_array_equal(r["ids"].cpu().numpy()[keep], ref["ids"][keep])
+    st = PT.compare_y(y_to_host_bits(y)[keep], ref["y"][keep])
+    assert st["finite"] and st["violations"] == 0, st
+    assert dev.error_word() == 0
+
+
+def test_prefill_nvfp4_skewed_loads():
+    L = layer(256, "nvfp4", skew=True)
+    x = S.make_workload_x(2048, 256, skew=True)
+    dev, xd, y, ref, st = full_check(L, x)
+    counts = np.diff(ref["offsets"])
+    assert counts.max() > 300 and (counts == 0).any()

@@ -90,3 +90,32 @@ def test_stack_rejects_bad_arguments():
     with pytest.raises(B.FlintError):                                   # eps must be positive
         B.flint_residual_rmsnorm(x.data_ptr(), 0, 8, 0.0, st.z.data_ptr(), 0)
     st.close()
+
+
+def test_stack_of_four_full_layers_matches_the_oracle_chain():
+    # four E = 256 int4 layers through the native stack entry point, against the oracle's own chain
+    # x <- x + layer(bf16(rmsnorm(x))) in fp64 (each layer fed the oracle's residual, not the
+    # device's): the residual after the last layer agrees within the sum of the layers' output
+    # tolerances, and every layer picks the oracle's experts wherever its top-6 is not a near tie
+    E, T, n = 256, 8, 4
+    layers = [S.make_layer(E, "int4", seed=1000 + l) for l in range(n)]
+    x0 = R.bf16_to_f64(S.make_workload_x(T, E)).astype(np.float32)
+    st = FlintMoEStack(layers, t_max=T, eps=EPS)
+    xs = torch.from_numpy(x0.copy()).cuda()
+    st.forward(xs)
+    torch.cuda.synchronize()
+    x_ref = x0.astype(np.float64)
+    tol = np.zeros((T, H))
+    for l, L in enumerate(layers):
+        step = R.stack_step(L, x_ref, eps=EPS)
+        ref = R.moe_forward(L, step["z"])
+        keep = ref["gap"] >= 1e-4
+        assert keep.sum() >= T - 2
+        ids = st.layers[l].routing(T)["ids"].cpu().numpy()
+        np.testing.assert_array_equal(ids[keep], ref["ids"][keep])
+        tol += PT.y_tolerance(step["y"])[1]
+        x_ref = step["x_next"]
+    err = np.abs(xs.cpu().numpy().astype(np.float64) - x_ref)
+    assert np.all(err <= tol + 2.0 ** -20 * np.abs(x_ref)), float((err / tol).max())
+    assert all(layer.error_word() == 0 for layer in st.layers)
+    st.close()

@@ -1,13 +1,17 @@
 """flint_moe_route_noalloc: routing for callers that cannot allocate device memory (for example code
 running under CUDA graph capture, or a plug-in whose host owns the allocator). Its logits scratch is a
 fixed device array inside the library instead of a caller workspace; its results must equal the
-routing that flint_moe_forward produces through the existing entry points, call after call.
+oracle's routing and the routing that flint_moe_forward produces through the existing entry points,
+call after call (ids exactly, weights to fp32 rounding: the two entry points form the same fp32 logits
+from exact bf16 products but sum them in different orders).
 
 This file is collected last on purpose, so that a run stopping at its first failure has already run
 every other test."""
 
 import numpy as np
 import pytest
+
+from oracle import flint_moe_ref as R
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -36,6 +40,12 @@ def test_noalloc_routing_matches_the_forward_routing_on_consecutive_calls():
         B.flint_moe_route_noalloc(x.data_ptr(), layer.tensors["router_w"].data_ptr(), T, E, K, 2.0 ** -14,
                                   ids.data_ptr(), w.data_ptr(), stream)
         torch.cuda.synchronize()
+        # the oracle's routing on fp64 logits (the redraw table keeps every 6th/7th gap >= 1e-4)
+        xb = x.cpu().view(torch.int16).numpy().view(np.uint16)
+        ref = R.route(R.bf16_to_f64(xb) @ R.bf16_to_f64(L["router_w"]).T, K)
+        assert np.all(ref["gap"] >= 1e-4)
+        np.testing.assert_array_equal(ids.cpu().numpy(), ref["ids"])
+        np.testing.assert_allclose(w.cpu().numpy(), ref["w"], rtol=2e-6, atol=1e-7)
         np.testing.assert_array_equal(ids.cpu().numpy(), want["ids"].cpu().numpy())
         np.testing.assert_allclose(w.cpu().numpy(), want["w"].cpu().numpy(), rtol=2e-6, atol=1e-7)
     layer.close()
