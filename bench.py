@@ -262,6 +262,110 @@ def job_tokens_per_s(world: int, T: int, steps: int, max_total_ms: float) -> flo
 
 # --------------------------------------------------------------------------------------------- ours
 
+def measure_per_T(layer, fmt, E, Ts, redraws, timed_steps, steps, warmup, dev_name):
+    """Decode forwards at each T: device time per forward and the HBM figures of its algorithmic bytes."""
+    import torch
+
+    from bit_routed_expert_sigmoid_b200 import synthetic as S
+    from bit_routed_expert_sigmoid_b200.layer import x_to_device
+    out = {}
+    for tt_ in Ts:
+        xt = x_to_device(S.make_x(tt_, redraws=redraws), dev_name)
+        yt = torch.empty((tt_, H), dtype=torch.bfloat16, device=dev_name)
+        f = lambda: layer.forward(xt, yt)  # noqa: E731
+        for _ in range(warmup):
+            f()
+        na = int((torch.diff(layer.routing(tt_)["offsets"]) > 0).sum().item())
+        ms = statistics.mean(timed_steps(f, steps))
+        ab = algorithmic_bytes(E, fmt, tt_, na)
+        out[str(tt_)] = {"us": round(ms * 1e3, 2), "tokens_per_s": round(tt_ / (ms * 1e-3), 1),
+                         "distinct_experts": na, "algorithmic_MB": round(ab / 1e6, 3),
+                         "GB_per_s": round(ab / (ms * 1e-3) / 1e9, 1),
+                         "pct_of_8TBps": round(100 * ab / (ms * 1e-3) / 1e9 / HBM_NOMINAL_GBS, 2)}
+    return out
+
+
+def measure_prefill(layer, fmt, E, skew, redraws, timed_steps, steps, dev_name, peaks, workload):
+    """One T = 2048 forward: device time, grouped-GEMM TFLOP/s, and the roofline of its slowest kernel
+    (per-kernel CUDA-event times from the library's stage events, an instrumented pass that serialises
+    the kernels)."""
+    import torch
+
+    from bit_routed_expert_sigmoid_b200 import binding as B
+    from bit_routed_expert_sigmoid_b200 import synthetic as S
+    from bit_routed_expert_sigmoid_b200.layer import x_to_device
+    Tp = 2048
+    xp = x_to_device(S.make_x(Tp, redraws=redraws, skew=skew), dev_name)
+    yp = torch.empty((Tp, H), dtype=torch.bfloat16, device=dev_name)
+    f = lambda: layer.forward(xp, yp)  # noqa: E731
+    for _ in range(3):
+        f()
+    ms = statistics.mean(timed_steps(f, steps))
+    n_active = int((torch.diff(layer.routing(Tp)["offsets"]) > 0).sum().item())
+    fl = grouped_gemm_flops(Tp)
+    tf = fl / (ms * 1e-3) / 1e12
+    stream = torch.cuda.current_stream()
+    n_st = B.flint_moe_stage_count(layer.handle, Tp)
+    names = [B.flint_moe_stage_name(layer.handle, Tp, i) for i in range(n_st)]
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)]
+    for e in evs:
+        e.record(stream)
+    torch.cuda.synchronize()
+    B.flint_moe_set_stage_events(layer.handle, [e.cuda_event for e in evs])
+    acc = np.zeros(n_st)
+    n_prof = max(3, steps // 2)
+    for _ in range(n_prof):
+        f()
+        torch.cuda.synchronize()
+        acc += [evs[i].elapsed_time(evs[i + 1]) for i in range(n_st)]
+    B.flint_moe_set_stage_events(layer.handle, None)
+    stage_ms = acc / n_prof
+    top = int(np.argmax(stage_ms))
+    st_flops = stage_flops(names[top], E, Tp, 6)
+    st_bytes = stage_bytes(names[top], E, fmt, Tp, 6, n_active)
+    achieved = st_flops / (stage_ms[top] * 1e-3) / 1e12
+    return {"us": round(ms * 1e3, 1), "tokens_per_s": round(Tp / (ms * 1e-3), 1),
+            "grouped_gemm_TFLOPs": round(tf, 2),
+            "pct_of_2250TF_dense_bf16": round(100 * tf / BF16_DENSE_NOMINAL_TFLOPS, 2),
+            "pct_of_measured_bf16": round(100 * tf / peaks["bf16_tflops"], 2),
+            "distinct_experts": n_active,
+            "stage_us_serialised": {n: round(float(t) * 1e3, 2) for n, t in zip(names, stage_ms)},
+            "roofline": {"bound": "tensor", "kernel": names[top], "achieved": round(achieved, 2),
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(achieved / peaks["bf16_tflops"], 4),
+                         "traffic": ncu_traffic(names[top], workload), "algorithmic_flops": st_flops,
+                         "algorithmic_bytes": st_bytes,
+                         "hbm_GB_per_s": round(st_bytes / (stage_ms[top] * 1e-3) / 1e9, 1),
+                         "kernel_us": round(float(stage_ms[top]) * 1e3, 2),
+                         "peak_source": peaks["source"] + " (bf16 burst; the kernel computes fp16 at the same rate)"}}
+
+
+def side_measurements(args, layer, redraws, timed_steps, dev_name, peaks) -> dict:
+    """The other configurations of the layer, measured in the same run as the headline: NVFP4 decode
+    (T = 1, 8), the T = 2048 prefill in both formats and with skewed expert loads (int4)."""
+    from bit_routed_expert_sigmoid_b200 import synthetic as S
+    from bit_routed_expert_sigmoid_b200.layer import FlintMoELayer
+    E = 256
+    n_dec = min(args.steps, 1000)
+    n_pf = max(3, min(args.steps // 20, 50))
+    out = {"prefill_T2048": measure_prefill(layer, "int4", E, False, redraws, timed_steps, n_pf, dev_name, peaks,
+                                            "prefill_int4")}
+    Ls = S.make_layer(E, "int4", skew=True)
+    lay = FlintMoELayer(Ls, t_max=2048, device=dev_name)
+    del Ls
+    out["prefill_T2048_skew"] = measure_prefill(lay, "int4", E, True, S.redraw_table(E, skew=True), timed_steps,
+                                                n_pf, dev_name, peaks, "prefill_int4_skew")
+    lay.close()
+    Ln = S.make_layer(E, "nvfp4")
+    lay = FlintMoELayer(Ln, t_max=2048, device=dev_name)
+    del Ln
+    out["per_T_nvfp4"] = measure_per_T(lay, "nvfp4", E, (1, 8), redraws, timed_steps, n_dec, args.warmup, dev_name)
+    out["prefill_T2048_nvfp4"] = measure_prefill(lay, "nvfp4", E, False, redraws, timed_steps, n_pf, dev_name, peaks,
+                                                 "prefill_nvfp4")
+    lay.close()
+    return out
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
 
@@ -377,36 +481,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
            "ms_per_step": round(e2e_total / len(e2e_ms), 5)}
 
     extras = {}
-    if not args.no_extras and args.workload == "decode_int4":
-        per_t = {}
-        for tt_ in (1, 2, 4, 8):
-            xt = x_to_device(S.make_x(tt_, redraws=redraws), dev_name)
-            yt = torch.empty((tt_, H), dtype=torch.bfloat16, device=dev_name)
-            f = lambda: layer.forward(xt, yt)  # noqa: E731
-            for _ in range(args.warmup):
-                f()
-            na = int((torch.diff(layer.routing(tt_)["offsets"]) > 0).sum().item())
-            ms = statistics.mean(timed_steps(f, min(args.steps, 1000)))
-            ab = algorithmic_bytes(E, fmt, tt_, na)
-            per_t[str(tt_)] = {"us": round(ms * 1e3, 2), "tokens_per_s": round(tt_ / (ms * 1e-3), 1),
-                               "distinct_experts": na, "algorithmic_MB": round(ab / 1e6, 3),
-                               "GB_per_s": round(ab / (ms * 1e-3) / 1e9, 1),
-                               "pct_of_8TBps": round(100 * ab / (ms * 1e-3) / 1e9 / HBM_NOMINAL_GBS, 2)}
-        extras["per_T"] = per_t
-    if not args.no_extras:
-        Tp = 2048
-        xp = x_to_device(S.make_x(Tp, redraws=redraws), dev_name)
-        yp = torch.empty((Tp, H), dtype=torch.bfloat16, device=dev_name)
-        f = lambda: layer.forward(xp, yp)  # noqa: E731
-        for _ in range(3):
-            f()
-        ms = statistics.mean(timed_steps(f, max(3, min(args.steps // 20, 50))))
-        fl = grouped_gemm_flops(Tp)
-        tf = fl / (ms * 1e-3) / 1e12
-        extras["prefill_T2048"] = {"us": round(ms * 1e3, 1), "tokens_per_s": round(Tp / (ms * 1e-3), 1),
-                                   "grouped_gemm_TFLOPs": round(tf, 2),
-                                   "pct_of_2250TF_dense_bf16": round(100 * tf / BF16_DENSE_NOMINAL_TFLOPS, 2),
-                                   "pct_of_measured_bf16": round(100 * tf / peaks["bf16_tflops"], 2)}
+    if not args.no_extras and world == 1 and args.workload == "decode_int4":
+        extras["per_T"] = measure_per_T(layer, fmt, E, (1, 2, 4, 8), redraws, timed_steps, min(args.steps, 1000),
+                                        args.warmup, dev_name)
+    if not args.no_extras and world == 1 and args.workload == "decode_int4":
+        extras.update(side_measurements(args, layer, redraws, timed_steps, dev_name, peaks))
     clk = clocks.stop()
 
     result = None
