@@ -49,7 +49,7 @@ class flint_moe_cfg(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int), ("n_experts", ctypes.c_int), ("top_k", ctypes.c_int),
                 ("inter", ctypes.c_int), ("inter_shared", ctypes.c_int), ("fmt", ctypes.c_int),
                 ("t_max", ctypes.c_int), ("routed_scale", ctypes.c_float), ("norm_floor", ctypes.c_float),
-                ("flags", ctypes.c_uint)]
+                ("flags", ctypes.c_uint), ("n_slots", ctypes.c_int)]
 
 
 class flint_moe_weights(ctypes.Structure):
@@ -68,6 +68,12 @@ def _load():
         "flint_moe_create": (I, [P(flint_moe_cfg), P(flint_moe_weights), V, S, P(V)]),
         "flint_moe_forward": (I, [V, V, I, V, V]),
         "flint_moe_forward_host": (I, [V, V, I, V, V]),
+        "flint_moe_forward_routed": (I, [V, V, I, V, V, V, V]),
+        "flint_cache_create": (I, [V, P(flint_moe_weights), P(V)]),
+        "flint_cache_destroy": (I, [V]),
+        "flint_cache_stats": (I, [V, P(ctypes.c_longlong), P(ctypes.c_longlong), P(ctypes.c_longlong)]),
+        "flint_moe_forward_cached": (I, [V, V, V, I, V, V]),
+        "flint_cache_plan": (I, [I, I, P(I), P(I), P(ctypes.c_ulonglong), ctypes.c_ulonglong, P(I), I, P(I)]),
         "flint_moe_routing": (I, [V, V, V, V, V, V]),
         "flint_moe_intermediate": (I, [V, I, V, S, V]),
         "flint_moe_error_word": (I, [V, P(ctypes.c_uint)]),
@@ -115,6 +121,45 @@ def flint_moe_create(cfg: flint_moe_cfg, weights: flint_moe_weights, workspace: 
 def flint_moe_forward(h: int, x: int, T: int, y: int, stream: int = 0) -> None:
     _check(_lib.flint_moe_forward(ctypes.c_void_p(h), ctypes.c_void_p(x), int(T), ctypes.c_void_p(y),
                                   ctypes.c_void_p(stream)), "flint_moe_forward")
+
+
+def flint_moe_forward_routed(h: int, x: int, T: int, ids: int, w: int, y: int, stream: int = 0) -> None:
+    _check(_lib.flint_moe_forward_routed(ctypes.c_void_p(h), ctypes.c_void_p(x), int(T), ctypes.c_void_p(ids),
+                                         ctypes.c_void_p(w), ctypes.c_void_p(y), ctypes.c_void_p(stream)),
+           "flint_moe_forward_routed")
+
+
+def flint_cache_create(layer: int, host: flint_moe_weights) -> int:
+    c = ctypes.c_void_p()
+    _check(_lib.flint_cache_create(ctypes.c_void_p(layer), ctypes.byref(host), ctypes.byref(c)), "flint_cache_create")
+    return c.value
+
+
+def flint_cache_destroy(c: int) -> None:
+    _check(_lib.flint_cache_destroy(ctypes.c_void_p(c)), "flint_cache_destroy")
+
+
+def flint_cache_stats(c: int) -> tuple:
+    h, m, b = ctypes.c_longlong(), ctypes.c_longlong(), ctypes.c_longlong()
+    _check(_lib.flint_cache_stats(ctypes.c_void_p(c), ctypes.byref(h), ctypes.byref(m), ctypes.byref(b)),
+           "flint_cache_stats")
+    return h.value, m.value, b.value
+
+
+def flint_moe_forward_cached(h: int, c: int, x: int, T: int, y: int, stream: int = 0) -> None:
+    _check(_lib.flint_moe_forward_cached(ctypes.c_void_p(h), ctypes.c_void_p(c), ctypes.c_void_p(x), int(T),
+                                         ctypes.c_void_p(y), ctypes.c_void_p(stream)), "flint_moe_forward_cached")
+
+
+def flint_cache_plan(E: int, S: int, slot_of, expert_of, last_use, tick: int, ids, loads) -> int:
+    """Host-only replacement rule (no CUDA): numpy int32 slot_of [E], expert_of [S], uint64 last_use [S]
+    (updated in place), int32 ids [P], int32 loads [2S] (out). Returns the number of misses or -1."""
+    P_ = ctypes.POINTER
+    return int(_lib.flint_cache_plan(int(E), int(S), slot_of.ctypes.data_as(P_(ctypes.c_int)),
+                                     expert_of.ctypes.data_as(P_(ctypes.c_int)),
+                                     last_use.ctypes.data_as(P_(ctypes.c_ulonglong)), ctypes.c_ulonglong(tick),
+                                     ids.ctypes.data_as(P_(ctypes.c_int)), int(ids.size),
+                                     loads.ctypes.data_as(P_(ctypes.c_int))))
 
 
 def flint_moe_forward_host(h: int, x_host: int, T: int, y_host: int, stream: int = 0) -> None:

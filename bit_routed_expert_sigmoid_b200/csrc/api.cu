@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstring>
 #include <new>
+#include <vector>
 
 #include "../../include/flint_moe.h"
 #include "kernels.cuh"
@@ -27,6 +28,7 @@ struct flint_moe_ctx {
   int* inv;
   int* active;
   int* n_active;
+  int* slot_of;                            // [kMaxE] weight slot of each expert (cache mode)
   int4* etab;
   int* cnt;
   unsigned* err;
@@ -83,6 +85,7 @@ flint_status check_cfg(const flint_moe_cfg* c) {
   if (!(c->norm_floor > 0.f) || !(c->routed_scale == c->routed_scale)) return FLINT_ERR_INVALID_ARG;
   if (c->hidden != kH || c->inter != kI || c->inter_shared != kIs) return FLINT_ERR_UNSUPPORTED;
   if (c->n_experts % 32 != 0 || c->n_experts > kMaxE) return FLINT_ERR_UNSUPPORTED;
+  if (c->n_slots < 0 || c->n_slots > c->n_experts) return FLINT_ERR_INVALID_ARG;
   return FLINT_OK;
 }
 
@@ -168,6 +171,7 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
   char* p_inv = take(P * 4);
   char* p_active = take(E * 4);
   char* p_nact = take(16);
+  char* p_slot = take(kMaxE * 4);
   char* p_etab = take(kMaxActive * 2 * 16);
   char* p_cnt = take(kCntInts * 4);
   char* p_err = take(16);
@@ -196,6 +200,7 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
     h->inv = reinterpret_cast<int*>(p_inv);
     h->active = reinterpret_cast<int*>(p_active);
     h->n_active = reinterpret_cast<int*>(p_nact);
+    h->slot_of = reinterpret_cast<int*>(p_slot);
     h->etab = reinterpret_cast<int4*>(p_etab);
     h->cnt = reinterpret_cast<int*>(p_cnt);
     h->err = reinterpret_cast<unsigned*>(p_err);
@@ -249,7 +254,8 @@ struct StageMarks {
     if (_e != cudaSuccess) return FLINT_ERR_CUDA; \
   } while (0)
 
-flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y, cudaStream_t s) {
+// route_in: h->ids and h->wts already hold this forward's routing (no router, no top-k).
+flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y, cudaStream_t s, bool route_in = false) {
   const flint_moe_cfg& c = h->cfg;
   const int E = c.n_experts, K = c.top_k;
   const int fmt = c.fmt == FLINT_W_INT4_G128_FWHT128 ? kInt4 : kNvfp4;
@@ -300,6 +306,9 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
     d.ys = h->ys;
     d.err = h->err;
     d.cnt = h->cnt;
+    d.slot_of = c.n_slots > 0 ? h->slot_of : nullptr;
+    d.n_wslots = c.n_slots;
+    d.route_in = route_in ? 1 : 0;
     FLINT_TRY(launch_decode(d, h->n_sm, s));
     FLINT_TRY(m.mark());
     return FLINT_OK;
@@ -317,6 +326,8 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   pp.hs_lo = h->hs_lo;
   pp.ys = h->ys;
   pp.err = h->err;
+  pp.slot_of = c.n_slots > 0 ? h->slot_of : nullptr;
+  pp.n_wslots = c.n_slots;
   // B = x as given (map encoded per call: x changes, rows past T read as zeros)
   CUtensorMap tm_x;
   if (!encode_bf16_tiles(&tm_x, x, T, kH)) return FLINT_ERR_CUDA;
@@ -333,12 +344,14 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
     FLINT_TRY(cudaEventRecord(h->ev_fork, s));
     FLINT_TRY(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
   }
-  pp.tm_a = h->tm_pf_router;
-  pp.tm_b = tm_x;
-  FLINT_TRY(launch_prefill_shared(pp, kPhaseRouter, h->n_sm, rs));
-  FLINT_TRY(m.mark());
-  FLINT_TRY(launch_topk(h->logits_part, kRouterSplit, h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, rs));
-  FLINT_TRY(m.mark());
+  if (!route_in) {
+    pp.tm_a = h->tm_pf_router;
+    pp.tm_b = tm_x;
+    FLINT_TRY(launch_prefill_shared(pp, kPhaseRouter, h->n_sm, rs));
+    FLINT_TRY(m.mark());
+    FLINT_TRY(launch_topk(h->logits_part, kRouterSplit, h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, rs));
+    FLINT_TRY(m.mark());
+  }
   FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, c.flags, h->err, rs));
   FLINT_TRY(m.mark());
   FLINT_TRY(launch_xg(x, T, K, h->inv, fmt == kInt4 ? 1 : 0, h->xg, rs));
@@ -415,17 +428,18 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
   h->ws_bytes = workspace_bytes;
   plan(h, *cfg, h->ws);
   h->last_T = 0;
+  const int n_wrows = cfg->n_slots > 0 ? cfg->n_slots : cfg->n_experts;   // experts (or slots) of the routed arrays
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       cudaMemset(h->err, 0, 16) != cudaSuccess || cudaMemset(h->cnt, 0, kCntInts * 4) != cudaSuccess ||
-      !encode_rows(&h->tm_gu, w.gu_codes, static_cast<uint64_t>(cfg->n_experts) * 2 * kI, kH / 2, 64, 8) ||
+      !encode_rows(&h->tm_gu, w.gu_codes, static_cast<uint64_t>(n_wrows) * 2 * kI, kH / 2, 64, 8) ||
       (cfg->fmt == FLINT_W_NVFP4 &&
-       !encode_rows(&h->tm_gu_sc, w.gu_scales, static_cast<uint64_t>(cfg->n_experts) * 2 * kI, kH / 16, 8, 8)) ||
+       !encode_rows(&h->tm_gu_sc, w.gu_scales, static_cast<uint64_t>(n_wrows) * 2 * kI, kH / 16, 8, 8)) ||
       !encode_rows(&h->tm_sh_gu, w.sh_gu, 2 * kIs, kH * 2, 256, 2) ||
       !encode_rows(&h->tm_sh_dn, w.sh_dn, kH, kIs * 2, 64, 16) ||
-      !encode_code_tiles(&h->tm_pf_gu, w.gu_codes, static_cast<uint64_t>(cfg->n_experts) * 2 * kI, kH / 2) ||
-      !encode_code_tiles(&h->tm_pf_dn, w.dn_codes, static_cast<uint64_t>(cfg->n_experts) * kH, kI / 2) ||
+      !encode_code_tiles(&h->tm_pf_gu, w.gu_codes, static_cast<uint64_t>(n_wrows) * 2 * kI, kH / 2) ||
+      !encode_code_tiles(&h->tm_pf_dn, w.dn_codes, static_cast<uint64_t>(n_wrows) * kH, kI / 2) ||
       !encode_bf16_tiles(&h->tm_pf_sh_gu, w.sh_gu, 2 * kIs, kH) ||
       !encode_bf16_tiles(&h->tm_pf_sh_dn, w.sh_dn, kH, kIs) ||
       !encode_bf16_tiles(&h->tm_pf_router, w.router_w, cfg->n_experts, kH) ||
@@ -452,7 +466,7 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
 }
 
 flint_status flint_moe_forward(flint_moe_t h, const void* x, int T, void* y, void* stream) {
-  if (!h) return FLINT_ERR_INVALID_ARG;
+  if (!h || h->cfg.n_slots > 0) return FLINT_ERR_INVALID_ARG;
   if (T < 0 || T > h->cfg.t_max) return FLINT_ERR_INVALID_ARG;
   if (T == 0) return FLINT_OK;
   if (!aligned16(x) || !aligned16(y) || x == y) return FLINT_ERR_INVALID_ARG;
@@ -463,7 +477,7 @@ flint_status flint_moe_forward(flint_moe_t h, const void* x, int T, void* y, voi
 }
 
 flint_status flint_moe_forward_host(flint_moe_t h, const void* x_host, int T, void* y_host, void* stream) {
-  if (!h) return FLINT_ERR_INVALID_ARG;
+  if (!h || h->cfg.n_slots > 0) return FLINT_ERR_INVALID_ARG;
   if (T < 0 || T > h->cfg.t_max) return FLINT_ERR_INVALID_ARG;
   if (T == 0) return FLINT_OK;
   if (!x_host || !y_host) return FLINT_ERR_INVALID_ARG;
@@ -475,6 +489,22 @@ flint_status flint_moe_forward_host(flint_moe_t h, const void* x_host, int T, vo
   h->last_T = T;
   FLINT_TRY(cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, s));
   return FLINT_OK;
+}
+
+flint_status flint_moe_forward_routed(flint_moe_t h, const void* x, int T, const int* ids, const float* w, void* y,
+                                      void* stream) {
+  if (!h || h->cfg.n_slots > 0) return FLINT_ERR_INVALID_ARG;
+  if (T < 0 || T > h->cfg.t_max) return FLINT_ERR_INVALID_ARG;
+  if (T == 0) return FLINT_OK;
+  if (!aligned16(x) || !aligned16(y) || x == y || !ids || !w) return FLINT_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ids) & 3u) || (reinterpret_cast<uintptr_t>(w) & 3u)) return FLINT_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t P = static_cast<size_t>(T) * h->cfg.top_k;
+  FLINT_TRY(cudaMemcpyAsync(h->ids, ids, P * 4, cudaMemcpyDeviceToDevice, s));
+  FLINT_TRY(cudaMemcpyAsync(h->wts, w, P * 4, cudaMemcpyDeviceToDevice, s));
+  flint_status st = run_forward(h, static_cast<const uint16_t*>(x), T, static_cast<uint16_t*>(y), s, true);
+  if (st == FLINT_OK) h->last_T = T;
+  return st;
 }
 
 flint_status flint_residual_rmsnorm(float* x, const void* y, int T, float eps, void* z, void* stream) {
@@ -490,7 +520,7 @@ flint_status flint_moe_stack_forward(const flint_moe_t* layers, int n_layers, fl
                                      void* y, void* stream) {
   if (!layers || n_layers < 1 || T < 0 || !(eps > 0.f)) return FLINT_ERR_INVALID_ARG;
   for (int l = 0; l < n_layers; ++l)
-    if (!layers[l] || T > layers[l]->cfg.t_max) return FLINT_ERR_INVALID_ARG;
+    if (!layers[l] || T > layers[l]->cfg.t_max || layers[l]->cfg.n_slots > 0) return FLINT_ERR_INVALID_ARG;
   if (T == 0) return FLINT_OK;
   if (!aligned16(x) || !aligned16(z) || !aligned16(y) || z == y) return FLINT_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -587,6 +617,146 @@ const char* flint_moe_status_string(flint_status s) {
     case FLINT_ERR_TIMEOUT: return "bounded device wait timed out";
   }
   return "unknown status";
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------------- expert cache
+
+struct flint_expert_cache {
+  flint_moe_t layer;
+  flint_moe_weights host;                  // routed weights of all E experts, host memory [E][...]
+  size_t b_gu_codes, b_gu_scales, b_dn_codes, b_dn_scales;   // bytes per expert
+  std::vector<int> slot_of, expert_of;
+  std::vector<unsigned long long> last_use;
+  unsigned long long tick;
+  std::vector<int> ids, loads;
+  long long hits, misses, bytes;
+};
+
+extern "C" int flint_cache_plan(int E, int S, int* slot_of, int* expert_of, unsigned long long* last_use,
+                                unsigned long long tick, const int* ids, int P, int* loads) {
+  if (E < 1 || S < 1 || !slot_of || !expert_of || !last_use || (P > 0 && !ids) || !loads) return -1;
+  // distinct ids in order of first appearance, checked before anything changes
+  std::vector<int> uniq;
+  std::vector<char> seen(static_cast<size_t>(E), 0);
+  for (int q = 0; q < P; ++q) {
+    const int e = ids[q];
+    if (e < 0 || e >= E) return -1;
+    if (!seen[e]) {
+      seen[e] = 1;
+      uniq.push_back(e);
+    }
+  }
+  if (static_cast<int>(uniq.size()) > S) return -1;
+  for (int e : uniq)                       // hits keep their slots
+    if (slot_of[e] >= 0) last_use[slot_of[e]] = tick;
+  int n = 0;
+  for (int e : uniq) {
+    if (slot_of[e] >= 0) continue;
+    int v = -1;
+    for (int sl = 0; sl < S && v < 0; ++sl)
+      if (expert_of[sl] < 0) v = sl;       // a free slot
+    if (v < 0)                             // else the least recently used slot this forward does not need
+      for (int sl = 0; sl < S; ++sl)
+        if (last_use[sl] != tick && (v < 0 || last_use[sl] < last_use[v])) v = sl;
+    if (expert_of[v] >= 0) slot_of[expert_of[v]] = -1;
+    expert_of[v] = e;
+    slot_of[e] = v;
+    last_use[v] = tick;
+    loads[2 * n] = e;
+    loads[2 * n + 1] = v;
+    ++n;
+  }
+  return n;
+}
+
+extern "C" {
+
+flint_status flint_cache_create(flint_moe_t layer, const flint_moe_weights* host, flint_cache_t* out) {
+  if (!out) return FLINT_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!layer || !host || layer->cfg.n_slots <= 0) return FLINT_ERR_INVALID_ARG;
+  const flint_moe_cfg& c = layer->cfg;
+  if (!host->gu_codes || !host->gu_scales || !host->dn_codes || !host->dn_scales) return FLINT_ERR_INVALID_ARG;
+  if (c.fmt == FLINT_W_NVFP4 && (!host->gu_tscale || !host->dn_tscale)) return FLINT_ERR_INVALID_ARG;
+  if ((host->gu_tscale != nullptr) != (layer->w.gu_tscale != nullptr) ||
+      (host->dn_tscale != nullptr) != (layer->w.dn_tscale != nullptr))
+    return FLINT_ERR_INVALID_ARG;
+  flint_expert_cache* k = new (std::nothrow) flint_expert_cache();
+  if (!k) return FLINT_ERR_INVALID_ARG;
+  const bool i4 = c.fmt == FLINT_W_INT4_G128_FWHT128;
+  k->layer = layer;
+  k->host = *host;
+  k->b_gu_codes = static_cast<size_t>(2 * kI) * (kH / 2);
+  k->b_gu_scales = i4 ? static_cast<size_t>(2 * kI) * (kH / kGroup) * 2 : static_cast<size_t>(2 * kI) * (kH / 16);
+  k->b_dn_codes = static_cast<size_t>(kH) * (kI / 2);
+  k->b_dn_scales = i4 ? static_cast<size_t>(kH) * (kI / kGroup) * 2 : static_cast<size_t>(kH) * (kI / 16);
+  k->slot_of.assign(c.n_experts, -1);
+  k->expert_of.assign(c.n_slots, -1);
+  k->last_use.assign(c.n_slots, 0);
+  k->tick = 0;
+  k->ids.assign(static_cast<size_t>(c.t_max) * c.top_k, 0);
+  k->loads.assign(2 * static_cast<size_t>(c.n_slots), 0);
+  k->hits = k->misses = k->bytes = 0;
+  *out = k;
+  return FLINT_OK;
+}
+
+flint_status flint_cache_destroy(flint_cache_t c) {
+  delete c;
+  return FLINT_OK;
+}
+
+flint_status flint_cache_stats(flint_cache_t c, long long* hits, long long* misses, long long* bytes) {
+  if (!c) return FLINT_ERR_INVALID_ARG;
+  if (hits) *hits = c->hits;
+  if (misses) *misses = c->misses;
+  if (bytes) *bytes = c->bytes;
+  return FLINT_OK;
+}
+
+flint_status flint_moe_forward_cached(flint_moe_t h, flint_cache_t k, const void* x, int T, void* y, void* stream) {
+  if (!h || !k || k->layer != h) return FLINT_ERR_INVALID_ARG;
+  const flint_moe_cfg& c = h->cfg;
+  if (T < 0 || T > c.t_max) return FLINT_ERR_INVALID_ARG;
+  if (T == 0) return FLINT_OK;
+  if (!aligned16(x) || !aligned16(y) || x == y) return FLINT_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int E = c.n_experts, K = c.top_k, P = T * K;
+  // routing on the device, ids back to the host
+  FLINT_TRY(launch_router_logits(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(h->w.router_w), T, E,
+                                 h->logits, s));
+  FLINT_TRY(launch_topk(h->logits, 1, nullptr, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, s));
+  FLINT_TRY(cudaMemcpyAsync(k->ids.data(), h->ids, static_cast<size_t>(P) * 4, cudaMemcpyDeviceToHost, s));
+  FLINT_TRY(cudaStreamSynchronize(s));
+  // slots for the selected experts; copies of the misses
+  const int n = flint_cache_plan(E, c.n_slots, k->slot_of.data(), k->expert_of.data(), k->last_use.data(), ++k->tick,
+                                 k->ids.data(), P, k->loads.data());
+  if (n < 0) return FLINT_ERR_UNSUPPORTED;
+  int distinct = 0;
+  for (int sl = 0; sl < c.n_slots; ++sl) distinct += k->last_use[sl] == k->tick;
+  k->hits += distinct - n;
+  k->misses += n;
+  for (int i = 0; i < n; ++i) {
+    const size_t e = static_cast<size_t>(k->loads[2 * i]), v = static_cast<size_t>(k->loads[2 * i + 1]);
+    auto copy = [&](const void* dev_base, const void* host_base, size_t bytes) -> cudaError_t {
+      k->bytes += static_cast<long long>(bytes);
+      return cudaMemcpyAsync(static_cast<char*>(const_cast<void*>(dev_base)) + v * bytes,
+                             static_cast<const char*>(host_base) + e * bytes, bytes, cudaMemcpyHostToDevice, s);
+    };
+    FLINT_TRY(copy(h->w.gu_codes, k->host.gu_codes, k->b_gu_codes));
+    FLINT_TRY(copy(h->w.gu_scales, k->host.gu_scales, k->b_gu_scales));
+    FLINT_TRY(copy(h->w.dn_codes, k->host.dn_codes, k->b_dn_codes));
+    FLINT_TRY(copy(h->w.dn_scales, k->host.dn_scales, k->b_dn_scales));
+    if (h->w.gu_tscale) FLINT_TRY(copy(h->w.gu_tscale, k->host.gu_tscale, 2 * sizeof(float)));
+    if (h->w.dn_tscale) FLINT_TRY(copy(h->w.dn_tscale, k->host.dn_tscale, sizeof(float)));
+  }
+  // the slot map (pageable source: the driver stages it before the call returns)
+  FLINT_TRY(cudaMemcpyAsync(h->slot_of, k->slot_of.data(), static_cast<size_t>(E) * 4, cudaMemcpyHostToDevice, s));
+  flint_status st = run_forward(h, static_cast<const uint16_t*>(x), T, static_cast<uint16_t*>(y), s, true);
+  if (st == FLINT_OK) h->last_T = T;
+  return st;
 }
 
 }  // extern "C"

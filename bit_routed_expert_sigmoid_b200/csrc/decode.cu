@@ -483,11 +483,13 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& r
       toks |= static_cast<unsigned>(tt) << (4 * n);
       m &= m - 1;
     }
-    const float tsg = p.gu_ts ? __ldg(p.gu_ts + 2 * e) : 1.f;
-    const float tsu = p.gu_ts ? __ldg(p.gu_ts + 2 * e + 1) : 1.f;
-    const float tsd = p.dn_ts ? __ldg(p.dn_ts + e) : 1.f;
+    // weight index: the expert's cache slot when the weights sit in slots, else the expert itself
+    const int wi = p.slot_of ? min(max(__ldg(p.slot_of + e), 0), p.n_wslots - 1) : e;
+    const float tsg = p.gu_ts ? __ldg(p.gu_ts + 2 * wi) : 1.f;
+    const float tsu = p.gu_ts ? __ldg(p.gu_ts + 2 * wi + 1) : 1.f;
+    const float tsd = p.dn_ts ? __ldg(p.dn_ts + wi) : 1.f;
     const int4 t0 = make_int4(e, off, cnt, static_cast<int>(toks));
-    const int4 t1 = make_int4(__float_as_int(tsg), __float_as_int(tsu), __float_as_int(tsd), 0);
+    const int4 t1 = make_int4(__float_as_int(tsg), __float_as_int(tsu), __float_as_int(tsd), wi);
     rs.etab[slot][0] = t0;
     rs.etab[slot][1] = t1;
     if (publish) {
@@ -516,8 +518,9 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& r
 }
 
 // An expert-table entry; the fields are clamped so that a corrupt table cannot address out of range.
+// w is the index of the expert's weights (its cache slot when the weights sit in slots, else e).
 struct ExpertInfo {
-  int e, off, n;
+  int e, w, off, n;
   unsigned toks;
   float tsg, tsu, tsd;
 };
@@ -541,6 +544,7 @@ struct WarpTable {
     const int4 x = h ? a[1] : a[0], y = h ? b[1] : b[0];
     ExpertInfo r;
     r.e = min(max(__shfl_sync(kFull, x.x, src), 0), p.E - 1);
+    r.w = min(max(__shfl_sync(kFull, y.w, src), 0), (p.slot_of ? p.n_wslots : p.E) - 1);
     r.n = min(max(__shfl_sync(kFull, x.z, src), 0), kDecodeMaxT);
     r.off = min(max(__shfl_sync(kFull, x.y, src), 0), p.T * p.K - r.n);
     r.toks = static_cast<unsigned>(__shfl_sync(kFull, x.w, src));
@@ -638,7 +642,7 @@ __device__ void gu_issue(const DecodeParams& p, DecShared<FMT>& sm, Ring<FMT>& r
     return;
   }
   const int i0 = 8 * ((tile - kShGuTiles) % kGuTilesPerExpert);
-  const int erow = ex.e * (2 * kI);
+  const int erow = ex.w * (2 * kI);
   if constexpr (FMT == kInt4) {
     constexpr uint32_t row_sc = (kH / kGroup) * 2;   // 16 bf16 group scales per row
     if (lane == 0) {
@@ -735,7 +739,7 @@ __device__ void dn_issue(const DecodeParams& p, Ring<FMT>& ring, int item, int r
     return;
   }
   const ExpertInfo ex = tab.get(p, item - kShDnSlices);
-  const size_t row0 = static_cast<size_t>(ex.e) * kH + r0;
+  const size_t row0 = static_cast<size_t>(ex.w) * kH + r0;
   if (lane == 0) {
     if constexpr (FMT == kInt4) {
       const size_t re = row0 & ~static_cast<size_t>(1);
@@ -790,14 +794,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
     // router rows c and c + G on the tensor cores (K quarter rw each), then the operand segments
     const int rw = warp - kRouteWarp0, ri = threadIdx.x - kRouteWarp0 * 32;
     RouterRows rr;
-    rr.load(p, rw, c + G * g);
+    if (!p.route_in) rr.load(p, rw, c + G * g);
     wait_stage(p, &sm.xbar, 0);
-    rr.mma(p, rw, sm.u.ab.xs[0], kTokPitch, sm.rs.rpart);
+    if (!p.route_in) rr.mma(p, rw, sm.u.ab.xs[0], kTokPitch, sm.rs.rpart);
     if (rw == kWarps - kRouteWarp0 - 1)
       for (int sg = c; sg < p.T * (kH / kGroup); sg += G)
         xq_segment(p, sg / (kH / kGroup), sg % (kH / kGroup), sm.u.ab.xs[0], kTokPitch);
     named_bar_sync(kBarRoute, kRouteThreads);
-    if (rw == 0) {                                 // quarters added in order: one logit per lane
+    if (rw == 0 && !p.route_in) {                  // quarters added in order: one logit per lane
       const int r = lane >> 3, tok = lane & 7, e = c + G * r;
       if (tok < p.T && e < p.E) {
         const float* q = &sm.rs.rpart[0][r][tok];
@@ -832,7 +836,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
   }
   // ---------------------------------------------------------------- phase B: routing (every warp)
   wait_stage(p, &sm.logits_ready, 0);              // barrier 1 is passed: every CTA's logits and operand are in
-  if (warp < p.T) {                                // token `warp`
+  if (p.route_in) {                                // the routing is given: ids by ascending id per token
+    for (int q = threadIdx.x; q < p.T * p.K; q += kThreads) {
+      sm.rs.ids[q] = min(max(__ldcg(p.ids + q), 0), p.E - 1);
+      sm.rs.w[q] = __ldcg(p.wts + q);
+    }
+  } else if (warp < p.T) {                         // token `warp`
     float lv[8];
     unsigned kv[8];
     load_logits(p, warp, lv);

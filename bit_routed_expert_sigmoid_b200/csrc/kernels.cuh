@@ -60,6 +60,9 @@ struct DecodeParams {
   float* ys;                      // [T][H] shared-expert output
   unsigned* err;
   int* cnt;                       // [kCntInts]
+  const int* slot_of;             // [E] weight slot of each expert (weights in cache slots), or null
+  int n_wslots;                   // weight slots when slot_of is set
+  int route_in;                   // 1: ids and wts hold the routing already (no router, no top-k)
 };
 
 // Launches the decode kernel on `s` (grid = n_sm CTAs, cooperative). The caller has checked with
@@ -79,6 +82,8 @@ struct PrefillParams {
   CUtensorMap tm_b;               // shared: bf16 activations (x, or hs_hi), box 64 x 128 rows, 128-byte swizzle
   CUtensorMap tm_b2;              // shared down: hs_lo
   int T, top_k, E;
+  const int* slot_of;             // [E] weight slot of each expert (weights in cache slots), or null
+  int n_wslots;                   // weight slots when slot_of is set
   float* logits;                  // router phase output: partial logits [kRouterSplit][T][E]
   const int* offsets;             // [E+1]
   const int* perm;                // [P]

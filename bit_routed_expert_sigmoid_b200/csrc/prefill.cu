@@ -170,13 +170,14 @@ struct TileTab {
   int n, total;
   int start[kMaxE + 1];   // first tile of expert i
   int e[kMaxE];
+  int w[kMaxE];           // weight index of expert i: its slot when the weights sit in cache slots, else i
   int off[kMaxE];         // first permuted row
   int cnt[kMaxE];         // permuted rows
   int nch[kMaxE];         // chunks of kPfN rows
 };
 
 struct PfTile {
-  int e, row0, n, rp;     // expert, first permuted row of the chunk, rows in it (1..kPfN), block pair
+  int e, w, row0, n, rp;  // expert, its weight index, first permuted row of the chunk, rows in it (1..kPfN), block pair
 };
 
 // Warp 0: tiles of expert e are rp-major over its chunks; experts in ascending order (an expert
@@ -194,6 +195,7 @@ __device__ void build_tiles(TileTab& tt, const PrefillParams& p, int rp_count) {
       const int c = max(p.offsets[e + 1] - off, 0);
       const int nch = (c + kPfN - 1) / kPfN;
       tt.e[i] = e;
+      tt.w[i] = (p.slot_of && c > 0) ? min(max(p.slot_of[e], 0), p.n_wslots - 1) : e;
       tt.off[i] = off;
       tt.cnt[i] = c;
       tt.nch[i] = nch;
@@ -226,6 +228,7 @@ __device__ __forceinline__ PfTile tile_at(const TileTab& tt, int t) {
   const int rp = local / nch, ch = local - rp * nch;
   PfTile r;
   r.e = tt.e[lo];
+  r.w = tt.w[lo];
   r.row0 = tt.off[lo] + ch * kPfN;
   r.n = min(kPfN, tt.cnt[lo] - ch * kPfN);
   r.rp = rp;
@@ -361,7 +364,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
     if (lane == 0) {
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
         const PfTile tl = tile_at(tt, t);
-        const int r0 = G::row(tl.e, tl.rp, 0), r1 = G::row(tl.e, tl.rp, 1);
+        const int r0 = G::row(tl.w, tl.rp, 0), r1 = G::row(tl.w, tl.rp, 1);
         for (int s = 0; s < G::S; ++s, ++it) {
           const int slot = it % kPfDA;
           if (it >= kPfDA && !pf_wait(&bb.code_empty[slot], ((it / kPfDA) - 1) & 1, abort, p.err)) break;
@@ -460,7 +463,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
     int row = 0;
     if (t < total) {
       const PfTile tl = tile_at(tt, t);
-      row = G::row(tl.e, tl.rp, b) + r;
+      row = G::row(tl.w, tl.rp, b) + r;
       if constexpr (FMT == kInt4) load_int4(row);
       else load_fp4(row, 0);
     }
@@ -471,7 +474,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
       int row_next = -1;
       if (t_next < total) {
         const PfTile tn = tile_at(tt, t_next);
-        row_next = G::row(tn.e, tn.rp, b) + r;
+        row_next = G::row(tn.w, tn.rp, b) + r;
       }
       uint32_t sc[kSc4];                         // consumed from sc[0], shifted down every 2 stages
 #pragma unroll
@@ -550,8 +553,8 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
       if constexpr (PHASE == kPhaseGateUp) {
         float tsg = 1.f, tsu = 1.f;
         if (p.tscale) {
-          tsg = p.tscale[2 * tl.e];
-          tsu = p.tscale[2 * tl.e + 1];
+          tsg = p.tscale[2 * tl.w];
+          tsu = p.tscale[2 * tl.w + 1];
         }
         for (int j0 = 0; j0 < tl.n; j0 += 32) {
 #pragma unroll
@@ -579,7 +582,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
           named_bar_sync(1, 128);
         }
       } else {
-        const float ts = p.tscale ? p.tscale[tl.e] : 1.f;
+        const float ts = p.tscale ? p.tscale[tl.w] : 1.f;
         for (int j0 = 0; j0 < tl.n; j0 += 16) {
           uint32_t d0[16], d1[16];
           tc_ld16(dbase + j0, d0);

@@ -30,18 +30,29 @@ class FlintMoELayer:
     are copied to the device once; the handle borrows them and the workspace."""
 
     def __init__(self, L: dict, t_max: int, *, top_k: int = 6, device="cuda", flags: int = 0,
-                 routed_scale: float = 1.0, norm_floor: float = 2.0 ** -14):
+                 routed_scale: float = 1.0, norm_floor: float = 2.0 ** -14, n_slots: int = 0):
         self.device = torch.device(device)
         self.E = int(L["E"])
         self.top_k = top_k
         self.t_max = t_max
+        self.n_slots = n_slots
         fmt = B.FLINT_W_INT4_G128_FWHT128 if L["fmt"] == "int4" else B.FLINT_W_NVFP4
         self.cfg = B.flint_moe_cfg(hidden=L["H"], n_experts=self.E, top_k=top_k, inter=L["I"],
                                    inter_shared=L["Is"], fmt=fmt, t_max=t_max, routed_scale=routed_scale,
-                                   norm_floor=norm_floor, flags=flags)
-        self.tensors = {k: _to_device(L.get(k), self.device)
-                        for k in ("router_w", "gu_codes", "gu_scales", "gu_tscale", "dn_codes", "dn_scales",
-                                  "dn_tscale", "sh_gu", "sh_dn")}
+                                   norm_floor=norm_floor, flags=flags, n_slots=n_slots)
+        routed = ("gu_codes", "gu_scales", "gu_tscale", "dn_codes", "dn_scales", "dn_tscale")
+        if n_slots > 0:
+            # routed experts in page-locked host memory; the device holds n_slots expert slots
+            self.host = {k: (torch.from_numpy(np.ascontiguousarray(L[k]).view(
+                np.int16 if L[k].dtype == np.uint16 else L[k].dtype)).pin_memory() if L.get(k) is not None else None)
+                for k in routed}
+            self.tensors = {k: _to_device(L.get(k), self.device) for k in ("router_w", "sh_gu", "sh_dn")}
+            for k, v in self.host.items():
+                self.tensors[k] = (torch.zeros((n_slots,) + tuple(v.shape[1:]), dtype=v.dtype, device=self.device)
+                                   if v is not None else None)
+        else:
+            self.tensors = {k: _to_device(L.get(k), self.device)
+                            for k in ("router_w", "sh_gu", "sh_dn") + routed}
         ptr = {k: (v.data_ptr() if v is not None else None) for k, v in self.tensors.items()}
         self.weights = B.flint_moe_weights(**ptr)
         self.ws_bytes = B.flint_moe_workspace_size(self.cfg)
@@ -51,6 +62,11 @@ class FlintMoELayer:
         base = self.workspace.data_ptr()
         self.ws_ptr = (base + 255) // 256 * 256
         self.handle = B.flint_moe_create(self.cfg, self.weights, self.ws_ptr, self.ws_bytes)
+        self.cache = None
+        if n_slots > 0:
+            hp = {k: (v.data_ptr() if v is not None else None) for k, v in self.host.items()}
+            self.host_weights = B.flint_moe_weights(**hp)
+            self.cache = B.flint_cache_create(self.handle, self.host_weights)
 
     def weight_bytes(self) -> int:
         return sum(v.numel() * v.element_size() for v in self.tensors.values() if v is not None)
@@ -61,8 +77,25 @@ class FlintMoELayer:
         if y is None:
             y = torch.empty((T, H), dtype=torch.bfloat16, device=self.device)
         s = (stream or torch.cuda.current_stream(self.device)).cuda_stream
-        B.flint_moe_forward(self.handle, x.data_ptr(), T, y.data_ptr(), s)
+        if self.cache is not None:
+            B.flint_moe_forward_cached(self.handle, self.cache, x.data_ptr(), T, y.data_ptr(), s)
+        else:
+            B.flint_moe_forward(self.handle, x.data_ptr(), T, y.data_ptr(), s)
         return y
+
+    def forward_routed(self, x: torch.Tensor, ids: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+        """Forward on a given routing: ids int32 [T][top_k] (ascending per token), w f32 [T][top_k]."""
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty((T, H), dtype=torch.bfloat16, device=self.device)
+        s = (stream or torch.cuda.current_stream(self.device)).cuda_stream
+        B.flint_moe_forward_routed(self.handle, x.data_ptr(), T, ids.data_ptr(), w.data_ptr(), y.data_ptr(), s)
+        return y
+
+    def cache_stats(self) -> dict:
+        h, m, b = B.flint_cache_stats(self.cache)
+        return {"hits": h, "misses": m, "bytes": b}
 
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None) -> None:
         """x_host, y_host: [T][H] 16-bit host tensors (pinned for asynchronous copies)."""
@@ -97,6 +130,9 @@ class FlintMoELayer:
         return B.flint_moe_error_word(self.handle)
 
     def close(self) -> None:
+        if getattr(self, "cache", None):
+            B.flint_cache_destroy(self.cache)
+            self.cache = None
         if getattr(self, "handle", None):
             B.flint_moe_destroy(self.handle)
             self.handle = None

@@ -70,6 +70,9 @@ typedef struct flint_moe_cfg {
   float routed_scale; /* multiplies the routed sum (Flint: 1.0) */
   float norm_floor;   /* floor of the selected-score sum (Flint: 2^-14) */
   unsigned flags;     /* FLINT_FLAG_* */
+  int n_slots;        /* 0: the routed experts' weights are device arrays over all E experts. > 0: they
+                         are n_slots device slots of an expert cache (n_slots <= E), filled from host
+                         memory by flint_moe_forward_cached, the only forward such a handle takes */
 } flint_moe_cfg;
 
 /* Weight pointers (device, caller-owned, row-major [out][in]).
@@ -126,6 +129,46 @@ flint_status flint_moe_forward(flint_moe_t h, const void* x, int T, void* y, voi
  * copies): copies x into the workspace, runs the forward and copies y back, all on `stream`.
  * The caller synchronises the stream before reading y_host. */
 flint_status flint_moe_forward_host(flint_moe_t h, const void* x_host, int T, void* y_host, void* stream);
+
+/* As flint_moe_forward, with the routing given instead of computed: ids int32 [T][top_k] (device,
+ * distinct expert ids in [0, E), ascending within a token) and w f32 [T][top_k] (device), e.g. from
+ * flint_moe_route_noalloc or another router. The layer then runs its permutation, experts and
+ * combine on that routing (ids out of range are clamped). */
+flint_status flint_moe_forward_routed(flint_moe_t h, const void* x, int T, const int* ids, const float* w, void* y,
+                                      void* stream);
+
+/* Host-resident routed experts with a device cache of hot experts (WaveCut/Flint-UD-Q4_K_XL-NInfer-v3
+ * README, "Running": the routed experts may live in host memory; "Memory": per-layer expert banks).
+ * The layer handle is created with cfg.n_slots = S > 0 and its routed weight pointers at S device
+ * slots ([S][...] in the same per-expert layout as the [E][...] arrays); `host` holds the routed
+ * weights of all E experts in HOST memory ([E][...], page-locked so that the copies run
+ * asynchronously; router_w, sh_gu and sh_dn are not used). The cache keeps which expert sits in which
+ * slot and replaces the least recently used expert that the current forward does not need. Host
+ * memory only: the cache object allocates no device memory. */
+typedef struct flint_expert_cache* flint_cache_t;
+flint_status flint_cache_create(flint_moe_t layer, const flint_moe_weights* host, flint_cache_t* out);
+flint_status flint_cache_destroy(flint_cache_t c);
+/* hits and misses count expert loads (one per distinct expert of a forward); bytes = host-to-device
+ * bytes copied into slots. Any pointer may be NULL. */
+flint_status flint_cache_stats(flint_cache_t c, long long* hits, long long* misses, long long* bytes);
+
+/* y = MoE(x) with the routed experts in host memory: the routing runs on the device (router logits and
+ * top-k), the selected ids are read back (this call SYNCHRONISES `stream` once, mid-forward), every
+ * selected expert not in a slot is copied into one (cudaMemcpyAsync on `stream`), the slot map is
+ * uploaded and the forward runs on that routing with the weights read from the slots. More distinct
+ * selected experts than slots: FLINT_ERR_UNSUPPORTED, nothing enqueued beyond the routing. */
+flint_status flint_moe_forward_cached(flint_moe_t h, flint_cache_t c, const void* x, int T, void* y, void* stream);
+
+/* The cache's replacement rule as a pure host function (no CUDA call; exposed for tests and for
+ * callers that manage slots themselves). State: slot_of [E] (slot of each expert or -1), expert_of [S]
+ * (expert in each slot or -1), last_use [S] (tick of each slot's last use). ids [P] are the selected
+ * experts of one forward at time `tick` (> every last_use). Every distinct id gets a slot: a hit keeps
+ * its slot; a miss takes a free slot, else the slot with the smallest last_use among slots not used at
+ * `tick`; the state is updated. loads [2*S] receives (expert, slot) pairs of the misses in the order
+ * their ids first appear. Returns the number of misses, or -1 (state unchanged) when the distinct ids
+ * exceed S or an id is out of range. */
+int flint_cache_plan(int E, int S, int* slot_of, int* expert_of, unsigned long long* last_use, unsigned long long tick,
+                     const int* ids, int P, int* loads);
 
 /* Residual stream step of a stack of layers (the model's routed blocks with their weightless
  * RMSNorm; Aijuus/flint-w4exp, model summary): x f32 [T][H] (device, in/out) += y bf16 [T][H] when y is
