@@ -38,6 +38,13 @@ What the layer computes, and where the pages say so:
   count of kekzle/Flint-NVFP4, "What is in the files").
 * Combine: y = routed_scale * sum_k w_k * expert_k(x) + shared(x), computed here
   in fp64 without rounding; routed_scale is 1 (no scaling is named anywhere).
+* W4A4 (NVFP4 weights only): the routed experts' inputs, x and the SwiGLU
+  intermediate h, are themselves quantised to NVFP4 before each projection
+  (kekzle/Flint-NVFP4, evaluation table and serving notes: imp quantises the
+  activations in prefill, W4A4). Reading: per row (a token's x, a slot's h) an
+  F32 scale amax / (6 * 448), an E4M3 scale per 16 values along K and E2M1
+  codes, each decision taken in fp32 (quantize_act_nvfp4); the products and
+  sums after it stay fp64 here.
 
 Storage conventions (the pages do not fix them; readings listed in the design
 notes): int4 codes are two's complement with the low nibble holding the even K
@@ -256,8 +263,63 @@ def shared_weights(L: dict) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
     return S[:Is], S[Is:], bf16_to_f64(L["sh_dn"])
 
 
+# ----------------------------------------------------------------------------------------------
+# activation quantisation (W4A4)
+# ----------------------------------------------------------------------------------------------
+
+_E2M1_MIDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
+def _e2m1_nearest_even(a):
+    """|value| (non-negative) -> E2M1 magnitude code 0..7: nearest of 0, .5, 1, 1.5, 2, 3, 4, 6; at a
+    midpoint the even code; above 6 saturates to 6."""
+    a = np.asarray(a, dtype=np.float64)
+    code = np.zeros(a.shape, dtype=np.int64)
+    for i, mid in enumerate(_E2M1_MIDS):
+        code = np.where((a > mid) | ((a == mid) & ((i + 1) % 2 == 0)), i + 1, code)
+    return code
+
+
+def _e4m3_nearest_even_pos(x):
+    """Non-negative fp32 value -> E4M3 (fn) byte, nearest with ties to even, saturating at 448."""
+    x = np.asarray(x, dtype=np.float64)
+    grid = e4m3fn_to_f64(np.arange(0x7F))                  # every finite non-negative code, ascending
+    idx = np.clip(np.searchsorted(grid, x), 1, 0x7E)
+    lo, hi = grid[idx - 1], grid[idx]
+    pick_hi = (x - lo > hi - x) | ((x - lo == hi - x) & (idx % 2 == 0))
+    code = np.where(pick_hi, idx, idx - 1)
+    return np.where(x >= 448.0, 0x7E, code).astype(np.uint8)
+
+
+def quantize_act_nvfp4(v) -> dict:
+    """Rows of activations [R][K] (K a multiple of 16) -> NVFP4 per row, every decision in IEEE fp32 in
+    this order: ts = amax / 2688 (1 for an all-zero row); per 16-block sb = E4M3(bm / (6 * ts)) (the
+    product and the quotient each rounded to fp32, then nearest-even E4M3, saturating at 448);
+    d = sb * ts (rounded to fp32); code = E2M1(v / d) (fp32 quotient, nearest, ties to the even code,
+    sign from v; 0 where d = 0). Returns {codes (signed E2M1 values' nibbles) [R][K], scales [R][K/16]
+    (E4M3 bytes), ts [R] (f32), values [R][K] (fp64 dequantised: e2m1 x sb x ts)}."""
+    v = np.asarray(v, dtype=np.float32)
+    R_, K = v.shape
+    a = np.abs(v)
+    amax = a.max(axis=1)
+    ts = np.where(amax > 0, (amax / np.float32(2688.0)).astype(np.float32), np.float32(1.0)).astype(np.float32)
+    bm = a.reshape(R_, K // 16, 16).max(axis=2)
+    six_ts = (np.float32(6.0) * ts).astype(np.float32)
+    q = (bm / six_ts[:, None]).astype(np.float32)
+    sb = _e4m3_nearest_even_pos(q)
+    sv = e4m3fn_to_f64(sb).astype(np.float32)
+    d = (sv * ts[:, None]).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = np.where(d[:, :, None] > 0, v.reshape(R_, K // 16, 16) / d[:, :, None], np.float32(0.0)).astype(np.float32)
+    mag = _e2m1_nearest_even(np.abs(r))
+    sign = np.signbit(v.reshape(R_, K // 16, 16)).astype(np.int64)
+    nib = (mag | (sign << 3)).reshape(R_, K)
+    vals = e2m1_to_f64(nib) * np.repeat(e4m3fn_to_f64(sb), 16, axis=1) * ts.astype(np.float64)[:, None]
+    return {"codes": nib, "scales": sb, "ts": ts, "values": vals}
+
+
 def moe_forward(L: dict, x_bits: np.ndarray, *, top_k: int = TOP_K, floor: float = NORM_FLOOR,
-                routed_scale: float = 1.0, keep: bool = False, expert_override=None) -> dict:
+                routed_scale: float = 1.0, keep: bool = False, expert_override=None, w4a4: bool = False) -> dict:
     """Whole-layer forward in fp64.
 
     x_bits: bf16 bits [T][H]. Returns y [T][H] (fp64, unrounded), the routing (logits, ids, w,
@@ -266,7 +328,9 @@ def moe_forward(L: dict, x_bits: np.ndarray, *, top_k: int = TOP_K, floor: float
     h (SwiGLU intermediate before re-rotation), h_in (the down projection's input) and o (the
     expert output before weighting).
 
-    expert_override(e) may return fp64 (gate, up, down) to use instead of the stored codes."""
+    expert_override(e) may return fp64 (gate, up, down) to use instead of the stored codes.
+    w4a4 (NVFP4 layers): the routed experts see their inputs quantised per row (quantize_act_nvfp4):
+    x before gate|up, and h (rounded to fp32 first, the precision it is formed in) before down."""
     x = bf16_to_f64(x_bits)
     T, H = x.shape
     E = L["E"]
@@ -290,7 +354,16 @@ def moe_forward(L: dict, x_bits: np.ndarray, *, top_k: int = TOP_K, floor: float
         flat = pm["perm"][lo:hi]
         toks = flat // top_k
         ks = flat % top_k
-        res = swiglu_mlp(x[toks], Wg, Wu, Wd, rotated)
+        if w4a4:
+            if rotated:
+                raise ValueError("W4A4 is defined for the NVFP4 format")
+            xq = quantize_act_nvfp4(x[toks].astype(np.float32))["values"]
+            g, u = xq @ Wg.T, xq @ Wu.T
+            h = silu(g) * u
+            hq = quantize_act_nvfp4(h.astype(np.float32))["values"]
+            res = {"x_in": xq, "g": g, "u": u, "h": h, "h_in": hq, "out": hq @ Wd.T}
+        else:
+            res = swiglu_mlp(x[toks], Wg, Wu, Wd, rotated)
         for j in range(hi - lo):
             y_routed[toks[j]] += w[toks[j], ks[j]] * res["out"][j]
         if keep:
