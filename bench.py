@@ -44,10 +44,14 @@ WORKLOADS = {
     "prefill_int4_skew": (256, "int4", 2048, True),
     "decode_nvfp4": (256, "nvfp4", 8, False),
     "prefill_nvfp4": (256, "nvfp4", 2048, False),
+    "prefill_nvfp4_w4a4": (256, "nvfp4", 2048, False),
     "stack47_int4": (256, "int4", 8, False),
 }
 # stacks: layers of the workload (layer l drawn with seed 1000 + l); T tokens decode through all of them
 STACK_LAYERS = {"stack47_int4": 47}
+# W4A4: the routed experts' activations quantised to NVFP4, block-scaled FP4 MMAs
+W4A4_WORKLOADS = {"prefill_nvfp4_w4a4"}
+FP4_OVER_BF16_NOMINAL = 4.0          # dense FP4 / dense bf16 tensor rate (9 / 2.25 PFLOP/s)
 # weight preparation: the bf16 gate|up and down banks of all E experts quantised once per step
 QUANT_WORKLOADS = {"quant_int4": (256, "int4"), "quant_nvfp4": (256, "nvfp4")}
 QUANT_SEED = 7
@@ -89,13 +93,22 @@ def grouped_gemm_flops(T: int, K: int = 6) -> int:
     return routed + shared
 
 
-def stage_bytes(name: str, E: int, fmt: str, T: int, K: int, n_active: int) -> int:
+def stage_bytes(name: str, E: int, fmt: str, T: int, K: int, n_active: int, w4a4: bool = False) -> int:
     """Algorithmic bytes of one kernel launch (weights it must stream plus its activations)."""
     P = T * K
     eb_gu = 2 * I * H // 2 + (2 * I * (H // 128) * 2 if fmt == "int4" else 2 * I * (H // 16) + 8)
     eb_dn = H * I // 2 + (H * (I // 128) * 2 if fmt == "int4" else H * (I // 16) + 4)
     sc_x = T * (H // 128) * 4 if fmt == "int4" else 0          # units of the 16-bit activation limbs
     sc_h = P * (I // 128) * 4 if fmt == "int4" else 0
+    if w4a4:
+        xa = P * (H // 2 + H // 16 + 4)                        # NVFP4 rows: codes, block scales, tensor scale
+        ha = P * (I // 2 + I // 16 + 4)
+        w4 = {"xq": T * H * 2 + xa + P * 4,
+              "gu_routed": n_active * eb_gu + xa + P * I * 4,
+              "hq": P * I * 4 + ha,
+              "dn_routed": n_active * eb_dn + ha + P * H * 2}
+        if name in w4:
+            return w4[name]
     return {
         # decode path (T <= 8): one kernel moves the whole layer
         "layer": algorithmic_bytes(E, fmt, T, n_active),
@@ -122,6 +135,33 @@ def stage_flops(name: str, E: int, T: int, K: int) -> int:
         "gu_shared": 2 * T * 2 * IS * H,
         "dn_shared": 2 * T * H * IS * 2,      # bf16 pair (hi + lo) of the hidden activations
     }.get(name, 0)
+
+
+def prefill_roofline(name: str, kernel_ms: float, E: int, fmt: str, T: int, n_active: int, peaks: dict,
+                     workload: str, w4a4: bool) -> dict:
+    """Roofline of one prefill kernel. W4A16: against the bf16 tensor peak (the kernel computes fp16,
+    same rate). W4A4: the FP4 peak is the measured bf16 peak x the nominal FP4/bf16 ratio, and the
+    kernel is judged against whichever of HBM and tensor time is the larger at its sizes."""
+    st_flops = stage_flops(name, E, T, 6)
+    st_bytes = stage_bytes(name, E, fmt, T, 6, n_active, w4a4)
+    sec = kernel_ms * 1e-3
+    tf = st_flops / sec / 1e12
+    gbs = st_bytes / sec / 1e9
+    base = {"kernel": name, "traffic": ncu_traffic(name, workload), "algorithmic_flops": st_flops,
+            "algorithmic_bytes": st_bytes, "kernel_us": round(kernel_ms * 1e3, 2)}
+    if not w4a4:
+        return {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(tf / peaks["bf16_tflops"], 4), "hbm_GB_per_s": round(gbs, 1), **base,
+                "peak_source": peaks["source"] + " (bf16 burst; the kernel computes fp16 at the same rate)"}
+    fp4 = peaks["bf16_tflops"] * FP4_OVER_BF16_NOMINAL
+    t_hbm, t_tc = st_bytes / (peaks["hbm_gbs"] * 1e9), st_flops / (fp4 * 1e12)
+    if t_hbm >= t_tc:
+        return {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(gbs / peaks["hbm_gbs"], 4), "tensor_TFLOPs": round(tf, 2), "fp4_peak_TFLOPs": round(fp4, 1),
+                **base, "peak_source": peaks["source"] + " (burst copy; HBM time exceeds FP4 tensor time here)"}
+    return {"bound": "tensor", "achieved": round(tf, 2), "peak": round(fp4, 1), "unit": "TFLOP/s",
+            "frac": round(tf / fp4, 4), "hbm_GB_per_s": round(gbs, 1), **base,
+            "peak_source": peaks["source"] + " (bf16 burst x 4, the nominal dense FP4/bf16 ratio)"}
 
 
 def measured_peaks() -> dict:
@@ -285,7 +325,7 @@ def measure_per_T(layer, fmt, E, Ts, redraws, timed_steps, steps, warmup, dev_na
     return out
 
 
-def measure_prefill(layer, fmt, E, skew, redraws, timed_steps, steps, dev_name, peaks, workload):
+def measure_prefill(layer, fmt, E, skew, redraws, timed_steps, steps, dev_name, peaks, workload, w4a4=False):
     """One T = 2048 forward: device time, grouped-GEMM TFLOP/s, and the roofline of its slowest kernel
     (per-kernel CUDA-event times from the library's stage events, an instrumented pass that serialises
     the kernels)."""
@@ -321,28 +361,21 @@ def measure_prefill(layer, fmt, E, skew, redraws, timed_steps, steps, dev_name, 
     B.flint_moe_set_stage_events(layer.handle, None)
     stage_ms = acc / n_prof
     top = int(np.argmax(stage_ms))
-    st_flops = stage_flops(names[top], E, Tp, 6)
-    st_bytes = stage_bytes(names[top], E, fmt, Tp, 6, n_active)
-    achieved = st_flops / (stage_ms[top] * 1e-3) / 1e12
     return {"us": round(ms * 1e3, 1), "tokens_per_s": round(Tp / (ms * 1e-3), 1),
             "grouped_gemm_TFLOPs": round(tf, 2),
             "pct_of_2250TF_dense_bf16": round(100 * tf / BF16_DENSE_NOMINAL_TFLOPS, 2),
             "pct_of_measured_bf16": round(100 * tf / peaks["bf16_tflops"], 2),
             "distinct_experts": n_active,
             "stage_us_serialised": {n: round(float(t) * 1e3, 2) for n, t in zip(names, stage_ms)},
-            "roofline": {"bound": "tensor", "kernel": names[top], "achieved": round(achieved, 2),
-                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": round(achieved / peaks["bf16_tflops"], 4),
-                         "traffic": ncu_traffic(names[top], workload), "algorithmic_flops": st_flops,
-                         "algorithmic_bytes": st_bytes,
-                         "hbm_GB_per_s": round(st_bytes / (stage_ms[top] * 1e-3) / 1e9, 1),
-                         "kernel_us": round(float(stage_ms[top]) * 1e3, 2),
-                         "peak_source": peaks["source"] + " (bf16 burst; the kernel computes fp16 at the same rate)"}}
+            "roofline": prefill_roofline(names[top], float(stage_ms[top]), E, fmt, Tp, n_active, peaks, workload,
+                                         w4a4)}
 
 
 def side_measurements(args, layer, redraws, timed_steps, dev_name, peaks) -> dict:
     """The other configurations of the layer, measured in the same run as the headline: NVFP4 decode
-    (T = 1, 8), the T = 2048 prefill in both formats and with skewed expert loads (int4)."""
+    (T = 1, 8), the T = 2048 prefill in both formats, with skewed expert loads (int4) and with NVFP4
+    activations (W4A4)."""
+    from bit_routed_expert_sigmoid_b200 import binding as B
     from bit_routed_expert_sigmoid_b200 import synthetic as S
     from bit_routed_expert_sigmoid_b200.layer import FlintMoELayer
     E = 256
@@ -358,10 +391,14 @@ def side_measurements(args, layer, redraws, timed_steps, dev_name, peaks) -> dic
     lay.close()
     Ln = S.make_layer(E, "nvfp4")
     lay = FlintMoELayer(Ln, t_max=2048, device=dev_name)
-    del Ln
     out["per_T_nvfp4"] = measure_per_T(lay, "nvfp4", E, (1, 8), redraws, timed_steps, n_dec, args.warmup, dev_name)
     out["prefill_T2048_nvfp4"] = measure_prefill(lay, "nvfp4", E, False, redraws, timed_steps, n_pf, dev_name, peaks,
                                                  "prefill_nvfp4")
+    lay.close()
+    lay = FlintMoELayer(Ln, t_max=2048, device=dev_name, flags=B.FLINT_FLAG_W4A4)
+    del Ln
+    out["prefill_T2048_nvfp4_w4a4"] = measure_prefill(lay, "nvfp4", E, False, redraws, timed_steps, n_pf, dev_name,
+                                                      peaks, "prefill_nvfp4_w4a4", w4a4=True)
     lay.close()
     return out
 
@@ -385,7 +422,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     K_TOP = 6
     L = S.make_layer(E, fmt, skew=skew)
     t_max = max(T, 8)
-    layer = FlintMoELayer(L, t_max=max(t_max, 2048 if not args.no_extras else t_max), device=dev_name)
+    w4a4 = args.workload in W4A4_WORKLOADS
+    layer = FlintMoELayer(L, t_max=max(t_max, 2048 if not args.no_extras else t_max), device=dev_name,
+                          flags=B.FLINT_FLAG_W4A4 if w4a4 else 0)
     # each rank takes its own batch of token rows (weak scaling: T tokens per GPU)
     redraws = S.redraw_table(E, skew=skew)
     x_bits = S.make_x(T, skew=skew, redraws=redraws, first_row=rank_first_row(rank, T))
@@ -447,18 +486,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     stage_ms = acc / n_prof
     top = int(np.argmax(stage_ms))
     peaks = measured_peaks()
-    st_bytes = stage_bytes(names[top], E, fmt, T, K_TOP, n_active)
+    st_bytes = stage_bytes(names[top], E, fmt, T, K_TOP, n_active, w4a4)
     st_flops = stage_flops(names[top], E, T, K_TOP)
     if T > 8 and st_flops:
-        # prefill: a dense contraction, against the bf16 tensor peak (the kernel computes in fp16,
-        # same tensor rate as bf16 on this part)
-        achieved = st_flops / (stage_ms[top] * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "kernel": names[top], "achieved": round(achieved, 2),
-                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                    "traffic": ncu_traffic(names[top], args.workload), "algorithmic_flops": st_flops,
-                    "algorithmic_bytes": st_bytes,
-                    "hbm_GB_per_s": round(st_bytes / (stage_ms[top] * 1e-3) / 1e9, 1),
-                    "peak_source": peaks["source"] + " (bf16 burst)"}
+        roofline = prefill_roofline(names[top], float(stage_ms[top]), E, fmt, T, n_active, peaks, args.workload, w4a4)
     else:
         achieved = st_bytes / (stage_ms[top] * 1e-3) / 1e9
         roofline = {"bound": "hbm", "kernel": names[top], "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
@@ -496,7 +527,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": ("w4a16: int4 codes as exact int8 on the integer tensor cores against 16-bit fixed-point "
+            "dtype": ("w4a4: NVFP4 weights x NVFP4 activations (per-row fp32 scale, E4M3 per 16) on tcgen05 "
+                      "kind::mxf4nvf4 block-scaled MMAs, fp32 accumulators in tensor memory; shared expert and "
+                      "router bf16" if w4a4 else
+                      "w4a16: int4 codes as exact int8 on the integer tensor cores against 16-bit fixed-point "
                       "activations (int32 sums), fp32 accumulate" if fmt == "int4" and T <= 8 else
                       "w4a16: fp16 tensor-core MMA, fp32 accumulate" if T <= 8 else
                       "w4a16: tcgen05 kind::f16 MMA (weights dequantised to exact fp16 in tensor memory, fp16 "
@@ -538,7 +572,7 @@ def cpu_baseline(args, L, x_bits, E) -> dict:
     xs = x_bits[:Ts]
     reps, t0 = 0, time.perf_counter()
     while True:
-        R.moe_forward(L, xs)
+        R.moe_forward(L, xs, w4a4=args.workload in W4A4_WORKLOADS)
         reps += 1
         el = time.perf_counter() - t0
         if el >= args.cpu_seconds or reps >= 1000:
@@ -591,11 +625,11 @@ def run_reference(args) -> dict:
     Ts = T if T <= 64 else 64
     x_bits = S.make_x(Ts, skew=skew, redraws=S.redraw_table(E, skew=skew))
     for _ in range(min(args.warmup, 1)):
-        R.moe_forward(L, x_bits)
+        R.moe_forward(L, x_bits, w4a4=args.workload in W4A4_WORKLOADS)
     steps = max(1, min(args.steps, 20 if Ts <= 8 else 5))
     t0 = time.perf_counter()
     for _ in range(steps):
-        R.moe_forward(L, x_bits)
+        R.moe_forward(L, x_bits, w4a4=args.workload in W4A4_WORKLOADS)
     el = time.perf_counter() - t0
     value = steps * Ts / el
     cores = blas_threads()

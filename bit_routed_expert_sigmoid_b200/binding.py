@@ -25,10 +25,19 @@ FLINT_ERR_TIMEOUT = 6
 FLINT_W_INT4_G128_FWHT128 = 0
 FLINT_W_NVFP4 = 1
 FLINT_FLAG_DEBUG_CHECKS = 0x1
+FLINT_FLAG_W4A4 = 0x2
 
 FLINT_BUF_LOGITS = 0
 FLINT_BUF_XQ = 1
 FLINT_BUF_YS = 2
+FLINT_BUF_XA = 3
+FLINT_BUF_XA_SF = 4
+FLINT_BUF_XA_TS = 5
+FLINT_BUF_H = 6
+FLINT_BUF_HA = 7
+FLINT_BUF_HA_SF = 8
+FLINT_BUF_HA_TS = 9
+FLINT_BUF_O = 10
 
 EXPORTS = (
     "flint_moe_workspace_size", "flint_moe_create", "flint_moe_forward", "flint_moe_forward_host",

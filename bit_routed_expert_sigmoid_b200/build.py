@@ -8,7 +8,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libflint_moe.so")
-SOURCES = ["api.cu", "route.cu", "decode.cu", "prefill.cu", "stack.cu", "noalloc.cu", "quant.cu"]
+SOURCES = ["api.cu", "route.cu", "decode.cu", "prefill.cu", "stack.cu", "noalloc.cu", "quant.cu", "w4a4.cu"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
               "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]
 

@@ -46,7 +46,14 @@ struct flint_moe_ctx {
   float* ys;
   uint16_t* x_stage;
   uint16_t* y_stage;
+  uint8_t* xa;                             // W4A4: x codes [P][H/2], scales [P][H/16], tensor scales [P]
+  uint8_t* xa_sf;
+  float* xa_ts;
+  uint8_t* ha;                             // W4A4: h codes [P][I/2], scales [P][I/16], tensor scales [P]
+  uint8_t* ha_sf;
+  float* ha_ts;
   int last_T;
+  bool w4a4;
   int n_sm;
   CUtensorMap tm_gu, tm_gu_sc, tm_sh_gu, tm_sh_dn;  // tensor maps of the decode kernel's weight copies
   CUtensorMap tm_pf_gu, tm_pf_dn;          // prefill: routed codes, 16-word x 128-row boxes, 64-byte swizzle
@@ -54,6 +61,10 @@ struct flint_moe_ctx {
   CUtensorMap tm_pf_router;                // prefill: router rows [E][H], 64 x 128 bf16 boxes
   CUtensorMap tm_pf_hs_hi, tm_pf_hs_lo;    // prefill: shared-expert hidden pair [t_max][Is]
   CUtensorMap tm_pf_xg, tm_pf_hq;          // prefill: routed activation rows (fp16, 64 x 16 boxes)
+  CUtensorMap tm_w4_gu, tm_w4_dn;          // W4A4: weight codes as bytes, 128 x 128-row boxes, 128-byte swizzle
+  CUtensorMap tm_w4_gu_sc, tm_w4_dn_sc;    // W4A4: weight block scales, 16-byte x 128-row boxes
+  CUtensorMap tm_w4_xa, tm_w4_ha;          // W4A4: activation codes, 128 x 16-row boxes, 128-byte swizzle
+  CUtensorMap tm_w4_xa_sc, tm_w4_ha_sc;    // W4A4: activation block scales, 16-byte x 16-row boxes
   // instrumentation (caller-owned cudaEvent_t handles)
   cudaEvent_t events[32];
   int n_events;
@@ -86,6 +97,7 @@ flint_status check_cfg(const flint_moe_cfg* c) {
   if (c->hidden != kH || c->inter != kI || c->inter_shared != kIs) return FLINT_ERR_UNSUPPORTED;
   if (c->n_experts % 32 != 0 || c->n_experts > kMaxE) return FLINT_ERR_UNSUPPORTED;
   if (c->n_slots < 0 || c->n_slots > c->n_experts) return FLINT_ERR_INVALID_ARG;
+  if ((c->flags & FLINT_FLAG_W4A4) && c->fmt != FLINT_W_NVFP4) return FLINT_ERR_UNSUPPORTED;
   return FLINT_OK;
 }
 
@@ -139,6 +151,16 @@ bool encode_f16_rows16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
   return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rows, cols * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// W4A4 operands: bytes, box of 128 bytes x box_rows rows with the 128-byte swizzle (codes) or of
+// 16 bytes without swizzle (block scales)
+bool encode_fp4_tiles(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
+  return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, row_bytes, 128, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool encode_sf_tiles(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
+  return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, row_bytes, 16, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 bool encode_code_tiles(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes) {
   return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, rows, row_bytes, 16, 128, CU_TENSOR_MAP_SWIZZLE_64B);
 }
@@ -189,6 +211,13 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
   char* p_ys = take(T * kH * 4);
   char* p_xs = take(T * kH * 2);
   char* p_ys2 = take(T * kH * 2);
+  const size_t PA = (c.flags & FLINT_FLAG_W4A4) ? P : 0;      // W4A4 buffers only when asked for
+  char* p_xa = take(PA * kH / 2);
+  char* p_xa_sf = take(PA * kH / 16);
+  char* p_xa_ts = take(PA * 4);
+  char* p_ha = take(PA * kI / 2);
+  char* p_ha_sf = take(PA * kI / 16);
+  char* p_ha_ts = take(PA * 4);
   if (h) {
     h->logits = reinterpret_cast<float*>(p_logits);
     h->logits_part = reinterpret_cast<float*>(p_lpart);
@@ -218,6 +247,12 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
     h->ys = reinterpret_cast<float*>(p_ys);
     h->x_stage = reinterpret_cast<uint16_t*>(p_xs);
     h->y_stage = reinterpret_cast<uint16_t*>(p_ys2);
+    h->xa = reinterpret_cast<uint8_t*>(p_xa);
+    h->xa_sf = reinterpret_cast<uint8_t*>(p_xa_sf);
+    h->xa_ts = reinterpret_cast<float*>(p_xa_ts);
+    h->ha = reinterpret_cast<uint8_t*>(p_ha);
+    h->ha_sf = reinterpret_cast<uint8_t*>(p_ha_sf);
+    h->ha_ts = reinterpret_cast<float*>(p_ha_ts);
   }
   return off;
 }
@@ -226,15 +261,24 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
 const char* const kDecodeStages[] = {"layer"};
 const char* const kGemvStages[] = {"router_logits", "topk", "permute", "xq", "gu_shared",
                                    "gu_routed", "dn_routed", "dn_shared", "combine"};
+// W4A4: the SwiGLU output is quantised between the routed projections
+const char* const kW4a4Stages[] = {"router_logits", "topk", "permute", "xq", "gu_shared",
+                                   "gu_routed", "hq", "dn_routed", "dn_shared", "combine"};
 
-int stage_count(const flint_moe_ctx*, int T) {
-  return T <= kDecodeMaxT ? static_cast<int>(sizeof(kDecodeStages) / sizeof(kDecodeStages[0]))
-                          : static_cast<int>(sizeof(kGemvStages) / sizeof(kGemvStages[0]));
+template <size_t N>
+constexpr int count_of(const char* const (&)[N]) {
+  return static_cast<int>(N);
+}
+
+int stage_count(const flint_moe_ctx* h, int T) {
+  if (T <= kDecodeMaxT) return count_of(kDecodeStages);
+  return h->w4a4 ? count_of(kW4a4Stages) : count_of(kGemvStages);
 }
 
 const char* stage_name(const flint_moe_ctx* h, int T, int i) {
   if (i < 0 || i >= stage_count(h, T)) return nullptr;
-  return T <= kDecodeMaxT ? kDecodeStages[i] : kGemvStages[i];
+  if (T <= kDecodeMaxT) return kDecodeStages[i];
+  return h->w4a4 ? kW4a4Stages[i] : kGemvStages[i];
 }
 
 // Records the next instrumentation event, if any.
@@ -354,7 +398,8 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   }
   FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, c.flags, h->err, rs));
   FLINT_TRY(m.mark());
-  FLINT_TRY(launch_xg(x, T, K, h->inv, fmt == kInt4 ? 1 : 0, h->xg, rs));
+  if (h->w4a4) FLINT_TRY(launch_act_quant_x(x, T, K, h->inv, h->xa, h->xa_sf, h->xa_ts, rs));
+  else FLINT_TRY(launch_xg(x, T, K, h->inv, fmt == kInt4 ? 1 : 0, h->xg, rs));
   FLINT_TRY(m.mark());
 
   pp.tm_a = h->tm_pf_sh_gu;                        // shared gate|up: B = x
@@ -369,18 +414,40 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
     FLINT_TRY(cudaEventRecord(h->ev_join, h->side));
     FLINT_TRY(cudaStreamWaitEvent(s, h->ev_join, 0));
   }
-  pp.tm_codes = h->tm_pf_gu;
-  pp.tm_act = h->tm_pf_xg;
-  pp.scales = h->w.gu_scales;
-  pp.tscale = h->w.gu_tscale;
-  FLINT_TRY(launch_prefill_routed(pp, fmt, kPhaseGateUp, h->n_sm, false, s));
-  FLINT_TRY(m.mark());
-  pp.tm_codes = h->tm_pf_dn;
-  pp.tm_act = h->tm_pf_hq;
-  pp.scales = h->w.dn_scales;
-  pp.tscale = h->w.dn_tscale;
-  FLINT_TRY(launch_prefill_routed(pp, fmt, kPhaseDown, h->n_sm, pdl, s));
-  FLINT_TRY(m.mark());
+  if (h->w4a4) {
+    pp.tm_codes = h->tm_w4_gu;
+    pp.tm_sc = h->tm_w4_gu_sc;
+    pp.tm_act = h->tm_w4_xa;
+    pp.tm_act_sc = h->tm_w4_xa_sc;
+    pp.act_ts = h->xa_ts;
+    pp.tscale = h->w.gu_tscale;
+    pp.h32 = h->h32;
+    FLINT_TRY(launch_w4a4_routed(pp, kPhaseGateUp, h->n_sm, false, s));
+    FLINT_TRY(m.mark());
+    FLINT_TRY(launch_act_quant_h(h->h32, T * K, h->ha, h->ha_sf, h->ha_ts, pdl, s));
+    FLINT_TRY(m.mark());
+    pp.tm_codes = h->tm_w4_dn;
+    pp.tm_sc = h->tm_w4_dn_sc;
+    pp.tm_act = h->tm_w4_ha;
+    pp.tm_act_sc = h->tm_w4_ha_sc;
+    pp.act_ts = h->ha_ts;
+    pp.tscale = h->w.dn_tscale;
+    FLINT_TRY(launch_w4a4_routed(pp, kPhaseDown, h->n_sm, pdl, s));
+    FLINT_TRY(m.mark());
+  } else {
+    pp.tm_codes = h->tm_pf_gu;
+    pp.tm_act = h->tm_pf_xg;
+    pp.scales = h->w.gu_scales;
+    pp.tscale = h->w.gu_tscale;
+    FLINT_TRY(launch_prefill_routed(pp, fmt, kPhaseGateUp, h->n_sm, false, s));
+    FLINT_TRY(m.mark());
+    pp.tm_codes = h->tm_pf_dn;
+    pp.tm_act = h->tm_pf_hq;
+    pp.scales = h->w.dn_scales;
+    pp.tscale = h->w.dn_tscale;
+    FLINT_TRY(launch_prefill_routed(pp, fmt, kPhaseDown, h->n_sm, pdl, s));
+    FLINT_TRY(m.mark());
+  }
   if (!fork) {
     pp.tm_a = h->tm_pf_sh_dn;
     pp.tm_b = h->tm_pf_hs_hi;
@@ -428,6 +495,7 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
   h->ws_bytes = workspace_bytes;
   plan(h, *cfg, h->ws);
   h->last_T = 0;
+  h->w4a4 = (cfg->flags & FLINT_FLAG_W4A4) != 0;
   const int n_wrows = cfg->n_slots > 0 ? cfg->n_slots : cfg->n_experts;   // experts (or slots) of the routed arrays
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -450,6 +518,18 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
       !create_side_stream(h)) {
     delete h;
     return FLINT_ERR_CUDA;
+  }
+  if (h->w4a4) {
+    const uint64_t P = static_cast<uint64_t>(cfg->t_max) * cfg->top_k;
+    if (!encode_fp4_tiles(&h->tm_w4_gu, w.gu_codes, static_cast<uint64_t>(n_wrows) * 2 * kI, kH / 2, 128) ||
+        !encode_sf_tiles(&h->tm_w4_gu_sc, w.gu_scales, static_cast<uint64_t>(n_wrows) * 2 * kI, kH / 16, 128) ||
+        !encode_fp4_tiles(&h->tm_w4_dn, w.dn_codes, static_cast<uint64_t>(n_wrows) * kH, kI / 2, 128) ||
+        !encode_sf_tiles(&h->tm_w4_dn_sc, w.dn_scales, static_cast<uint64_t>(n_wrows) * kH, kI / 16, 128) ||
+        !encode_fp4_tiles(&h->tm_w4_xa, h->xa, P, kH / 2, 16) || !encode_sf_tiles(&h->tm_w4_xa_sc, h->xa_sf, P, kH / 16, 16) ||
+        !encode_fp4_tiles(&h->tm_w4_ha, h->ha, P, kI / 2, 16) || !encode_sf_tiles(&h->tm_w4_ha_sc, h->ha_sf, P, kI / 16, 16)) {
+      delete h;
+      return FLINT_ERR_CUDA;
+    }
   }
   // the decode kernel keeps every CTA resident (one per SM) and gives each at most 16 rows of y
   int per_sm = 0;
@@ -564,6 +644,16 @@ flint_status flint_moe_intermediate(flint_moe_t h, int which, void* dst, size_t 
       }
       break;
     case FLINT_BUF_YS: src = h->ys; have = T * kH * 4; break;
+    case FLINT_BUF_XA: case FLINT_BUF_XA_SF: case FLINT_BUF_XA_TS: case FLINT_BUF_H:
+    case FLINT_BUF_HA: case FLINT_BUF_HA_SF: case FLINT_BUF_HA_TS: case FLINT_BUF_O: {
+      if (!h->w4a4 || T <= kDecodeMaxT) return FLINT_ERR_INVALID_ARG;
+      const size_t P = T * h->cfg.top_k;
+      const void* const srcs[] = {h->xa, h->xa_sf, h->xa_ts, h->h32, h->ha, h->ha_sf, h->ha_ts, h->o};
+      const size_t sizes[] = {P * kH / 2, P * kH / 16, P * 4, P * kI * 4, P * kI / 2, P * kI / 16, P * 4, P * kH * 2};
+      src = srcs[which - FLINT_BUF_XA];
+      have = sizes[which - FLINT_BUF_XA];
+      break;
+    }
     default: return FLINT_ERR_INVALID_ARG;
   }
   if (bytes > have) return FLINT_ERR_INVALID_ARG;

@@ -23,6 +23,13 @@ def _to_device(a, device):
     return torch.from_numpy(a).to(device)
 
 
+# W4A4 intermediates (permuted rows): columns per row (0: one value per row) and dtype
+_W4A4_BUFS = {B.FLINT_BUF_XA: (H // 2, torch.uint8), B.FLINT_BUF_XA_SF: (H // 16, torch.uint8),
+              B.FLINT_BUF_XA_TS: (0, torch.float32), B.FLINT_BUF_H: (I, torch.float32),
+              B.FLINT_BUF_HA: (I // 2, torch.uint8), B.FLINT_BUF_HA_SF: (I // 16, torch.uint8),
+              B.FLINT_BUF_HA_TS: (0, torch.float32), B.FLINT_BUF_O: (H, torch.float16)}
+
+
 class FlintMoELayer:
     """One Flint MoE layer resident on a CUDA device.
 
@@ -120,6 +127,10 @@ class FlintMoELayer:
             t = torch.empty((T, H), dtype=torch.float16, device=self.device)
         elif which == B.FLINT_BUF_YS:
             t = torch.empty((T, H), dtype=torch.float32, device=self.device)
+        elif which in _W4A4_BUFS:
+            P = T * self.top_k
+            cols, dtype = _W4A4_BUFS[which]
+            t = torch.empty((P, cols) if cols else (P,), dtype=dtype, device=self.device)
         else:
             raise ValueError(which)
         s = torch.cuda.current_stream(self.device).cuda_stream

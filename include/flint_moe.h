@@ -58,6 +58,14 @@ typedef enum flint_wformat {
 
 /* cfg.flags */
 #define FLINT_FLAG_DEBUG_CHECKS 0x1u  /* device-side range checks on ids / offsets; sets the error word */
+/* W4A4 prefill (FLINT_W_NVFP4 only; forwards with T > 8): the routed experts' inputs, x and the
+ * SwiGLU output h, are quantised to NVFP4 per row before each projection, and the projections run
+ * as block-scaled FP4 MMAs (kekzle/Flint-NVFP4, evaluation table and serving notes: imp quantises
+ * activations in prefill). Per row: a tensor scale amax / (6 * 448) (1 for an all-zero row), an E4M3
+ * scale per 16 values (nearest, ties to even, saturating), E2M1 codes (nearest, ties to even), each
+ * quotient and product rounded to fp32 in that order. Decode (T <= 8) keeps 16-bit activations.
+ * Adds ~1.3 KB per permuted row (t_max * top_k rows) to the workspace. */
+#define FLINT_FLAG_W4A4 0x2u
 
 typedef struct flint_moe_cfg {
   int hidden;         /* H: 2048 (the only width this build has kernels for) */
@@ -197,7 +205,16 @@ enum {
                              8-element block stored in the order 0,4,1,5,2,6,3,7 for int4; [T][H]
                              after a forward with T <= 8, [T*top_k][H] in permuted row order (row p
                              holds token perm[p] / top_k) after a larger one */
-  FLINT_BUF_YS = 2        /* f32 [T][H] shared-expert output */
+  FLINT_BUF_YS = 2,       /* f32 [T][H] shared-expert output */
+  /* W4A4 prefill only (FLINT_FLAG_W4A4, T > 8), permuted row order, P = T * top_k rows: */
+  FLINT_BUF_XA = 3,       /* u8 [P][H/2] NVFP4 codes of x (low nibble = even column) */
+  FLINT_BUF_XA_SF = 4,    /* u8 [P][H/16] their E4M3 block scales */
+  FLINT_BUF_XA_TS = 5,    /* f32 [P] their tensor scales */
+  FLINT_BUF_H = 6,        /* f32 [P][I] SwiGLU output h */
+  FLINT_BUF_HA = 7,       /* u8 [P][I/2] NVFP4 codes of h */
+  FLINT_BUF_HA_SF = 8,    /* u8 [P][I/16] */
+  FLINT_BUF_HA_TS = 9,    /* f32 [P] */
+  FLINT_BUF_O = 10        /* fp16 [P][H] routed expert outputs before weighting */
 };
 flint_status flint_moe_intermediate(flint_moe_t h, int which, void* dst, size_t bytes, void* stream);
 
