@@ -135,22 +135,31 @@ struct PfTile {
 };
 
 // Warp 0: tiles of expert e are rp-major over its chunks; experts in ascending order (an expert
-// without rows has none).
+// without rows has none). Every lane loads the offsets (and weight slots) of all its experts before
+// the scans, so the table costs one global-load latency rather than one per 32 experts.
 __device__ void build_tiles(TileTab& tt, const PrefillParams& p, int rp_count) {
+  constexpr int kPer = kMaxE / 32;
   const int lane = threadIdx.x & 31;
   const int n = min(p.E, kMaxE);
+  int off[kPer], end[kPer], slot[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = 32 * j + lane;
+    off[j] = i < n ? __ldg(p.offsets + i) : 0;
+    end[j] = i < n ? __ldg(p.offsets + i + 1) : 0;
+    slot[j] = (i < n && p.slot_of) ? __ldg(p.slot_of + i) : i;
+  }
   int base = 0;
-  for (int i0 = 0; i0 < n; i0 += 32) {
-    const int i = i0 + lane;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = 32 * j + lane;
     int tiles = 0;
     if (i < n) {
-      const int e = i;
-      const int off = p.offsets[e];
-      const int c = max(p.offsets[e + 1] - off, 0);
+      const int c = max(end[j] - off[j], 0);
       const int nch = (c + kPfN - 1) / kPfN;
-      tt.e[i] = e;
-      tt.w[i] = (p.slot_of && c > 0) ? min(max(p.slot_of[e], 0), p.n_wslots - 1) : e;
-      tt.off[i] = off;
+      tt.e[i] = i;
+      tt.w[i] = (p.slot_of && c > 0) ? min(max(slot[j], 0), p.n_wslots - 1) : i;
+      tt.off[i] = off[j];
       tt.cnt[i] = c;
       tt.nch[i] = nch;
       tiles = rp_count * nch;

@@ -18,9 +18,14 @@
 //               and their raw block scales (128 rows x 16 bytes) per stage
 //   warp 3      TMA: the chunk's activation codes (16-row boxes, 128-byte swizzle) and raw scales;
 //               after griddepcontrol.wait, as they are the previous kernel's output
-//   warp 2      scale layout: rewrites the raw scales of a stage into the MMA's scale layout (below)
-//   warp 1      TMEM allocation, tcgen05.cp of the stage's scales into tensor memory and MMA issue
-//   warps 4..7  epilogue, one per 32-lane quarter of tensor memory
+//   warps 2, 13 scale layout: rewrite the raw scales of a stage into the MMA's scale layout (below);
+//               warp 2 those of weight block 0 and of the activations, warp 13 those of block 1
+//   warps 1, 12 MMA issue, one warp per weight block: tcgen05.cp of the block's and the activations'
+//               scales into its own tensor-memory columns, then the block's MMAs; warp 1 also owns
+//               the tensor-memory allocation
+//   warps 4..11 epilogue, two per 32-lane quarter of tensor memory (warp w reads lanes 32 (w % 4)..),
+//               warps 4..7 the even 16-column groups of a tile, warps 8..11 the odd ones (a down
+//               tile has only two stages to hide its epilogue behind)
 //
 // Scale layout of one MMA (K = 64, four 16-blocks): a row m = m0 + 32 m1 of the operand (m0 < 32,
 // m1 < 4) has its four E4M3 scales as bytes 0..3 of tensor-memory column m1 in lane m0 (copied to
@@ -157,17 +162,19 @@ constexpr int kW4OffBar = (kW4OffTab + static_cast<int>(sizeof(TileTab)) + 7) / 
 
 struct W4Bars {
   uint64_t full_a[kW4D], full_b[kW4D], sf_ready[kW4D], empty[kW4D];
-  uint64_t acc_full[2], acc_empty[2], done;
+  uint64_t acc_full[2], acc_empty[2], done[2];
   uint32_t tmem;
   int abort;
 };
 constexpr int kW4Smem = kW4OffBar + static_cast<int>(sizeof(W4Bars)) + 1024;
 static_assert(kW4Smem <= 227 * 1024, "shared memory per CTA");
 
-// tensor memory: accumulators [slot 2][block 2] x 64 columns, then per ring slot 48 scale columns
-// (block 0: 4 K-steps x 4, block 1, activations)
+// tensor memory: accumulators [slot 2][block 2] x 64 columns, then per ring slot 64 scale columns:
+// per weight block (the MMA warp that issues it) 16 of the block's scales (4 K-steps x 4) and 16 of
+// the activations'
+constexpr int kW4Threads = 448;
 constexpr uint32_t kW4ColSf = 256;
-constexpr uint32_t kW4SfSlot = 48;
+constexpr uint32_t kW4SfSlot = 64;
 static_assert(kW4ColSf + kW4D * kW4SfSlot <= 512, "tensor-memory columns");
 
 template <int PHASE>
@@ -217,7 +224,7 @@ __device__ __forceinline__ void tc_mma_fp4_w(uint32_t d, uint64_t adesc, uint64_
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 template <int PHASE>
-__global__ void __launch_bounds__(256, 1) w4a4_kernel(const __grid_constant__ PrefillParams p) {
+__global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_constant__ PrefillParams p) {
   using G = W4Geom<PHASE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
@@ -230,14 +237,15 @@ __global__ void __launch_bounds__(256, 1) w4a4_kernel(const __grid_constant__ Pr
     for (int i = 0; i < kW4D; ++i) {
       mbar_init(&bb.full_a[i], 1);
       mbar_init(&bb.full_b[i], 1);
-      mbar_init(&bb.sf_ready[i], 1);
-      mbar_init(&bb.empty[i], 1);
+      mbar_init(&bb.sf_ready[i], 2);
+      mbar_init(&bb.empty[i], 2);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&bb.acc_full[a], 1);
-      mbar_init(&bb.acc_empty[a], 4);
+      mbar_init(&bb.acc_full[a], 2);
+      mbar_init(&bb.acc_empty[a], 8);
     }
-    mbar_init(&bb.done, 1);
+    mbar_init(&bb.done[0], 1);
+    mbar_init(&bb.done[1], 1);
     bb.abort = 0;
     fence_mbar_init();
   }
@@ -299,8 +307,9 @@ __global__ void __launch_bounds__(256, 1) w4a4_kernel(const __grid_constant__ Pr
       }
       for (int j = max(it - kW4D, 0); j < it; ++j) pf_wait(&bb.full_b[j % kW4D], (j / kW4D) & 1, abort, p.err);
     }
-  } else if (warp == 2) {
-    // ---- raw scales -> MMA scale atoms (lane = m0)
+  } else if (warp == 2 || warp == 13) {
+    // ---- raw scales -> MMA scale atoms (lane = m0); warp 2: block 0 and activations, warp 13: block 1
+    const int b_lo = warp == 2 ? 0 : 1;
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       bool ok = true;
@@ -313,7 +322,9 @@ __global__ void __launch_bounds__(256, 1) w4a4_kernel(const __grid_constant__ Pr
         }
         uint8_t* st = sm + slot * kW4Stage;
 #pragma unroll
-        for (int b = 0; b < 3; ++b) {           // weight block 0, weight block 1, activations
+        for (int bi = 0; bi < 2; ++bi) {        // (weight block 0, activations) or weight block 1
+          const int b = bi == 0 ? b_lo : 2;
+          if (b_lo == 1 && bi == 1) break;
           const uint8_t* raw = b < 2 ? st + kW4OffRawA + b * kW4RawA : st + kW4OffRawB;
           const int nm1 = b < 2 ? 4 : kW4BRows / 32;
           uint4 r[4];
@@ -332,8 +343,9 @@ __global__ void __launch_bounds__(256, 1) w4a4_kernel(const __grid_constant__ Pr
       }
       if (!ok) break;
     }
-  } else if (warp == 1) {
-    // ---- scale copies and MMA issue (uniform control flow; an elected lane issues)
+  } else if (warp == 1 || warp == 12) {
+    // ---- scale copies and MMA issue for one weight block (uniform control flow; an elected lane issues)
+    const int b = warp == 1 ? 0 : 1;
     int it = 0, ti = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++ti) {
@@ -342,6 +354,7 @@ __global__ void __launch_bounds__(256, 1) w4a4_kernel(const __grid_constant__ Pr
       const int as = ti & 1;
       if (ti >= 2 && !pf_wait_all(&bb.acc_empty[as], ((ti >> 1) - 1) & 1, abort, p.err)) break;
       tc_fence_after();
+      const uint32_t d = tmem + as * 128 + b * 64;
       for (int s = 0; s < G::S; ++s, ++it) {
         const int slot = it % kW4D;
         if (!pf_wait_all(&bb.sf_ready[slot], (it / kW4D) & 1, abort, p.err) ||
@@ -352,54 +365,54 @@ __global__ void __launch_bounds__(256, 1) w4a4_kernel(const __grid_constant__ Pr
         }
         tc_fence_after();
         const uint32_t st = smem_u32(sm + slot * kW4Stage);
-        const uint32_t sf = tmem + kW4ColSf + slot * kW4SfSlot;
+        const uint32_t sfa = tmem + kW4ColSf + slot * kW4SfSlot + b * 32, sfb = sfa + 16;
 #pragma unroll
-        for (int b = 0; b < 3; ++b)
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tc_cp_atom_w(sf + b * 16 + j * 4, sdesc_atom(st + kW4OffAtom + (b * 4 + j) * kW4Atom));
+        for (int j = 0; j < 4; ++j) {
+          tc_cp_atom_w(sfa + j * 4, sdesc_atom(st + kW4OffAtom + (b * 4 + j) * kW4Atom));
+          tc_cp_atom_w(sfb + j * 4, sdesc_atom(st + kW4OffAtom + (2 * 4 + j) * kW4Atom));
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int b = 0; b < 2; ++b)
-            tc_mma_fp4_w(tmem + as * 128 + b * 64, sdesc_sw128(st + kW4OffA + b * kW4ABox + j * 32),
-                         sdesc_sw128(st + kW4OffB + j * 32), idesc, sf + b * 16 + j * 4, sf + 32 + j * 4,
-                         (s | j) ? 1u : 0u);
+          tc_mma_fp4_w(d, sdesc_sw128(st + kW4OffA + b * kW4ABox + j * 32), sdesc_sw128(st + kW4OffB + j * 32),
+                       idesc, sfa + j * 4, sfb + j * 4, (s | j) ? 1u : 0u);
         tc_commit_w(&bb.empty[slot]);
       }
       if (ok) tc_commit_w(&bb.acc_full[as]);
     }
-    tc_commit_w(&bb.done);                         // every MMA and copy of this warp has completed
-    pf_wait_all(&bb.done, 0, abort, p.err);
-  } else {
-    // ---- epilogue: lane quarter q holds weight rows 32q.. of both blocks
-    const int q = warp & 3, r = 32 * q + lane;
+    tc_commit_w(&bb.done[b]);                      // every MMA and copy of this warp has completed
+    pf_wait_all(&bb.done[b], 0, abort, p.err);
+  } else if (warp >= 4 && warp < 12) {
+    // ---- epilogue: lane quarter q holds weight rows 32q.. of both blocks; set k the 16-column
+    // groups 2i + k
+    const int q = warp & 3, r = 32 * q + lane, k = (warp - 4) >> 2;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    pdl_wait();                                    // the activation tensor scales are the previous kernel's output
     int ti = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++ti) {
       const PfTile tl = tile_at(tt, t);
       const int as = ti & 1;
+      // the tile's scales are loaded before the wait for its accumulators: the weight tensor scales
+      // and one activation tensor scale per column (column c in lane c % 32 of ts_lo / ts_hi)
+      float tw0, tw1;
+      if constexpr (PHASE == kPhaseGateUp) {
+        tw0 = __ldg(p.tscale + 2 * tl.w);
+        tw1 = __ldg(p.tscale + 2 * tl.w + 1);
+      } else {
+        tw0 = tw1 = __ldg(p.tscale + tl.w);
+      }
+      const float ts_lo = lane < tl.n ? __ldg(p.act_ts + tl.row0 + lane) : 0.f;
+      const float ts_hi = lane + 32 < tl.n ? __ldg(p.act_ts + tl.row0 + 32 + lane) : 0.f;
       if (!pf_wait_all(&bb.acc_full[as], (ti >> 1) & 1, abort, p.err)) break;
       tc_fence_after();
       const uint32_t dbase = lane_base + as * 128;
-      float tw0, tw1;
-      if constexpr (PHASE == kPhaseGateUp) {
-        tw0 = p.tscale[2 * tl.w];
-        tw1 = p.tscale[2 * tl.w + 1];
-      } else {
-        tw0 = tw1 = p.tscale[tl.w];
-      }
-      for (int j0 = 0; j0 < tl.n; j0 += 16) {
+      for (int j0 = 16 * k; j0 < tl.n; j0 += 32) {
         uint32_t d0[16], d1[16];
         tc_ld16(dbase + j0, d0);
         tc_ld16(dbase + 64 + j0, d1);
-        // the activation rows' tensor scales, one per column (lanes c and c + 16 hold column c)
-        const int cl = j0 + (lane & 15);
-        const float tsa = cl < tl.n ? __ldg(p.act_ts + tl.row0 + cl) : 0.f;
         tc_wait_ld();
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float ta = __shfl_sync(kAll, tsa, c);
+          const float ta = __shfl_sync(kAll, j0 < 32 ? ts_lo : ts_hi, (j0 + c) & 31);
           if (j0 + c < tl.n) {
             const size_t row = static_cast<size_t>(tl.row0 + j0 + c);
             const float v0 = __uint_as_float(d0[c]) * (tw0 * ta), v1 = __uint_as_float(d1[c]) * (tw1 * ta);
@@ -477,8 +490,8 @@ cudaError_t launch_w4a4_routed(const PrefillParams& p, int phase, int n_sm, bool
       return e;
     smem_set = true;
   }
-  return phase == kPhaseGateUp ? launch_pdl(w4a4_kernel<kPhaseGateUp>, n_sm, 256, kW4Smem, pdl, s, p)
-                               : launch_pdl(w4a4_kernel<kPhaseDown>, n_sm, 256, kW4Smem, pdl, s, p);
+  return phase == kPhaseGateUp ? launch_pdl(w4a4_kernel<kPhaseGateUp>, n_sm, kW4Threads, kW4Smem, pdl, s, p)
+                               : launch_pdl(w4a4_kernel<kPhaseDown>, n_sm, kW4Threads, kW4Smem, pdl, s, p);
 }
 
 }  // namespace flint
