@@ -52,6 +52,11 @@ struct flint_moe_ctx {
   uint8_t* ha;                             // W4A4: h codes [P][I/2], scales [P][I/16], tensor scales [P]
   uint8_t* ha_sf;
   float* ha_ts;
+  int* rowc;                               // W4A4: chunk position (chunk * 64 + row in chunk) of each permuted row
+  uint8_t* xa_atoms;                       // W4A4: block scales of x and h as MMA atoms [chunk][K/64][512]
+  uint8_t* ha_atoms;
+  uint8_t* w_atoms_gu;                     // W4A4: weight block scales as MMA atoms [rows / 128][K/64][512]
+  uint8_t* w_atoms_dn;
   int last_T;
   bool w4a4;
   int n_sm;
@@ -62,9 +67,7 @@ struct flint_moe_ctx {
   CUtensorMap tm_pf_hs_hi, tm_pf_hs_lo;    // prefill: shared-expert hidden pair [t_max][Is]
   CUtensorMap tm_pf_xg, tm_pf_hq;          // prefill: routed activation rows (fp16, 64 x 16 boxes)
   CUtensorMap tm_w4_gu, tm_w4_dn;          // W4A4: weight codes as bytes, 128 x 128-row boxes, 128-byte swizzle
-  CUtensorMap tm_w4_gu_sc, tm_w4_dn_sc;    // W4A4: weight block scales, 16-byte x 128-row boxes
   CUtensorMap tm_w4_xa, tm_w4_ha;          // W4A4: activation codes, 128 x 16-row boxes, 128-byte swizzle
-  CUtensorMap tm_w4_xa_sc, tm_w4_ha_sc;    // W4A4: activation block scales, 16-byte x 16-row boxes
   // instrumentation (caller-owned cudaEvent_t handles)
   cudaEvent_t events[32];
   int n_events;
@@ -97,7 +100,7 @@ flint_status check_cfg(const flint_moe_cfg* c) {
   if (c->hidden != kH || c->inter != kI || c->inter_shared != kIs) return FLINT_ERR_UNSUPPORTED;
   if (c->n_experts % 32 != 0 || c->n_experts > kMaxE) return FLINT_ERR_UNSUPPORTED;
   if (c->n_slots < 0 || c->n_slots > c->n_experts) return FLINT_ERR_INVALID_ARG;
-  if ((c->flags & FLINT_FLAG_W4A4) && c->fmt != FLINT_W_NVFP4) return FLINT_ERR_UNSUPPORTED;
+  if ((c->flags & FLINT_FLAG_W4A4) && (c->fmt != FLINT_W_NVFP4 || c->n_slots > 0)) return FLINT_ERR_UNSUPPORTED;
   return FLINT_OK;
 }
 
@@ -151,14 +154,9 @@ bool encode_f16_rows16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
   return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rows, cols * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// W4A4 operands: bytes, box of 128 bytes x box_rows rows with the 128-byte swizzle (codes) or of
-// 16 bytes without swizzle (block scales)
+// W4A4 codes: bytes, box of 128 bytes x box_rows rows with the 128-byte swizzle
 bool encode_fp4_tiles(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
   return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, row_bytes, 128, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
-}
-
-bool encode_sf_tiles(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
-  return encode_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, row_bytes, 16, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 bool encode_code_tiles(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes) {
@@ -218,6 +216,13 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
   char* p_ha = take(PA * kI / 2);
   char* p_ha_sf = take(PA * kI / 16);
   char* p_ha_ts = take(PA * 4);
+  const size_t CA = PA ? w4a4_chunk_capacity(P, static_cast<int>(E)) : 0;
+  const size_t WR = PA ? static_cast<size_t>(c.n_experts) : 0;          // W4A4 handles take no cache slots
+  char* p_rowc = take(PA * 4);
+  char* p_xa_atoms = take(CA * (kH / 64) * 512);
+  char* p_ha_atoms = take(CA * (kI / 64) * 512);
+  char* p_w_atoms_gu = take(WR * (2 * kI / 128) * (kH / 64) * 512);
+  char* p_w_atoms_dn = take(WR * (kH / 128) * (kI / 64) * 512);
   if (h) {
     h->logits = reinterpret_cast<float*>(p_logits);
     h->logits_part = reinterpret_cast<float*>(p_lpart);
@@ -253,6 +258,11 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
     h->ha = reinterpret_cast<uint8_t*>(p_ha);
     h->ha_sf = reinterpret_cast<uint8_t*>(p_ha_sf);
     h->ha_ts = reinterpret_cast<float*>(p_ha_ts);
+    h->rowc = reinterpret_cast<int*>(p_rowc);
+    h->xa_atoms = reinterpret_cast<uint8_t*>(p_xa_atoms);
+    h->ha_atoms = reinterpret_cast<uint8_t*>(p_ha_atoms);
+    h->w_atoms_gu = reinterpret_cast<uint8_t*>(p_w_atoms_gu);
+    h->w_atoms_dn = reinterpret_cast<uint8_t*>(p_w_atoms_dn);
   }
   return off;
 }
@@ -398,7 +408,9 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   }
   FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, c.flags, h->err, rs));
   FLINT_TRY(m.mark());
-  if (h->w4a4) FLINT_TRY(launch_act_quant_x(x, T, K, h->inv, h->xa, h->xa_sf, h->xa_ts, rs));
+  if (h->w4a4)
+    FLINT_TRY(launch_act_quant_x(x, T, K, E, h->ids, h->inv, h->offsets, h->xa, h->xa_sf, h->xa_atoms, h->xa_ts, h->rowc,
+                                 rs));
   else FLINT_TRY(launch_xg(x, T, K, h->inv, fmt == kInt4 ? 1 : 0, h->xg, rs));
   FLINT_TRY(m.mark());
 
@@ -416,20 +428,20 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
   }
   if (h->w4a4) {
     pp.tm_codes = h->tm_w4_gu;
-    pp.tm_sc = h->tm_w4_gu_sc;
+    pp.w_atoms = h->w_atoms_gu;
     pp.tm_act = h->tm_w4_xa;
-    pp.tm_act_sc = h->tm_w4_xa_sc;
+    pp.act_atoms = h->xa_atoms;
     pp.act_ts = h->xa_ts;
     pp.tscale = h->w.gu_tscale;
     pp.h32 = h->h32;
     FLINT_TRY(launch_w4a4_routed(pp, kPhaseGateUp, h->n_sm, false, s));
     FLINT_TRY(m.mark());
-    FLINT_TRY(launch_act_quant_h(h->h32, T * K, h->ha, h->ha_sf, h->ha_ts, pdl, s));
+    FLINT_TRY(launch_act_quant_h(h->h32, T * K, h->rowc, h->ha, h->ha_sf, h->ha_atoms, h->ha_ts, pdl, s));
     FLINT_TRY(m.mark());
     pp.tm_codes = h->tm_w4_dn;
-    pp.tm_sc = h->tm_w4_dn_sc;
+    pp.w_atoms = h->w_atoms_dn;
     pp.tm_act = h->tm_w4_ha;
-    pp.tm_act_sc = h->tm_w4_ha_sc;
+    pp.act_atoms = h->ha_atoms;
     pp.act_ts = h->ha_ts;
     pp.tscale = h->w.dn_tscale;
     FLINT_TRY(launch_w4a4_routed(pp, kPhaseDown, h->n_sm, pdl, s));
@@ -522,11 +534,15 @@ flint_status flint_moe_create(const flint_moe_cfg* cfg, const flint_moe_weights*
   if (h->w4a4) {
     const uint64_t P = static_cast<uint64_t>(cfg->t_max) * cfg->top_k;
     if (!encode_fp4_tiles(&h->tm_w4_gu, w.gu_codes, static_cast<uint64_t>(n_wrows) * 2 * kI, kH / 2, 128) ||
-        !encode_sf_tiles(&h->tm_w4_gu_sc, w.gu_scales, static_cast<uint64_t>(n_wrows) * 2 * kI, kH / 16, 128) ||
         !encode_fp4_tiles(&h->tm_w4_dn, w.dn_codes, static_cast<uint64_t>(n_wrows) * kH, kI / 2, 128) ||
-        !encode_sf_tiles(&h->tm_w4_dn_sc, w.dn_scales, static_cast<uint64_t>(n_wrows) * kH, kI / 16, 128) ||
-        !encode_fp4_tiles(&h->tm_w4_xa, h->xa, P, kH / 2, 16) || !encode_sf_tiles(&h->tm_w4_xa_sc, h->xa_sf, P, kH / 16, 16) ||
-        !encode_fp4_tiles(&h->tm_w4_ha, h->ha, P, kI / 2, 16) || !encode_sf_tiles(&h->tm_w4_ha_sc, h->ha_sf, P, kI / 16, 16)) {
+        !encode_fp4_tiles(&h->tm_w4_xa, h->xa, P, kH / 2, 16) || !encode_fp4_tiles(&h->tm_w4_ha, h->ha, P, kI / 2, 16) ||
+        // the weight scales in the MMA's layout, once (the weights' own writes complete first)
+        cudaDeviceSynchronize() != cudaSuccess ||
+        launch_pack_sf_atoms(static_cast<const uint8_t*>(w.gu_scales), n_wrows * 2 * kI, kH, h->w_atoms_gu, 0) !=
+            cudaSuccess ||
+        launch_pack_sf_atoms(static_cast<const uint8_t*>(w.dn_scales), n_wrows * kH, kI, h->w_atoms_dn, 0) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(0) != cudaSuccess) {
       delete h;
       return FLINT_ERR_CUDA;
     }

@@ -81,8 +81,6 @@ struct PrefillParams {
   CUtensorMap tm_a;               // dense phases: bf16 weights (shared expert, router), box 64 x 128 rows, 128-byte swizzle
   CUtensorMap tm_b;               // shared: bf16 activations (x, or hs_hi), box 64 x 128 rows, 128-byte swizzle
   CUtensorMap tm_b2;              // shared down: hs_lo
-  CUtensorMap tm_sc;              // W4A4: weight block scales [rows][K/16] bytes, box 16 bytes x 128 rows
-  CUtensorMap tm_act_sc;          // W4A4: activation block scales [P][K/16] bytes, box 16 bytes x 16 rows
   int T, top_k, E;
   const int* slot_of;             // [E] weight slot of each expert (weights in cache slots), or null
   int n_wslots;                   // weight slots when slot_of is set
@@ -99,6 +97,8 @@ struct PrefillParams {
   unsigned* err;
   const float* act_ts;            // W4A4: activation rows' tensor scales [P]
   float* h32;                     // W4A4 gate|up output h [P][I] (fp32)
+  const uint8_t* w_atoms;         // W4A4: weight block scales as MMA atoms [rows / 128][K/64][512]
+  const uint8_t* act_atoms;       // W4A4: activation block scales as MMA atoms [chunk][K/64][512]
 };
 
 // pdl: launched as a programmatic dependent of the previous kernel in the stream (the routed down
@@ -109,13 +109,19 @@ cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, c
 // W4A4 (NVFP4 weights and activations). tm_codes: weight codes as bytes [rows][K/2], box 128 x 128
 // rows, 128-byte swizzle; tm_act: activation codes [P][K/2], box 128 x 16 rows, 128-byte swizzle.
 cudaError_t launch_w4a4_routed(const PrefillParams& p, int phase, int n_sm, bool pdl, cudaStream_t s);
-// x (bf16 [T][H]) -> NVFP4 codes [P][H/2], scales [P][H/16] and tensor scales [P], written to each
-// token's permuted rows inv[t][k]
-cudaError_t launch_act_quant_x(const uint16_t* x, int T, int K, const int* inv, uint8_t* codes, uint8_t* scales,
-                               float* ts, cudaStream_t s);
-// h (fp32 [P][I]) -> codes [P][I/2], scales [P][I/16], tensor scales [P]
-cudaError_t launch_act_quant_h(const float* h, int P, uint8_t* codes, uint8_t* scales, float* ts, bool pdl,
+// Chunks (64 permuted rows of one expert) the activation atom arrays must hold for P rows.
+size_t w4a4_chunk_capacity(size_t P, int E);
+// Weight block scales [rows][K/16] -> MMA atoms [rows / 128][K/64][512 bytes] (rows % 128 == 0).
+cudaError_t launch_pack_sf_atoms(const uint8_t* scales, int rows, int K, uint8_t* atoms, cudaStream_t s);
+// x (bf16 [T][H]) -> NVFP4 codes [P][H/2], scales [P][H/16], tensor scales [P] and scale atoms
+// [chunk][H/64][512], written to each token's permuted rows inv[t][k]; rowc[p] = the row's chunk *
+// 64 + its row in the chunk
+cudaError_t launch_act_quant_x(const uint16_t* x, int T, int K, int E, const int* ids, const int* inv,
+                               const int* offsets, uint8_t* codes, uint8_t* scales, uint8_t* atoms, float* ts, int* rowc,
                                cudaStream_t s);
+// h (fp32 [P][I]) -> codes [P][I/2], scales [P][I/16], tensor scales [P], atoms [chunk][I/64][512]
+cudaError_t launch_act_quant_h(const float* h, int P, const int* rowc, uint8_t* codes, uint8_t* scales, uint8_t* atoms,
+                               float* ts, bool pdl, cudaStream_t s);
 
 // Residual stream of a layer stack: x (f32 [T][H]) += y (bf16, when not null); then, when z is not
 // null, z = bf16(rmsnorm(x)) with eps.

@@ -128,10 +128,12 @@ struct TileTab {
   int off[kMaxE];         // first permuted row
   int cnt[kMaxE];         // permuted rows
   int nch[kMaxE];         // chunks of kPfN rows
+  int cbase[kMaxE];       // index of expert i's first chunk among all experts' chunks (ascending expert)
 };
 
 struct PfTile {
   int e, w, row0, n, rp;  // expert, its weight index, first permuted row of the chunk, rows in it (1..kPfN), block pair
+  int c;                  // chunk index (cbase of the expert + chunk)
 };
 
 // Warp 0: tiles of expert e are rp-major over its chunks; experts in ascending order (an expert
@@ -149,11 +151,11 @@ __device__ void build_tiles(TileTab& tt, const PrefillParams& p, int rp_count) {
     end[j] = i < n ? __ldg(p.offsets + i + 1) : 0;
     slot[j] = (i < n && p.slot_of) ? __ldg(p.slot_of + i) : i;
   }
-  int base = 0;
+  int base = 0, cb = 0;
 #pragma unroll
   for (int j = 0; j < kPer; ++j) {
     const int i = 32 * j + lane;
-    int tiles = 0;
+    int tiles = 0, nchunks = 0;
     if (i < n) {
       const int c = max(end[j] - off[j], 0);
       const int nch = (c + kPfN - 1) / kPfN;
@@ -163,15 +165,23 @@ __device__ void build_tiles(TileTab& tt, const PrefillParams& p, int rp_count) {
       tt.cnt[i] = c;
       tt.nch[i] = nch;
       tiles = rp_count * nch;
+      nchunks = nch;
     }
-    int v = tiles;
+    int v = tiles, vc = nchunks;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
-      const int u = __shfl_up_sync(kAll, v, d);
-      if (lane >= d) v += u;
+      const int u = __shfl_up_sync(kAll, v, d), uc = __shfl_up_sync(kAll, vc, d);
+      if (lane >= d) {
+        v += u;
+        vc += uc;
+      }
     }
-    if (i < n) tt.start[i] = base + v - tiles;
+    if (i < n) {
+      tt.start[i] = base + v - tiles;
+      tt.cbase[i] = cb + vc - nchunks;
+    }
     base += __shfl_sync(kAll, v, 31);
+    cb += __shfl_sync(kAll, vc, 31);
   }
   if (lane == 0) {
     tt.n = n;
@@ -195,6 +205,7 @@ __device__ __forceinline__ PfTile tile_at(const TileTab& tt, int t) {
   r.row0 = tt.off[lo] + ch * kPfN;
   r.n = min(kPfN, tt.cnt[lo] - ch * kPfN);
   r.rp = rp;
+  r.c = tt.cbase[lo] + ch;
   return r;
 }
 

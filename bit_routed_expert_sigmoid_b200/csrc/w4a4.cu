@@ -3,37 +3,42 @@
 // kekzle/Flint-NVFP4, evaluation table and serving notes: in prefill the activations entering each
 // routed projection are quantised to NVFP4 as well, and the projections run on the FP4 tensor cores.
 // Here that is:
-//   act_quant_kernel   a row (a token's x, scattered to its top-k permuted rows; or a permuted row of
-//                      the SwiGLU output h) -> E2M1 codes, one E4M3 scale per 16 values and one fp32
-//                      scale per row (amax / (6 x 448)); every decision in IEEE fp32, in the order
-//                      ts, block scale, quotient, code
-//   w4a4_kernel        routed grouped GEMM on tcgen05.mma kind::mxf4nvf4 (block16: E2M1 operands from
-//                      shared memory, E4M3 scales from tensor memory, fp32 accumulators in tensor
-//                      memory); epilogue x (weight scale x activation scale); gate|up -> h = silu(g) u
-//                      in fp32, down -> o in fp16 (combined per token by the prefill combine kernel)
+//   act_quant_*_kernel  a row (a token's x, written to its top-k permuted rows; or a permuted row of
+//                       the SwiGLU output h) -> E2M1 codes, one E4M3 scale per 16 values and one fp32
+//                       scale per row (amax / (6 x 448)); every decision in IEEE fp32, in the order
+//                       ts, block scale, quotient, code
+//   w4a4_kernel         routed grouped GEMM on tcgen05.mma kind::mxf4nvf4 (block16: E2M1 operands
+//                       from shared memory, E4M3 scales from tensor memory, fp32 accumulators in
+//                       tensor memory); epilogue x (weight scale x activation scale); gate|up ->
+//                       h = silu(g) u in fp32, down -> o in fp16 (combined per token by the prefill
+//                       combine kernel)
 //
-// The routed GEMM uses the tile table of the W4A16 routed kernel: a tile is (expert, a chunk of up
+// Scale layout of one MMA (K = 64, four 16-blocks): row m = m0 + 32 m1 of an operand (m0 < 32,
+// m1 < 4) has its four E4M3 scales as bytes 0..3 of tensor-memory column m1 in lane m0, copied to
+// all four lane quarters by tcgen05.cp .32x128b.warpx4 from a 512-byte "atom" whose 16-byte row m0
+// holds [m1][block]. The scales are stored in that layout ahead of the GEMM, so a stage (four
+// K-steps) of a 128-row weight block or of a 64-row activation chunk is one contiguous 2 KB copy:
+//   weights      [row block of 128][K/64][atom], packed once when the handle is made
+//                (pack_sf_atoms_kernel) from the [row][K/16] scales
+//   activations  [chunk][K/64][atom], written by the quantisers; a chunk is 64 consecutive permuted
+//                rows of one expert (the GEMM's N), numbered over all experts in ascending order,
+//                and only m1 = 0, 1 of its atoms are meaningful
+//
+// The routed GEMM walks the tile table of the W4A16 routed kernel: a tile is (expert, a chunk of up
 // to 64 of its permuted rows, a pair of 128-row weight blocks). One persistent CTA per SM; warps:
 //   warp 0      TMA: the pair of weight-code blocks (128 rows x 128 bytes = 256 K, 128-byte swizzle)
-//               and their raw block scales (128 rows x 16 bytes) per stage
-//   warp 3      TMA: the chunk's activation codes (16-row boxes, 128-byte swizzle) and raw scales;
+//               and a bulk copy of each block's scale atoms, per stage
+//   warp 3      TMA: the chunk's activation codes (16-row boxes) and a bulk copy of its scale atoms;
 //               after griddepcontrol.wait, as they are the previous kernel's output
-//   warps 2, 13 scale layout: rewrite the raw scales of a stage into the MMA's scale layout (below);
-//               warp 2 those of weight block 0 and of the activations, warp 13 those of block 1
-//   warps 1, 12 MMA issue, one warp per weight block: tcgen05.cp of the block's and the activations'
-//               scales into its own tensor-memory columns, then the block's MMAs; warp 1 also owns
-//               the tensor-memory allocation
+//   warps 1, 2  MMA issue, one warp per weight block: tcgen05.cp of the block's and the chunk's
+//               atoms into the warp's own tensor-memory columns, then the block's four MMAs; warp 1
+//               also owns the tensor-memory allocation
 //   warps 4..11 epilogue, two per 32-lane quarter of tensor memory (warp w reads lanes 32 (w % 4)..),
-//               warps 4..7 the even 16-column groups of a tile, warps 8..11 the odd ones (a down
-//               tile has only two stages to hide its epilogue behind)
-//
-// Scale layout of one MMA (K = 64, four 16-blocks): a row m = m0 + 32 m1 of the operand (m0 < 32,
-// m1 < 4) has its four E4M3 scales as bytes 0..3 of tensor-memory column m1 in lane m0 (copied to
-// all four lane quarters by tcgen05.cp .32x128b.warpx4 from a 512-byte shared-memory atom whose row
-// m0 holds 16 bytes: m1-major, block-minor). The raw scales of a weight or activation row are
-// contiguous along K ([row][K/16] bytes), so the atom for K-step j takes the j-th 32-bit word of
-// rows m0, m0+32, m0+64 and m0+96.
+//               warps 4..7 the 16-column groups 0 and 2 of a tile, warps 8..11 groups 1 and 3; the
+//               accumulators are released as soon as they are in registers
 #include <cuda_fp8.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -43,8 +48,10 @@ namespace flint {
 
 namespace {
 
+constexpr int kAtom = 512;                         // bytes of one scale atom (one MMA K-step)
+
 // ---------------------------------------------------------------------------------------------
-// activation quantiser
+// activation quantisers
 
 __device__ __forceinline__ uint32_t f32_to_e4m3_satfinite(float q) {
   return static_cast<uint32_t>(__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3));
@@ -82,43 +89,33 @@ __device__ __forceinline__ uint32_t quant8(const float (&v)[8], float ts, uint32
   return w;
 }
 
-// Rows of K values, 8 values per thread (K / 8 threads per row), 256 threads per CTA.
-// SRC_BF16: rows are bf16 tokens, each written to its top_k permuted rows inv[t][k]; else rows are
-// fp32 permuted rows written in place.
-template <int K, bool SRC_BF16>
-__global__ void __launch_bounds__(256) act_quant_kernel(const void* __restrict__ src, int rows, int top_k,
-                                                        const int* __restrict__ inv, uint8_t* __restrict__ codes,
-                                                        uint8_t* __restrict__ scales, float* __restrict__ ts_out) {
-  constexpr int kTpr = K / 8;                    // threads per row
-  constexpr int kRows = 256 / kTpr;              // rows per CTA
-  constexpr int kWpr = (kTpr + 31) / 32;         // warps per row
-  static_assert(kTpr % 32 == 0 && kRows >= 1, "whole warps per row");
-  __shared__ float wmax[8];
-  const int lr = threadIdx.x / kTpr, i = threadIdx.x % kTpr;
-  const int row = blockIdx.x * kRows + lr;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if constexpr (!SRC_BF16) pdl_wait();           // h is the previous kernel's output
-  pdl_trigger();
-  float v[8];
-  if (row < rows) {
-    if constexpr (SRC_BF16) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(src) + static_cast<size_t>(row) * K) + i);
-      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        v[2 * j] = bf16lo_to_f32(u[j]);
-        v[2 * j + 1] = bf16hi_to_f32(u[j]);
-      }
-    } else {
-      const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(src) + static_cast<size_t>(row) * K) + 2 * i;
-      const float4 a = p[0], b = p[1];
-      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = 0.f;
+// The four block scales of a K-step (16-blocks held by lanes g, g + 2, g + 4, g + 6 of the 8-lane
+// group g) as one word, the first block in the low byte.
+__device__ __forceinline__ uint32_t kstep_scales(uint32_t sb, int lane) {
+  const int g = lane & ~7;
+  return __shfl_sync(kAll, sb, g) | (__shfl_sync(kAll, sb, g + 2) << 8) | (__shfl_sync(kAll, sb, g + 4) << 16) |
+         (__shfl_sync(kAll, sb, g + 6) << 24);
+}
+
+// One quantised row (thread i holds values 8i..8i+7 of K) to its destination: codes, raw scales,
+// tensor scale, and the scale atoms of its chunk position pos = chunk * 64 + row in chunk.
+template <int K>
+__device__ __forceinline__ void store_row(int i, int lane, size_t dst, int pos, uint32_t w, uint32_t sb, uint32_t step_sc,
+                                          float ts, uint8_t* codes, uint8_t* scales, uint8_t* atoms, float* ts_out) {
+  reinterpret_cast<uint32_t*>(codes + dst * (K / 2))[i] = w;
+  if ((i & 1) == 0) scales[dst * (K / 16) + (i >> 1)] = static_cast<uint8_t>(sb);
+  if ((lane & 7) == 0) {
+    const int c = pos >> 6, n = pos & 63, j = i >> 3;
+    *reinterpret_cast<uint32_t*>(atoms + (static_cast<size_t>(c) * (K / 64) + j) * kAtom + (n & 31) * 16 + (n >> 5) * 4) =
+        step_sc;
   }
+  if (i == 0) ts_out[dst] = ts;
+}
+
+// Row amax over the K / 8 threads of a row (whole warps), then the row's tensor scale.
+template <int K>
+__device__ __forceinline__ float row_tscale(const float (&v)[8], float* wmax, int lr, int warp, int lane) {
+  constexpr int kWpr = K / 8 / 32;
   float am = 0.f;
 #pragma unroll
   for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(v[j]));
@@ -128,16 +125,117 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const void* __restrict__
   __syncthreads();
 #pragma unroll
   for (int k = 0; k < kWpr; ++k) am = fmaxf(am, wmax[lr * kWpr + k]);
-  const float ts = am > 0.f ? __fdiv_rn(am, 2688.f) : 1.f;
+  return am > 0.f ? __fdiv_rn(am, 2688.f) : 1.f;
+}
+
+// x: one token per CTA (256 threads x 8 values). Warp 0 first numbers the chunks of all experts
+// (exclusive prefix of ceil(count / 64) over ascending expert ids, from the offsets) and places
+// each of the token's top-k permuted rows: its chunk position, also stored in rowc for the h
+// quantiser.
+__global__ void __launch_bounds__(256) act_quant_x_kernel(const uint16_t* __restrict__ x, int top_k, int E,
+                                                          const int* __restrict__ ids, const int* __restrict__ inv,
+                                                          const int* __restrict__ offsets, uint8_t* __restrict__ codes,
+                                                          uint8_t* __restrict__ scales, uint8_t* __restrict__ atoms,
+                                                          float* __restrict__ ts_out, int* __restrict__ rowc) {
+  static_assert(kH / 8 == 256, "one token per 256 threads");
+  constexpr int kPer = kMaxE / 32;
+  __shared__ float wmax[8];
+  __shared__ int cb[kMaxE];
+  __shared__ int dst_row[kMaxTopK], dst_pos[kMaxTopK];
+  const int t = blockIdx.x, i = threadIdx.x, warp = i >> 5, lane = i & 31;
+  if (warp == 0) {
+    int nch[kPer], sum = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int e = kPer * lane + j;
+      nch[j] = e < E ? (__ldg(offsets + e + 1) - __ldg(offsets + e) + 63) >> 6 : 0;
+      sum += nch[j];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int u = __shfl_up_sync(kAll, incl, d);
+      if (lane >= d) incl += u;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      cb[kPer * lane + j] = run;
+      run += nch[j];
+    }
+    __syncwarp();
+    if (lane < top_k) {
+      const int e = min(max(__ldg(ids + t * top_k + lane), 0), E - 1);
+      const int p = __ldg(inv + t * top_k + lane);
+      const int local = p - __ldg(offsets + e);
+      const int pos = (cb[e] + (local >> 6)) * 64 + (local & 63);
+      dst_row[lane] = p;
+      dst_pos[lane] = pos;
+      rowc[p] = pos;
+    }
+  }
+  float v[8];
+  const uint4 wx = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * kH) + i);
+  const uint32_t u[4] = {wx.x, wx.y, wx.z, wx.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    v[2 * j] = bf16lo_to_f32(u[j]);
+    v[2 * j + 1] = bf16hi_to_f32(u[j]);
+  }
+  const float ts = row_tscale<kH>(v, wmax, 0, warp, lane);     // its __syncthreads also publishes dst_*
   uint32_t sb;
   const uint32_t w = quant8(v, ts, sb);
-  if (row >= rows) return;
-  const int nd = SRC_BF16 ? top_k : 1;
-  for (int k = 0; k < nd; ++k) {
-    const size_t dst = SRC_BF16 ? static_cast<size_t>(__ldg(inv + static_cast<size_t>(row) * top_k + k)) : row;
-    reinterpret_cast<uint32_t*>(codes + dst * (K / 2))[i] = w;
-    if ((i & 1) == 0) scales[dst * (K / 16) + (i >> 1)] = static_cast<uint8_t>(sb);
-    if (i == 0) ts_out[dst] = ts;
+  const uint32_t step_sc = kstep_scales(sb, lane);
+  for (int k = 0; k < top_k; ++k)
+    store_row<kH>(i, lane, static_cast<size_t>(dst_row[k]), dst_pos[k], w, sb, step_sc, ts, codes, scales, atoms, ts_out);
+}
+
+// h: permuted rows of I values, 64 threads each, 4 per CTA; the chunk position of row p is rowc[p].
+__global__ void __launch_bounds__(256) act_quant_h_kernel(const float* __restrict__ h, int P, const int* __restrict__ rowc,
+                                                          uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                          uint8_t* __restrict__ atoms, float* __restrict__ ts_out) {
+  constexpr int kTpr = kI / 8, kRows = 256 / kTpr;
+  __shared__ float wmax[8];
+  const int lr = threadIdx.x / kTpr, i = threadIdx.x % kTpr;
+  const int row = blockIdx.x * kRows + lr;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();                                      // h is the previous kernel's output
+  pdl_trigger();
+  float v[8];
+  int pos = 0;
+  if (row < P) {
+    const float4* src = reinterpret_cast<const float4*>(h + static_cast<size_t>(row) * kI) + 2 * i;
+    const float4 a = src[0], b = src[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    pos = __ldg(rowc + row);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = 0.f;
+  }
+  const float ts = row_tscale<kI>(v, wmax, lr, warp, lane);
+  uint32_t sb;
+  const uint32_t w = quant8(v, ts, sb);
+  const uint32_t step_sc = kstep_scales(sb, lane);
+  if (row < P) store_row<kI>(i, lane, static_cast<size_t>(row), pos, w, sb, step_sc, ts, codes, scales, atoms, ts_out);
+}
+
+// Weight scales [rows][K/16] -> atoms [rows / 128][K/64][512 bytes]: one thread per (row block,
+// K-step, m0) writes the 16 bytes of rows m0, m0 + 32, m0 + 64, m0 + 96.
+__global__ void pack_sf_atoms_kernel(const uint8_t* __restrict__ sc, int rows, int K, uint8_t* __restrict__ out) {
+  const int steps = K / 64;
+  const size_t n = static_cast<size_t>(rows / 128) * steps * 32;
+  for (size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; idx < n;
+       idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int m0 = static_cast<int>(idx & 31);
+    const size_t q = idx >> 5;
+    const int j = static_cast<int>(q % steps);
+    const size_t rb = q / steps;
+    uint32_t wv[4];
+#pragma unroll
+    for (int m1 = 0; m1 < 4; ++m1)
+      wv[m1] = *reinterpret_cast<const uint32_t*>(sc + (rb * 128 + m0 + 32 * m1) * (K / 16) + 4 * j);
+    *reinterpret_cast<uint4*>(out + (rb * steps + j) * kAtom + m0 * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
   }
 }
 
@@ -147,21 +245,21 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const void* __restrict__
 constexpr int kW4D = 4;                            // ring depth (stages of 256 K)
 constexpr int kW4ABox = 128 * 128;                 // weight codes: 128 rows x 128 bytes
 constexpr int kW4BRows = kPfN;                     // activation rows per tile (MMA N, up to)
-constexpr int kW4RawA = 128 * 16;                  // raw weight scales of a block and stage
-constexpr int kW4RawB = kW4BRows * 16;
-constexpr int kW4Atom = 512;
+constexpr int kW4StepAtoms = 4 * kAtom;            // a stage's atoms of one operand block (2 KB)
 constexpr int kW4OffA = 0;
 constexpr int kW4OffB = kW4OffA + 2 * kW4ABox;
-constexpr int kW4OffRawA = kW4OffB + kW4BRows * 128;
-constexpr int kW4OffRawB = kW4OffRawA + 2 * kW4RawA;
-constexpr int kW4OffAtom = kW4OffRawB + kW4RawB;   // atoms: block 0 (K-steps 0..3), block 1, activations
-constexpr int kW4Stage = kW4OffAtom + 12 * kW4Atom;
+constexpr int kW4OffSfA = kW4OffB + kW4BRows * 128;  // atoms of weight blocks 0 and 1
+constexpr int kW4OffSfB = kW4OffSfA + 2 * kW4StepAtoms;
+constexpr int kW4Stage = kW4OffSfB + kW4StepAtoms;
 static_assert(kW4Stage % 1024 == 0 && kW4OffB % 1024 == 0, "128-byte swizzled operands on 1024-byte boundaries");
 constexpr int kW4OffTab = kW4D * kW4Stage;
-constexpr int kW4OffBar = (kW4OffTab + static_cast<int>(sizeof(TileTab)) + 7) / 8 * 8;
+// down epilogue: per epilogue warp a 16-token x 32-output fp16 slab, to turn its column-per-lane
+// results into 16-byte row stores
+constexpr int kW4OffSlab = (kW4OffTab + static_cast<int>(sizeof(TileTab)) + 15) / 16 * 16;
+constexpr int kW4OffBar = kW4OffSlab + 8 * 16 * 32 * 2;
 
 struct W4Bars {
-  uint64_t full_a[kW4D], full_b[kW4D], sf_ready[kW4D], empty[kW4D];
+  uint64_t full_a[kW4D], full_b[kW4D], empty[kW4D];
   uint64_t acc_full[2], acc_empty[2], done[2];
   uint32_t tmem;
   int abort;
@@ -169,10 +267,10 @@ struct W4Bars {
 constexpr int kW4Smem = kW4OffBar + static_cast<int>(sizeof(W4Bars)) + 1024;
 static_assert(kW4Smem <= 227 * 1024, "shared memory per CTA");
 
-// tensor memory: accumulators [slot 2][block 2] x 64 columns, then per ring slot 64 scale columns:
-// per weight block (the MMA warp that issues it) 16 of the block's scales (4 K-steps x 4) and 16 of
-// the activations'
-constexpr int kW4Threads = 448;
+// tensor memory: accumulators [slot 2][block 2] x 64 columns, then per ring slot and weight block
+// (the MMA warp that issues it) 16 columns of the block's scales (4 K-steps x 4) and 16 of the
+// chunk's
+constexpr int kW4Threads = 384;
 constexpr uint32_t kW4ColSf = 256;
 constexpr uint32_t kW4SfSlot = 64;
 static_assert(kW4ColSf + kW4D * kW4SfSlot <= 512, "tensor-memory columns");
@@ -181,12 +279,12 @@ template <int PHASE>
 struct W4Geom;
 template <>
 struct W4Geom<kPhaseGateUp> {
-  static constexpr int S = kH / 256, RP = kI / 128;
+  static constexpr int K = kH, S = kH / 256, RP = kI / 128;
   __device__ static int row(int w, int rp, int b) { return w * 2 * kI + b * kI + rp * 128; }
 };
 template <>
 struct W4Geom<kPhaseDown> {
-  static constexpr int S = kI / 256, RP = kH / 256;
+  static constexpr int K = kI, S = kI / 256, RP = kH / 256;
   __device__ static int row(int w, int rp, int b) { return w * kH + rp * 256 + b * 128; }
 };
 
@@ -221,11 +319,10 @@ __device__ __forceinline__ void tc_mma_fp4_w(uint32_t d, uint64_t adesc, uint64_
       : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
 template <int PHASE>
 __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_constant__ PrefillParams p) {
   using G = W4Geom<PHASE>;
+  constexpr int kSteps = G::K / 64;              // atoms per row block / chunk
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   TileTab& tt = *reinterpret_cast<TileTab*>(sm + kW4OffTab);
@@ -237,7 +334,6 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
     for (int i = 0; i < kW4D; ++i) {
       mbar_init(&bb.full_a[i], 1);
       mbar_init(&bb.full_b[i], 1);
-      mbar_init(&bb.sf_ready[i], 2);
       mbar_init(&bb.empty[i], 2);
     }
     for (int a = 0; a < 2; ++a) {
@@ -262,7 +358,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
   pdl_trigger();
 
   if (warp == 0) {
-    // ---- weight codes and raw scales
+    // ---- weight codes and scale atoms
     if (lane == 0) {
       int it = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
@@ -272,17 +368,19 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
           const int slot = it % kW4D;
           if (it >= kW4D && !pf_wait(&bb.empty[slot], ((it / kW4D) - 1) & 1, abort, p.err)) break;
           uint8_t* st = sm + slot * kW4Stage;
-          mbar_arrive_expect_tx(&bb.full_a[slot], 2 * kW4ABox + 2 * kW4RawA);
+          mbar_arrive_expect_tx(&bb.full_a[slot], 2 * kW4ABox + 2 * kW4StepAtoms);
           tma_2d(st + kW4OffA, &p.tm_codes, s * 128, r0, &bb.full_a[slot]);
           tma_2d(st + kW4OffA + kW4ABox, &p.tm_codes, s * 128, r1, &bb.full_a[slot]);
-          tma_2d(st + kW4OffRawA, &p.tm_sc, s * 16, r0, &bb.full_a[slot]);
-          tma_2d(st + kW4OffRawA + kW4RawA, &p.tm_sc, s * 16, r1, &bb.full_a[slot]);
+          bulk_g2s(st + kW4OffSfA, p.w_atoms + (static_cast<size_t>(r0 / 128) * kSteps + 4 * s) * kAtom, kW4StepAtoms,
+                   &bb.full_a[slot]);
+          bulk_g2s(st + kW4OffSfA + kW4StepAtoms, p.w_atoms + (static_cast<size_t>(r1 / 128) * kSteps + 4 * s) * kAtom,
+                   kW4StepAtoms, &bb.full_a[slot]);
         }
       }
       for (int j = max(it - kW4D, 0); j < it; ++j) pf_wait(&bb.full_a[j % kW4D], (j / kW4D) & 1, abort, p.err);
     }
   } else if (warp == 3) {
-    // ---- activation codes and raw scales: the chunk's rows rounded up to 16
+    // ---- activation codes (the chunk's rows rounded up to 16) and the chunk's scale atoms
     if (lane == 0) {
       pdl_wait();
       int it = 0;
@@ -297,55 +395,19 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
             break;
           }
           uint8_t* st = sm + slot * kW4Stage;
-          mbar_arrive_expect_tx(&bb.full_b[slot], nbox * (16 * 128 + 16 * 16));
-          for (int q = 0; q < nbox; ++q) {
+          mbar_arrive_expect_tx(&bb.full_b[slot], nbox * 16 * 128 + kW4StepAtoms);
+          for (int q = 0; q < nbox; ++q)
             tma_2d(st + kW4OffB + q * 2048, &p.tm_act, s * 128, tl.row0 + 16 * q, &bb.full_b[slot]);
-            tma_2d(st + kW4OffRawB + q * 256, &p.tm_act_sc, s * 16, tl.row0 + 16 * q, &bb.full_b[slot]);
-          }
+          bulk_g2s(st + kW4OffSfB, p.act_atoms + (static_cast<size_t>(tl.c) * kSteps + 4 * s) * kAtom, kW4StepAtoms,
+                   &bb.full_b[slot]);
         }
         if (!ok) break;
       }
       for (int j = max(it - kW4D, 0); j < it; ++j) pf_wait(&bb.full_b[j % kW4D], (j / kW4D) & 1, abort, p.err);
     }
-  } else if (warp == 2 || warp == 13) {
-    // ---- raw scales -> MMA scale atoms (lane = m0); warp 2: block 0 and activations, warp 13: block 1
-    const int b_lo = warp == 2 ? 0 : 1;
-    int it = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      bool ok = true;
-      for (int s = 0; s < G::S; ++s, ++it) {
-        const int slot = it % kW4D;
-        if (!pf_wait_all(&bb.full_a[slot], (it / kW4D) & 1, abort, p.err) ||
-            !pf_wait_all(&bb.full_b[slot], (it / kW4D) & 1, abort, p.err)) {
-          ok = false;
-          break;
-        }
-        uint8_t* st = sm + slot * kW4Stage;
-#pragma unroll
-        for (int bi = 0; bi < 2; ++bi) {        // (weight block 0, activations) or weight block 1
-          const int b = bi == 0 ? b_lo : 2;
-          if (b_lo == 1 && bi == 1) break;
-          const uint8_t* raw = b < 2 ? st + kW4OffRawA + b * kW4RawA : st + kW4OffRawB;
-          const int nm1 = b < 2 ? 4 : kW4BRows / 32;
-          uint4 r[4];
-#pragma unroll
-          for (int m1 = 0; m1 < 4; ++m1)
-            r[m1] = m1 < nm1 ? *reinterpret_cast<const uint4*>(raw + (lane + 32 * m1) * 16) : make_uint4(0, 0, 0, 0);
-          uint8_t* atom = st + kW4OffAtom + b * 4 * kW4Atom + lane * 16;
-          *reinterpret_cast<uint4*>(atom + 0 * kW4Atom) = make_uint4(r[0].x, r[1].x, r[2].x, r[3].x);
-          *reinterpret_cast<uint4*>(atom + 1 * kW4Atom) = make_uint4(r[0].y, r[1].y, r[2].y, r[3].y);
-          *reinterpret_cast<uint4*>(atom + 2 * kW4Atom) = make_uint4(r[0].z, r[1].z, r[2].z, r[3].z);
-          *reinterpret_cast<uint4*>(atom + 3 * kW4Atom) = make_uint4(r[0].w, r[1].w, r[2].w, r[3].w);
-        }
-        fence_proxy_async_smem();               // the atoms are read by tcgen05.cp (async proxy)
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bb.sf_ready[slot]);
-      }
-      if (!ok) break;
-    }
-  } else if (warp == 1 || warp == 12) {
+  } else if (warp == 1 || warp == 2) {
     // ---- scale copies and MMA issue for one weight block (uniform control flow; an elected lane issues)
-    const int b = warp == 1 ? 0 : 1;
+    const int b = warp - 1;
     int it = 0, ti = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++ti) {
@@ -357,8 +419,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
       const uint32_t d = tmem + as * 128 + b * 64;
       for (int s = 0; s < G::S; ++s, ++it) {
         const int slot = it % kW4D;
-        if (!pf_wait_all(&bb.sf_ready[slot], (it / kW4D) & 1, abort, p.err) ||
-            !pf_wait_all(&bb.full_a[slot], (it / kW4D) & 1, abort, p.err) ||
+        if (!pf_wait_all(&bb.full_a[slot], (it / kW4D) & 1, abort, p.err) ||
             !pf_wait_all(&bb.full_b[slot], (it / kW4D) & 1, abort, p.err)) {
           ok = false;
           break;
@@ -368,8 +429,8 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
         const uint32_t sfa = tmem + kW4ColSf + slot * kW4SfSlot + b * 32, sfb = sfa + 16;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          tc_cp_atom_w(sfa + j * 4, sdesc_atom(st + kW4OffAtom + (b * 4 + j) * kW4Atom));
-          tc_cp_atom_w(sfb + j * 4, sdesc_atom(st + kW4OffAtom + (2 * 4 + j) * kW4Atom));
+          tc_cp_atom_w(sfa + j * 4, sdesc_atom(st + kW4OffSfA + b * kW4StepAtoms + j * kAtom));
+          tc_cp_atom_w(sfb + j * 4, sdesc_atom(st + kW4OffSfB + j * kAtom));
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j)
@@ -383,51 +444,102 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
     pf_wait_all(&bb.done[b], 0, abort, p.err);
   } else if (warp >= 4 && warp < 12) {
     // ---- epilogue: lane quarter q holds weight rows 32q.. of both blocks; set k the 16-column
-    // groups 2i + k
+    // groups k and k + 2
     const int q = warp & 3, r = 32 * q + lane, k = (warp - 4) >> 2;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    __half* slab = reinterpret_cast<__half*>(sm + kW4OffSlab) + (warp - 4) * 16 * 32;
     pdl_wait();                                    // the activation tensor scales are the previous kernel's output
-    int ti = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++ti) {
-      const PfTile tl = tile_at(tt, t);
-      const int as = ti & 1;
-      // the tile's scales are loaded before the wait for its accumulators: the weight tensor scales
-      // and one activation tensor scale per column (column c in lane c % 32 of ts_lo / ts_hi)
-      float tw0, tw1;
+    // A tile's scales (the weight tensor scales and one activation tensor scale per column, column c
+    // in lane c % 32 of ts_lo / ts_hi) are loaded one tile ahead, so their latency is hidden.
+    struct Scales {
+      float tw0, tw1, ts_lo, ts_hi;
+    };
+    auto load_scales = [&](const PfTile& tl) {
+      Scales sc;
       if constexpr (PHASE == kPhaseGateUp) {
-        tw0 = __ldg(p.tscale + 2 * tl.w);
-        tw1 = __ldg(p.tscale + 2 * tl.w + 1);
+        sc.tw0 = __ldg(p.tscale + 2 * tl.w);
+        sc.tw1 = __ldg(p.tscale + 2 * tl.w + 1);
       } else {
-        tw0 = tw1 = __ldg(p.tscale + tl.w);
+        sc.tw0 = sc.tw1 = __ldg(p.tscale + tl.w);
       }
-      const float ts_lo = lane < tl.n ? __ldg(p.act_ts + tl.row0 + lane) : 0.f;
-      const float ts_hi = lane + 32 < tl.n ? __ldg(p.act_ts + tl.row0 + 32 + lane) : 0.f;
+      sc.ts_lo = lane < tl.n ? __ldg(p.act_ts + tl.row0 + lane) : 0.f;
+      sc.ts_hi = lane + 32 < tl.n ? __ldg(p.act_ts + tl.row0 + 32 + lane) : 0.f;
+      return sc;
+    };
+    int ti = 0;
+    PfTile tl{};
+    Scales sc{};
+    if (static_cast<int>(blockIdx.x) < total) {
+      tl = tile_at(tt, blockIdx.x);
+      sc = load_scales(tl);
+    }
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++ti) {
+      const int as = ti & 1;
+      PfTile tn{};
+      Scales sn{};
+      if (t + static_cast<int>(gridDim.x) < total) {
+        tn = tile_at(tt, t + gridDim.x);
+        sn = load_scales(tn);
+      }
       if (!pf_wait_all(&bb.acc_full[as], (ti >> 1) & 1, abort, p.err)) break;
       tc_fence_after();
+      // this warp's column groups (k and k + 2) of both blocks into registers, then the
+      // accumulators are released before the math and the stores
       const uint32_t dbase = lane_base + as * 128;
-      for (int j0 = 16 * k; j0 < tl.n; j0 += 32) {
-        uint32_t d0[16], d1[16];
-        tc_ld16(dbase + j0, d0);
-        tc_ld16(dbase + 64 + j0, d1);
-        tc_wait_ld();
+      const int ng = tl.n > 16 * (k + 2) ? 2 : tl.n > 16 * k ? 1 : 0;
+      uint32_t dv[2][2][16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float ta = __shfl_sync(kAll, j0 < 32 ? ts_lo : ts_hi, (j0 + c) & 31);
-          if (j0 + c < tl.n) {
-            const size_t row = static_cast<size_t>(tl.row0 + j0 + c);
-            const float v0 = __uint_as_float(d0[c]) * (tw0 * ta), v1 = __uint_as_float(d1[c]) * (tw1 * ta);
-            if constexpr (PHASE == kPhaseGateUp) {
-              p.h32[row * kI + tl.rp * 128 + r] = silu_fast(v0) * v1;
-            } else {
-              p.o[row * kH + tl.rp * 256 + r] = __float2half_rn(v0);
-              p.o[row * kH + tl.rp * 256 + 128 + r] = __float2half_rn(v1);
-            }
-          }
+      for (int g = 0; g < 2; ++g) {
+        if (g < ng) {
+          tc_ld16(dbase + 16 * (k + 2 * g), dv[g][0]);
+          tc_ld16(dbase + 64 + 16 * (k + 2 * g), dv[g][1]);
         }
       }
+      tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bb.acc_empty[as]);
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        if (g >= ng) break;
+        const int j0 = 16 * (k + 2 * g);
+        if constexpr (PHASE == kPhaseGateUp) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float ta = __shfl_sync(kAll, j0 < 32 ? sc.ts_lo : sc.ts_hi, (j0 + c) & 31);
+            if (j0 + c < tl.n) {
+              const size_t row = static_cast<size_t>(tl.row0 + j0 + c);
+              const float v0 = __uint_as_float(dv[g][0][c]) * (sc.tw0 * ta);
+              const float v1 = __uint_as_float(dv[g][1][c]) * (sc.tw1 * ta);
+              p.h32[row * kI + tl.rp * 128 + r] = silu_fast(v0) * v1;
+            }
+          }
+        } else {
+          // o rows through the slab: lane = output (32q + lane of the block), 16 tokens, then each
+          // lane stores 16-byte pieces (8 outputs) of two token rows
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float ta = __shfl_sync(kAll, j0 < 32 ? sc.ts_lo : sc.ts_hi, (j0 + c) & 31);
+              slab[c * 32 + lane] = __float2half_rn(__uint_as_float(dv[g][b][c]) * (sc.tw0 * ta));
+            }
+            __syncwarp();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int piece = lane + 32 * h, c = piece >> 2, f = (piece & 3) * 8;
+              if (j0 + c < tl.n) {
+                const uint4 v = *reinterpret_cast<const uint4*>(slab + c * 32 + f);
+                *reinterpret_cast<uint4*>(p.o + static_cast<size_t>(tl.row0 + j0 + c) * kH + tl.rp * 256 + b * 128 +
+                                          32 * q + f) = v;
+              }
+            }
+            __syncwarp();
+          }
+        }
+      }
+      tl = tn;
+      sc = sn;
     }
   }
 
@@ -454,15 +566,27 @@ cudaError_t launch_pdl(Kern kernel, int grid, int threads, int smem, bool pdl, c
 
 }  // namespace
 
-cudaError_t launch_act_quant_x(const uint16_t* x, int T, int K, const int* inv, uint8_t* codes, uint8_t* scales,
-                               float* ts, cudaStream_t s) {
-  if (T <= 0) return cudaSuccess;
-  act_quant_kernel<kH, true><<<T, 256, 0, s>>>(x, T, K, inv, codes, scales, ts);
+size_t w4a4_chunk_capacity(size_t P, int E) { return (P + 63) / 64 + static_cast<size_t>(E); }
+
+cudaError_t launch_pack_sf_atoms(const uint8_t* scales, int rows, int K, uint8_t* atoms, cudaStream_t s) {
+  if (rows % 128 != 0 || K % 64 != 0) return cudaErrorInvalidValue;
+  const size_t n = static_cast<size_t>(rows / 128) * (K / 64) * 32;
+  if (n == 0) return cudaSuccess;
+  const int grid = static_cast<int>(std::min<size_t>((n + 255) / 256, 65535));
+  pack_sf_atoms_kernel<<<grid, 256, 0, s>>>(scales, rows, K, atoms);
   return cudaGetLastError();
 }
 
-cudaError_t launch_act_quant_h(const float* h, int P, uint8_t* codes, uint8_t* scales, float* ts, bool pdl,
+cudaError_t launch_act_quant_x(const uint16_t* x, int T, int K, int E, const int* ids, const int* inv,
+                               const int* offsets, uint8_t* codes, uint8_t* scales, uint8_t* atoms, float* ts, int* rowc,
                                cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  act_quant_x_kernel<<<T, 256, 0, s>>>(x, K, E, ids, inv, offsets, codes, scales, atoms, ts, rowc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_act_quant_h(const float* h, int P, const int* rowc, uint8_t* codes, uint8_t* scales, uint8_t* atoms,
+                               float* ts, bool pdl, cudaStream_t s) {
   if (P <= 0) return cudaSuccess;
   constexpr int kRows = 256 / (kI / 8);
   cudaLaunchConfig_t cfg{};
@@ -474,8 +598,7 @@ cudaError_t launch_act_quant_h(const float* h, int P, uint8_t* codes, uint8_t* s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, act_quant_kernel<kI, false>, static_cast<const void*>(h), P, 1,
-                            static_cast<const int*>(nullptr), codes, scales, ts);
+  return cudaLaunchKernelEx(&cfg, act_quant_h_kernel, h, P, rowc, codes, scales, atoms, ts);
 }
 
 cudaError_t launch_w4a4_routed(const PrefillParams& p, int phase, int n_sm, bool pdl, cudaStream_t s) {
