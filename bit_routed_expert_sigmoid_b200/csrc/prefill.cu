@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
     bb.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0) build_tiles(tt, p, G::RP);
+  if (warp == 0) build_tiles<false>(tt, p, G::RP);
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&bb.tmem)));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
     int it = 0;
     if (lane == 0) {
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-        const PfTile tl = tile_at(tt, t);
+        const PfTile tl = tile_at<false>(tt, t);
         const int r0 = G::row(tl.w, tl.rp, 0), r1 = G::row(tl.w, tl.rp, 1);
         for (int s = 0; s < G::S; ++s, ++it) {
           const int slot = it % kPfDA;
@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
       pdl_wait();     // the activation rows are the previous kernel's output
       int it = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-        const PfTile tl = tile_at(tt, t);
+        const PfTile tl = tile_at<false>(tt, t);
         const int nbox = (tl.n + 15) >> 4;
         bool ok = true;
         for (int s = 0; s < G::S; ++s, ++it) {
@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
     int it = 0, ti = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++ti) {
-      const PfTile tl = tile_at(tt, t);
+      const PfTile tl = tile_at<false>(tt, t);
       const int npad = (tl.n + 15) & ~15;
       const uint32_t idesc = idesc_m128(npad, false);
       const int as = ti & 1;
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
     int t = blockIdx.x;
     int row = 0;
     if (t < total) {
-      const PfTile tl = tile_at(tt, t);
+      const PfTile tl = tile_at<false>(tt, t);
       row = G::row(tl.w, tl.rp, b) + r;
       if constexpr (FMT == kInt4) load_int4(row);
       else load_fp4(row, 0);
@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
       const int t_next = t + gridDim.x;
       int row_next = -1;
       if (t_next < total) {
-        const PfTile tn = tile_at(tt, t_next);
+        const PfTile tn = tile_at<false>(tt, t_next);
         row_next = G::row(tn.w, tn.rp, b) + r;
       }
       uint32_t sc[kSc4];                         // consumed from sc[0], shifted down every 2 stages
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
     int ti = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++ti) {
-      const PfTile tl = tile_at(tt, t);
+      const PfTile tl = tile_at<false>(tt, t);
       const int as = ti & 1;
       if (!pf_wait_all(&bb.acc_full[as][0], (ti >> 1) & 1, abort, p.err) ||
           !pf_wait_all(&bb.acc_full[as][1], (ti >> 1) & 1, abort, p.err))

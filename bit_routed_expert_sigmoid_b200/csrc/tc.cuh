@@ -138,7 +138,9 @@ struct PfTile {
 
 // Warp 0: tiles of expert e are rp-major over its chunks; experts in ascending order (an expert
 // without rows has none). Every lane loads the offsets (and weight slots) of all its experts before
-// the scans, so the table costs one global-load latency rather than one per 32 experts.
+// the scans, so the table costs one global-load latency rather than one per 32 experts. kChunks:
+// also number every expert's chunks (cbase; only the W4A4 kernels address data by chunk).
+template <bool kChunks>
 __device__ void build_tiles(TileTab& tt, const PrefillParams& p, int rp_count) {
   constexpr int kPer = kMaxE / 32;
   const int lane = threadIdx.x & 31;
@@ -178,7 +180,7 @@ __device__ void build_tiles(TileTab& tt, const PrefillParams& p, int rp_count) {
     }
     if (i < n) {
       tt.start[i] = base + v - tiles;
-      tt.cbase[i] = cb + vc - nchunks;
+      if constexpr (kChunks) tt.cbase[i] = cb + vc - nchunks;
     }
     base += __shfl_sync(kAll, v, 31);
     cb += __shfl_sync(kAll, vc, 31);
@@ -190,6 +192,7 @@ __device__ void build_tiles(TileTab& tt, const PrefillParams& p, int rp_count) {
   }
 }
 
+template <bool kChunks>
 __device__ __forceinline__ PfTile tile_at(const TileTab& tt, int t) {
   int lo = 0, hi = tt.n - 1;                 // last i with start[i] <= t (t < total)
   while (lo < hi) {
@@ -205,7 +208,7 @@ __device__ __forceinline__ PfTile tile_at(const TileTab& tt, int t) {
   r.row0 = tt.off[lo] + ch * kPfN;
   r.n = min(kPfN, tt.cnt[lo] - ch * kPfN);
   r.rp = rp;
-  r.c = tt.cbase[lo] + ch;
+  r.c = kChunks ? tt.cbase[lo] + ch : 0;
   return r;
 }
 

@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
     bb.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0) build_tiles(tt, p, G::RP);
+  if (warp == 0) build_tiles<true>(tt, p, G::RP);
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&bb.tmem)));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
     if (lane == 0) {
       int it = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-        const PfTile tl = tile_at(tt, t);
+        const PfTile tl = tile_at<true>(tt, t);
         const int r0 = G::row(tl.w, tl.rp, 0), r1 = G::row(tl.w, tl.rp, 1);
         for (int s = 0; s < G::S; ++s, ++it) {
           const int slot = it % kW4D;
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
       pdl_wait();
       int it = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-        const PfTile tl = tile_at(tt, t);
+        const PfTile tl = tile_at<true>(tt, t);
         const int nbox = (tl.n + 15) >> 4;
         bool ok = true;
         for (int s = 0; s < G::S; ++s, ++it) {
@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
     int it = 0, ti = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++ti) {
-      const PfTile tl = tile_at(tt, t);
+      const PfTile tl = tile_at<true>(tt, t);
       const uint32_t idesc = idesc_mxf4nvf4((tl.n + 15) & ~15);
       const int as = ti & 1;
       if (ti >= 2 && !pf_wait_all(&bb.acc_empty[as], ((ti >> 1) - 1) & 1, abort, p.err)) break;
@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
     PfTile tl{};
     Scales sc{};
     if (static_cast<int>(blockIdx.x) < total) {
-      tl = tile_at(tt, blockIdx.x);
+      tl = tile_at<true>(tt, blockIdx.x);
       sc = load_scales(tl);
     }
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++ti) {
@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
       PfTile tn{};
       Scales sn{};
       if (t + static_cast<int>(gridDim.x) < total) {
-        tn = tile_at(tt, t + gridDim.x);
+        tn = tile_at<true>(tt, t + gridDim.x);
         sn = load_scales(tn);
       }
       if (!pf_wait_all(&bb.acc_full[as], (ti >> 1) & 1, abort, p.err)) break;

@@ -178,6 +178,22 @@ def test_w4a4_full_size_workload_sampled():
     dev.close()
 
 
+def test_w4a4_is_deterministic():
+    # repeated forwards agree bit for bit: y, and the gate|up output h before its quantisation
+    L = layer(256)
+    T = 200
+    x = x_to_device(S.make_workload_x(T, 256))
+    dev = FlintMoELayer(L, t_max=T, flags=B.FLINT_FLAG_W4A4)
+    runs = []
+    for _ in range(3):
+        y = dev.forward(x).clone()
+        runs.append((y.view(torch.int16), dev.intermediate(B.FLINT_BUF_H, T)))
+    torch.cuda.synchronize()
+    for y, h in runs[1:]:
+        assert torch.equal(runs[0][0], y) and torch.equal(runs[0][1], h)
+    dev.close()
+
+
 def test_w4a4_leaves_decode_unchanged():
     # T <= 8 runs the decode kernel with 16-bit activations, with or without the flag
     L = layer(32)
