@@ -180,7 +180,7 @@ def ncu_traffic(kernel: str, workload: str):
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
-    cur = source_hash(TRAFFIC_SOURCES.get(kernel))
+    cur = source_hash(traffic_sources(kernel, workload))
     for line in open(path):
         line = line.split("#")[0].strip()
         if not line:
@@ -195,9 +195,17 @@ def ncu_traffic(kernel: str, workload: str):
 # recorded figure stands while these files are unchanged
 TRAFFIC_SOURCES = {
     "layer": ("common.cuh", "decode.cu", "frag.cuh", "kernels.cuh"),
-    "gu_routed": ("common.cuh", "kernels.cuh", "prefill.cu"),
+    "gu_routed": ("common.cuh", "kernels.cuh", "prefill.cu", "tc.cuh"),
     "quant": ("quant.cu",),
 }
+# W4A4 workloads: the routed kernels are those of w4a4.cu
+TRAFFIC_SOURCES_W4A4 = {k: ("common.cuh", "kernels.cuh", "tc.cuh", "w4a4.cu") for k in ("gu_routed", "dn_routed")}
+
+
+def traffic_sources(kernel: str, workload: str):
+    if workload in W4A4_WORKLOADS and kernel in TRAFFIC_SOURCES_W4A4:
+        return TRAFFIC_SOURCES_W4A4[kernel]
+    return TRAFFIC_SOURCES.get(kernel)
 
 
 def _code_only(text: str) -> str:
