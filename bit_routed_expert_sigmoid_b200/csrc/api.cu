@@ -53,6 +53,7 @@ struct flint_moe_ctx {
   uint8_t* ha_sf;
   float* ha_ts;
   int* rowc;                               // W4A4: chunk position (chunk * 64 + row in chunk) of each permuted row
+  int* chunk_base;                         // W4A4: [E] first 64-row chunk of each expert
   uint8_t* xa_atoms;                       // W4A4: block scales of x and h as MMA atoms [chunk][K/64][512]
   uint8_t* ha_atoms;
   uint8_t* w_atoms_gu;                     // W4A4: weight block scales as MMA atoms [rows / 128][K/64][512]
@@ -219,6 +220,7 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
   const size_t CA = PA ? w4a4_chunk_capacity(P, static_cast<int>(E)) : 0;
   const size_t WR = PA ? static_cast<size_t>(c.n_experts) : 0;          // W4A4 handles take no cache slots
   char* p_rowc = take(PA * 4);
+  char* p_cbase = take(PA ? E * 4 : 0);
   char* p_xa_atoms = take(CA * (kH / 64) * 512);
   char* p_ha_atoms = take(CA * (kI / 64) * 512);
   char* p_w_atoms_gu = take(WR * (2 * kI / 128) * (kH / 64) * 512);
@@ -259,6 +261,7 @@ size_t plan(flint_moe_ctx* h, const flint_moe_cfg& c, char* base) {
     h->ha_sf = reinterpret_cast<uint8_t*>(p_ha_sf);
     h->ha_ts = reinterpret_cast<float*>(p_ha_ts);
     h->rowc = reinterpret_cast<int*>(p_rowc);
+    h->chunk_base = reinterpret_cast<int*>(p_cbase);
     h->xa_atoms = reinterpret_cast<uint8_t*>(p_xa_atoms);
     h->ha_atoms = reinterpret_cast<uint8_t*>(p_ha_atoms);
     h->w_atoms_gu = reinterpret_cast<uint8_t*>(p_w_atoms_gu);
@@ -406,11 +409,12 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
     FLINT_TRY(launch_topk(h->logits_part, kRouterSplit, h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, rs));
     FLINT_TRY(m.mark());
   }
-  FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, c.flags, h->err, rs));
+  FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, h->w4a4 ? h->chunk_base : nullptr,
+                           c.flags, h->err, rs));
   FLINT_TRY(m.mark());
   if (h->w4a4)
-    FLINT_TRY(launch_act_quant_x(x, T, K, E, h->ids, h->inv, h->offsets, h->xa, h->xa_sf, h->xa_atoms, h->xa_ts, h->rowc,
-                                 rs));
+    FLINT_TRY(launch_act_quant_x(x, T, K, E, h->ids, h->inv, h->offsets, h->chunk_base, h->xa, h->xa_sf, h->xa_atoms,
+                                 h->xa_ts, h->rowc, rs));
   else FLINT_TRY(launch_xg(x, T, K, h->inv, fmt == kInt4 ? 1 : 0, h->xg, rs));
   FLINT_TRY(m.mark());
 

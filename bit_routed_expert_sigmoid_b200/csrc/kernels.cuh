@@ -117,8 +117,8 @@ cudaError_t launch_pack_sf_atoms(const uint8_t* scales, int rows, int K, uint8_t
 // [chunk][H/64][512], written to each token's permuted rows inv[t][k]; rowc[p] = the row's chunk *
 // 64 + its row in the chunk
 cudaError_t launch_act_quant_x(const uint16_t* x, int T, int K, int E, const int* ids, const int* inv,
-                               const int* offsets, uint8_t* codes, uint8_t* scales, uint8_t* atoms, float* ts, int* rowc,
-                               cudaStream_t s);
+                               const int* offsets, const int* chunk_base, uint8_t* codes, uint8_t* scales,
+                               uint8_t* atoms, float* ts, int* rowc, cudaStream_t s);
 // h (fp32 [P][I]) -> codes [P][I/2], scales [P][I/16], tensor scales [P], atoms [chunk][I/64][512]
 cudaError_t launch_act_quant_h(const float* h, int P, const int* rowc, uint8_t* codes, uint8_t* scales, uint8_t* atoms,
                                float* ts, bool pdl, cudaStream_t s);
@@ -131,8 +131,11 @@ cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* wr, int T, i
 // written to logits_out [T][E] when it is not null.
 cudaError_t launch_topk(const float* logits, int nsplit, float* logits_out, int T, int E, int K, float floor_, int* ids,
                         float* wts, unsigned flags, unsigned* err, cudaStream_t s);
+// chunk_base (may be null): [E] the first 64-row chunk of each expert, chunks numbered over all experts
+// in ascending order (an exclusive prefix of ceil(count / 64)); the W4A4 path addresses its
+// activation scale atoms by chunk.
 cudaError_t launch_permute(const int* ids, int T, int K, int E, int* counts, int* offsets, int* perm, int* inv,
-                           unsigned flags, unsigned* err, cudaStream_t s);
+                           int* chunk_base, unsigned flags, unsigned* err, cudaStream_t s);
 cudaError_t launch_xg(const uint16_t* x, int T, int K, const int* inv, int rotate, __half* xg, cudaStream_t s);
 
 cudaError_t launch_prefill_combine(const __half* o, const float* ys, const float* w, const int* inv, int T, int K,

@@ -174,9 +174,10 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
   pdl_trigger();   // the next kernel's CTAs take the SMs this grid leaves (it is resident in full)
 
   if (warp == 0) {
-    // ---- codes: two TMA boxes (128 rows x 64 bytes) per stage
+    // ---- codes: two TMA boxes (128 rows x 64 bytes) per stage (read once: evicted first from L2)
     int it = 0;
     if (lane == 0) {
+      const uint64_t pol = l2_evict_first();
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
         const PfTile tl = tile_at<false>(tt, t);
         const int r0 = G::row(tl.w, tl.rp, 0), r1 = G::row(tl.w, tl.rp, 1);
@@ -185,8 +186,8 @@ __global__ void __launch_bounds__(PfRoles<FMT, PHASE>::kThreads, 1) pf_routed_ke
           if (it >= kPfDA && !pf_wait(&bb.code_empty[slot], ((it / kPfDA) - 1) & 1, abort, p.err)) break;
           uint8_t* st = sm + kOffCode + slot * kPfCodeStage;
           mbar_arrive_expect_tx(&bb.code_full[slot], kPfCodeStage);
-          tma_2d(st, &p.tm_codes, s * (kPfSK / 8), r0, &bb.code_full[slot]);
-          tma_2d(st + kPfCodeStage / 2, &p.tm_codes, s * (kPfSK / 8), r1, &bb.code_full[slot]);
+          tma_2d_hint(st, &p.tm_codes, s * (kPfSK / 8), r0, &bb.code_full[slot], pol);
+          tma_2d_hint(st + kPfCodeStage / 2, &p.tm_codes, s * (kPfSK / 8), r1, &bb.code_full[slot], pol);
         }
       }
       // no copy may still be in flight when the CTA exits

@@ -187,10 +187,11 @@ __device__ __forceinline__ int clamp_id(int v, int E) { return (v < 0 || v >= E)
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __restrict__ ids, int P, int E,
                                                                int* __restrict__ counts, int* __restrict__ offsets,
                                                                int* __restrict__ perm, int* __restrict__ inv,
-                                                               unsigned flags, unsigned* __restrict__ err) {
+                                                               int* __restrict__ chunk_base, unsigned flags,
+                                                               unsigned* __restrict__ err) {
   __shared__ int h_total[kMaxE], h_before[kMaxE], first[kMaxE];
   __shared__ int wcnt[kPermWarps * kMaxE];        // [warp][expert]: pairs of the expert in the warp
-  __shared__ int scan_w[kMaxE / 32];
+  __shared__ int scan_w[kMaxE / 32], scan_c[kMaxE / 32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c0 = blockIdx.x * kPermThreads;
   const int i = c0 + tid;
@@ -242,16 +243,24 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __rest
   __syncthreads();
   // offsets: exclusive scan of the totals over the experts; per expert, exclusive scan of the warp
   // counts over the warps
-  int incl = 0, tot = 0;
+  int incl = 0, tot = 0, incl_c = 0, nch = 0;
   if (tid < kMaxE) {
     tot = tid < E ? h_total[tid] : 0;
     incl = tot;
+    nch = (tot + 63) >> 6;                         // 64-row chunks of the expert (W4A4 chunk numbering)
+    incl_c = nch;
 #pragma unroll
     for (int m = 1; m < 32; m <<= 1) {
-      const int o = __shfl_up_sync(0xFFFFFFFFu, incl, m);
-      if (lane >= m) incl += o;
+      const int o = __shfl_up_sync(0xFFFFFFFFu, incl, m), oc = __shfl_up_sync(0xFFFFFFFFu, incl_c, m);
+      if (lane >= m) {
+        incl += o;
+        incl_c += oc;
+      }
     }
-    if (lane == 31) scan_w[warp] = incl;
+    if (lane == 31) {
+      scan_w[warp] = incl;
+      scan_c[warp] = incl_c;
+    }
     if (tid < E) {
       int c[kPermWarps];
 #pragma unroll
@@ -273,6 +282,11 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __rest
       counts[tid] = tot;
       offsets[tid] = off;
       if (tid == E - 1) offsets[E] = off + tot;
+      if (chunk_base) {
+        int cb = incl_c - nch;
+        for (int w = 0; w < warp; ++w) cb += scan_c[w];
+        chunk_base[tid] = cb;
+      }
     }
   }
   __syncthreads();
@@ -327,10 +341,10 @@ cudaError_t launch_topk(const float* logits, int nsplit, float* logits_out, int 
 }
 
 cudaError_t launch_permute(const int* ids, int T, int K, int E, int* counts, int* offsets, int* perm, int* inv,
-                           unsigned flags, unsigned* err, cudaStream_t s) {
+                           int* chunk_base, unsigned flags, unsigned* err, cudaStream_t s) {
   const int P = T * K;
   const int grid = P > 0 ? (P + kPermThreads - 1) / kPermThreads : 1;
-  permute_kernel<<<grid, kPermThreads, 0, s>>>(ids, P, E, counts, offsets, perm, inv, flags, err);
+  permute_kernel<<<grid, kPermThreads, 0, s>>>(ids, P, E, counts, offsets, perm, inv, chunk_base, flags, err);
   return cudaGetLastError();
 }
 

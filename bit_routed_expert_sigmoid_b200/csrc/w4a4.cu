@@ -21,8 +21,9 @@
 //   weights      [row block of 128][K/64][atom], packed once when the handle is made
 //                (pack_sf_atoms_kernel) from the [row][K/16] scales
 //   activations  [chunk][K/64][atom], written by the quantisers; a chunk is 64 consecutive permuted
-//                rows of one expert (the GEMM's N), numbered over all experts in ascending order,
-//                and only m1 = 0, 1 of its atoms are meaningful
+//                rows of one expert (the GEMM's N), numbered over all experts in ascending order (the
+//                permutation kernel writes each expert's first chunk), and only m1 = 0, 1 of its atoms
+//                are meaningful
 //
 // The routed GEMM walks the tile table of the W4A16 routed kernel: a tile is (expert, a chunk of up
 // to 64 of its permuted rows, a pair of 128-row weight blocks). One persistent CTA per SM; warps:
@@ -128,51 +129,27 @@ __device__ __forceinline__ float row_tscale(const float (&v)[8], float* wmax, in
   return am > 0.f ? __fdiv_rn(am, 2688.f) : 1.f;
 }
 
-// x: one token per CTA (256 threads x 8 values). Warp 0 first numbers the chunks of all experts
-// (exclusive prefix of ceil(count / 64) over ascending expert ids, from the offsets) and places
-// each of the token's top-k permuted rows: its chunk position, also stored in rowc for the h
-// quantiser.
+// x: one token per CTA (256 threads x 8 values). Warp 0 first places each of the token's top-k
+// permuted rows in its expert's 64-row chunks (chunk_base from the permutation kernel): its chunk
+// position, also stored in rowc for the h quantiser.
 __global__ void __launch_bounds__(256) act_quant_x_kernel(const uint16_t* __restrict__ x, int top_k, int E,
                                                           const int* __restrict__ ids, const int* __restrict__ inv,
-                                                          const int* __restrict__ offsets, uint8_t* __restrict__ codes,
+                                                          const int* __restrict__ offsets,
+                                                          const int* __restrict__ chunk_base, uint8_t* __restrict__ codes,
                                                           uint8_t* __restrict__ scales, uint8_t* __restrict__ atoms,
                                                           float* __restrict__ ts_out, int* __restrict__ rowc) {
   static_assert(kH / 8 == 256, "one token per 256 threads");
-  constexpr int kPer = kMaxE / 32;
   __shared__ float wmax[8];
-  __shared__ int cb[kMaxE];
   __shared__ int dst_row[kMaxTopK], dst_pos[kMaxTopK];
   const int t = blockIdx.x, i = threadIdx.x, warp = i >> 5, lane = i & 31;
-  if (warp == 0) {
-    int nch[kPer], sum = 0;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int e = kPer * lane + j;
-      nch[j] = e < E ? (__ldg(offsets + e + 1) - __ldg(offsets + e) + 63) >> 6 : 0;
-      sum += nch[j];
-    }
-    int incl = sum;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int u = __shfl_up_sync(kAll, incl, d);
-      if (lane >= d) incl += u;
-    }
-    int run = incl - sum;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      cb[kPer * lane + j] = run;
-      run += nch[j];
-    }
-    __syncwarp();
-    if (lane < top_k) {
-      const int e = min(max(__ldg(ids + t * top_k + lane), 0), E - 1);
-      const int p = __ldg(inv + t * top_k + lane);
-      const int local = p - __ldg(offsets + e);
-      const int pos = (cb[e] + (local >> 6)) * 64 + (local & 63);
-      dst_row[lane] = p;
-      dst_pos[lane] = pos;
-      rowc[p] = pos;
-    }
+  if (warp == 0 && lane < top_k) {
+    const int e = min(max(__ldg(ids + t * top_k + lane), 0), E - 1);
+    const int p = __ldg(inv + t * top_k + lane);
+    const int local = p - __ldg(offsets + e);
+    const int pos = (__ldg(chunk_base + e) + (local >> 6)) * 64 + (local & 63);
+    dst_row[lane] = p;
+    dst_pos[lane] = pos;
+    rowc[p] = pos;
   }
   float v[8];
   const uint4 wx = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * kH) + i);
@@ -358,8 +335,9 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
   pdl_trigger();
 
   if (warp == 0) {
-    // ---- weight codes and scale atoms
+    // ---- weight codes and scale atoms (read once: evicted first from L2)
     if (lane == 0) {
+      const uint64_t pol = l2_evict_first();
       int it = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
         const PfTile tl = tile_at<true>(tt, t);
@@ -369,12 +347,13 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
           if (it >= kW4D && !pf_wait(&bb.empty[slot], ((it / kW4D) - 1) & 1, abort, p.err)) break;
           uint8_t* st = sm + slot * kW4Stage;
           mbar_arrive_expect_tx(&bb.full_a[slot], 2 * kW4ABox + 2 * kW4StepAtoms);
-          tma_2d(st + kW4OffA, &p.tm_codes, s * 128, r0, &bb.full_a[slot]);
-          tma_2d(st + kW4OffA + kW4ABox, &p.tm_codes, s * 128, r1, &bb.full_a[slot]);
-          bulk_g2s(st + kW4OffSfA, p.w_atoms + (static_cast<size_t>(r0 / 128) * kSteps + 4 * s) * kAtom, kW4StepAtoms,
-                   &bb.full_a[slot]);
-          bulk_g2s(st + kW4OffSfA + kW4StepAtoms, p.w_atoms + (static_cast<size_t>(r1 / 128) * kSteps + 4 * s) * kAtom,
-                   kW4StepAtoms, &bb.full_a[slot]);
+          tma_2d_hint(st + kW4OffA, &p.tm_codes, s * 128, r0, &bb.full_a[slot], pol);
+          tma_2d_hint(st + kW4OffA + kW4ABox, &p.tm_codes, s * 128, r1, &bb.full_a[slot], pol);
+          bulk_g2s_hint(st + kW4OffSfA, p.w_atoms + (static_cast<size_t>(r0 / 128) * kSteps + 4 * s) * kAtom,
+                        kW4StepAtoms, &bb.full_a[slot], pol);
+          bulk_g2s_hint(st + kW4OffSfA + kW4StepAtoms,
+                        p.w_atoms + (static_cast<size_t>(r1 / 128) * kSteps + 4 * s) * kAtom, kW4StepAtoms,
+                        &bb.full_a[slot], pol);
         }
       }
       for (int j = max(it - kW4D, 0); j < it; ++j) pf_wait(&bb.full_a[j % kW4D], (j / kW4D) & 1, abort, p.err);
@@ -578,10 +557,10 @@ cudaError_t launch_pack_sf_atoms(const uint8_t* scales, int rows, int K, uint8_t
 }
 
 cudaError_t launch_act_quant_x(const uint16_t* x, int T, int K, int E, const int* ids, const int* inv,
-                               const int* offsets, uint8_t* codes, uint8_t* scales, uint8_t* atoms, float* ts, int* rowc,
-                               cudaStream_t s) {
+                               const int* offsets, const int* chunk_base, uint8_t* codes, uint8_t* scales,
+                               uint8_t* atoms, float* ts, int* rowc, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  act_quant_x_kernel<<<T, 256, 0, s>>>(x, K, E, ids, inv, offsets, codes, scales, atoms, ts, rowc);
+  act_quant_x_kernel<<<T, 256, 0, s>>>(x, K, E, ids, inv, offsets, chunk_base, codes, scales, atoms, ts, rowc);
   return cudaGetLastError();
 }
 
