@@ -64,7 +64,10 @@ typedef enum flint_wformat {
  * activations in prefill). Per row: a tensor scale amax / (6 * 448) (1 for an all-zero row), an E4M3
  * scale per 16 values (nearest, ties to even, saturating), E2M1 codes (nearest, ties to even), each
  * quotient and product rounded to fp32 in that order. Decode (T <= 8) keeps 16-bit activations.
- * Adds ~1.3 KB per permuted row (t_max * top_k rows) to the workspace. */
+ * flint_moe_create copies the weight block scales into the MMA's layout (workspace; it synchronises
+ * the device first), so the weights must not change while the handle lives; not with n_slots > 0
+ * (FLINT_ERR_UNSUPPORTED). Adds ~60 MB to the workspace at E = 256, t_max = 2048 (scale atoms of
+ * the weights, and NVFP4 rows of x and h with their atoms, ~1.8 KB per permuted row). */
 #define FLINT_FLAG_W4A4 0x2u
 
 typedef struct flint_moe_cfg {
