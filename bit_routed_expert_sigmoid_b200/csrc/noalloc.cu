@@ -1,10 +1,8 @@
 // Routing entry point that needs no device memory from its caller beyond inputs and outputs.
 //
-// Some callers cannot allocate device memory at the moment they need routing: code that runs
-// while a CUDA graph is being captured (a cudaMalloc there is an error, and the allocation would
-// not be replayed), plug-ins whose host framework owns the device allocator and hands out no
-// workspace, and latency-critical loops that cannot afford the implicit device synchronisation a
-// cudaMalloc/cudaFree may perform. flint_moe_route_noalloc serves them: it runs the same router
+// Some callers cannot allocate device memory at the moment they need routing: plug-ins whose host
+// framework owns the device allocator and hands out no workspace, and latency-critical loops that
+// cannot afford the implicit device synchronisation a cudaMalloc/cudaFree may perform. flint_moe_route_noalloc serves them: it runs the same router
 // logits and top-k kernels as flint_moe_forward, but the fp32 logits it produces between the two
 // kernels live in a fixed, file-scope device array instead of a caller-provided workspace.
 //

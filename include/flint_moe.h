@@ -239,8 +239,8 @@ const char* flint_moe_stage_name(flint_moe_t h, int T, int i);
 
 /* Routing without any caller-provided device memory beyond inputs and outputs (this entry point
  * has no counterpart in the published descriptions of the layer; it exists for callers that cannot
- * allocate: code running while a CUDA graph is captured, plug-ins whose host owns the allocator,
- * loops that cannot afford the synchronisation an allocation may cause).
+ * allocate: plug-ins whose host owns the allocator, loops that cannot afford the synchronisation an
+ * allocation may cause).
  * Computes, for T tokens, the routing of flint_moe_forward: ids [T][top_k] (int32, ascending expert
  * id) and weights w [T][top_k] (f32). x bf16 [T][2048] and router_w bf16 [n_experts][2048] are
  * device inputs, ids and w device outputs, all caller-owned. Its fp32 logits come from the same
@@ -250,9 +250,8 @@ const char* flint_moe_stage_name(flint_moe_t h, int T, int i);
  * held on every GPU that loads the library until the process exits), so T <= 64 and n_experts <= 256
  * (a multiple of 32); larger sizes return FLINT_ERR_INVALID_ARG without launching anything. Calls no
  * cudaMalloc or cudaFree. The first call in a CUDA context looks up the array's device address (once
- * per device and context, with that device current), so make that first call before any stream
- * capture; a context destroyed and re-created (cudaDeviceReset) is noticed and the address looked up
- * again. All calls share the one array: calls whose kernels may overlap on the GPU (different streams
+ * per device and context, with that device current); a context destroyed and re-created
+ * (cudaDeviceReset) is noticed and the address looked up again. All calls share the one array: calls whose kernels may overlap on the GPU (different streams
  * without ordering) race on it and must be serialised by the caller. */
 flint_status flint_moe_route_noalloc(const void* x, const void* router_w, int T, int n_experts, int top_k,
                                      float norm_floor, int* ids, float* w, void* stream);

@@ -1,6 +1,6 @@
-"""flint_moe_route_noalloc: routing for callers that cannot allocate device memory (for example code
-running under CUDA graph capture, or a plug-in whose host owns the allocator). Its logits scratch is a
-fixed device array inside the library instead of a caller workspace; its results must equal the
+"""flint_moe_route_noalloc: routing for callers that cannot allocate device memory (for example a
+plug-in whose host owns the allocator). Its logits scratch is a fixed device array inside the library
+instead of a caller workspace; its results must equal the
 oracle's routing and the routing that flint_moe_forward produces through the existing entry points,
 call after call (ids exactly, weights to fp32 rounding: the two entry points form the same fp32 logits
 from exact bf16 products but sum them in different orders).
