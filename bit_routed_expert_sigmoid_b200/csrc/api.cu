@@ -406,16 +406,19 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
     pp.tm_b = tm_x;
     FLINT_TRY(launch_prefill_shared(pp, kPhaseRouter, h->n_sm, rs));
     FLINT_TRY(m.mark());
-    FLINT_TRY(launch_topk(h->logits_part, kRouterSplit, h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, rs));
+    FLINT_TRY(launch_topk(h->logits_part, kRouterSplit, h->logits, T, E, K, c.norm_floor, h->ids, h->wts, c.flags, h->err, rs,
+                          pdl));
     FLINT_TRY(m.mark());
   }
+  // the chain's kernels are programmatic dependents of their predecessor (the permutation only when the
+  // top-k ran right before it on this stream)
   FLINT_TRY(launch_permute(h->ids, T, K, E, h->counts, h->offsets, h->perm, h->inv, h->w4a4 ? h->chunk_base : nullptr,
-                           c.flags, h->err, rs));
+                           c.flags, h->err, rs, pdl && !route_in));
   FLINT_TRY(m.mark());
   if (h->w4a4)
     FLINT_TRY(launch_act_quant_x(x, T, K, E, h->ids, h->inv, h->offsets, h->chunk_base, h->xa, h->xa_sf, h->xa_atoms,
-                                 h->xa_ts, h->rowc, rs));
-  else FLINT_TRY(launch_xg(x, T, K, h->inv, fmt == kInt4 ? 1 : 0, h->xg, rs));
+                                 h->xa_ts, h->rowc, rs, pdl));
+  else FLINT_TRY(launch_xg(x, T, K, h->inv, fmt == kInt4 ? 1 : 0, h->xg, rs, pdl));
   FLINT_TRY(m.mark());
 
   pp.tm_a = h->tm_pf_sh_gu;                        // shared gate|up: B = x
@@ -426,7 +429,7 @@ flint_status run_forward(flint_moe_ctx* h, const uint16_t* x, int T, uint16_t* y
     pp.tm_a = h->tm_pf_sh_dn;
     pp.tm_b = h->tm_pf_hs_hi;
     pp.tm_b2 = h->tm_pf_hs_lo;
-    FLINT_TRY(launch_prefill_shared(pp, kPhaseDown, h->n_sm, s));
+    FLINT_TRY(launch_prefill_shared(pp, kPhaseDown, h->n_sm, s, pdl));
     FLINT_TRY(cudaEventRecord(h->ev_join, h->side));
     FLINT_TRY(cudaStreamWaitEvent(s, h->ev_join, 0));
   }

@@ -10,6 +10,12 @@
 
 namespace flint {
 
+// Programmatic dependent launch: the next kernel of the stream may be scheduled once every CTA of this
+// one has called launch_dependents (or exited); wait blocks until the previous kernel has completed
+// and its writes are visible (a no-op without a programmatic predecessor).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 constexpr int kH = 2048;        // hidden width
 constexpr int kI = 512;         // routed SwiGLU width
 constexpr int kIs = 1024;       // shared-expert SwiGLU width

@@ -8,6 +8,24 @@
 
 namespace flint {
 
+// Launches kernel<<<grid, threads, smem, s>>>(args...); with pdl as a programmatic dependent of the
+// previous kernel in the stream (the kernel then calls griddepcontrol.wait before it reads that
+// kernel's output, and may start its prologue while that kernel finishes).
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl_kernel(Kern kernel, int grid, int threads, int smem, bool pdl, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ---- decode path (T <= kDecodeMaxT): one persistent kernel, launched cooperatively ----
 constexpr int kDecodeMaxT = 8;
 constexpr int kMaxActive = 64;                 // active experts of a decode forward (T * top_k <= 64)
@@ -104,7 +122,7 @@ struct PrefillParams {
 // pdl: launched as a programmatic dependent of the previous kernel in the stream (the routed down
 // kernel streams its weights while the gate|up kernel finishes; it waits for it before reading h).
 cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, int n_sm, bool pdl, cudaStream_t s);
-cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, cudaStream_t s);
+cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, cudaStream_t s, bool pdl = false);
 
 // W4A4 (NVFP4 weights and activations). tm_codes: weight codes as bytes [rows][K/2], box 128 x 128
 // rows, 128-byte swizzle; tm_act: activation codes [P][K/2], box 128 x 16 rows, 128-byte swizzle.
@@ -118,7 +136,7 @@ cudaError_t launch_pack_sf_atoms(const uint8_t* scales, int rows, int K, uint8_t
 // 64 + its row in the chunk
 cudaError_t launch_act_quant_x(const uint16_t* x, int T, int K, int E, const int* ids, const int* inv,
                                const int* offsets, const int* chunk_base, uint8_t* codes, uint8_t* scales,
-                               uint8_t* atoms, float* ts, int* rowc, cudaStream_t s);
+                               uint8_t* atoms, float* ts, int* rowc, cudaStream_t s, bool pdl = false);
 // h (fp32 [P][I]) -> codes [P][I/2], scales [P][I/16], tensor scales [P], atoms [chunk][I/64][512]
 cudaError_t launch_act_quant_h(const float* h, int P, const int* rowc, uint8_t* codes, uint8_t* scales, uint8_t* atoms,
                                float* ts, bool pdl, cudaStream_t s);
@@ -130,13 +148,14 @@ cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* wr, int T, i
 // logits: `nsplit` partial logit arrays [nsplit][T][E], summed in slice order; the sums are also
 // written to logits_out [T][E] when it is not null.
 cudaError_t launch_topk(const float* logits, int nsplit, float* logits_out, int T, int E, int K, float floor_, int* ids,
-                        float* wts, unsigned flags, unsigned* err, cudaStream_t s);
+                        float* wts, unsigned flags, unsigned* err, cudaStream_t s, bool pdl = false);
 // chunk_base (may be null): [E] the first 64-row chunk of each expert, chunks numbered over all experts
 // in ascending order (an exclusive prefix of ceil(count / 64)); the W4A4 path addresses its
 // activation scale atoms by chunk.
 cudaError_t launch_permute(const int* ids, int T, int K, int E, int* counts, int* offsets, int* perm, int* inv,
-                           int* chunk_base, unsigned flags, unsigned* err, cudaStream_t s);
-cudaError_t launch_xg(const uint16_t* x, int T, int K, const int* inv, int rotate, __half* xg, cudaStream_t s);
+                           int* chunk_base, unsigned flags, unsigned* err, cudaStream_t s, bool pdl = false);
+cudaError_t launch_xg(const uint16_t* x, int T, int K, const int* inv, int rotate, __half* xg, cudaStream_t s,
+                      bool pdl = false);
 
 cudaError_t launch_prefill_combine(const __half* o, const float* ys, const float* w, const int* inv, int T, int K,
                                    float routed_scale, uint16_t* y, bool pdl, cudaStream_t s);

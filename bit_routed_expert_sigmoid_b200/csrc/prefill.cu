@@ -509,9 +509,11 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shared_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bb.tmem;
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
+      pdl_wait();    // a programmatic launch (shared down) reads the previous kernel's hidden pair
       int it = 0;
       for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
         const int ks = t / (nrp * nch), tr = t - ks * (nrp * nch);   // K slice (router only)
@@ -667,21 +669,6 @@ cudaError_t allow_smem(Kern kernel, int bytes) {
 
 }  // namespace
 
-template <typename Kern, typename... Args>
-cudaError_t launch_maybe_pdl(Kern kernel, int grid, int threads, int smem, bool pdl, cudaStream_t s, Args... args) {
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, args...);
-}
-
 cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, int n_sm, bool pdl, cudaStream_t s) {
   static bool smem_set = false;
   if (!smem_set) {
@@ -694,21 +681,21 @@ cudaError_t launch_prefill_routed(const PrefillParams& p, int fmt, int phase, in
   }
   if (fmt == kInt4) {
     return phase == kPhaseGateUp
-               ? launch_maybe_pdl(pf_routed_kernel<kInt4, kPhaseGateUp>, n_sm, PfRoles<kInt4, kPhaseGateUp>::kThreads,
+               ? launch_pdl_kernel(pf_routed_kernel<kInt4, kPhaseGateUp>, n_sm, PfRoles<kInt4, kPhaseGateUp>::kThreads,
                                   kPfSmem, pdl, s, p)
-               : launch_maybe_pdl(pf_routed_kernel<kInt4, kPhaseDown>, n_sm, PfRoles<kInt4, kPhaseDown>::kThreads,
+               : launch_pdl_kernel(pf_routed_kernel<kInt4, kPhaseDown>, n_sm, PfRoles<kInt4, kPhaseDown>::kThreads,
                                   kPfSmem, pdl, s, p);
   } else {
     return phase == kPhaseGateUp
-               ? launch_maybe_pdl(pf_routed_kernel<kNvfp4, kPhaseGateUp>, n_sm, PfRoles<kNvfp4, kPhaseGateUp>::kThreads,
+               ? launch_pdl_kernel(pf_routed_kernel<kNvfp4, kPhaseGateUp>, n_sm, PfRoles<kNvfp4, kPhaseGateUp>::kThreads,
                                   kPfSmem, pdl, s, p)
-               : launch_maybe_pdl(pf_routed_kernel<kNvfp4, kPhaseDown>, n_sm, PfRoles<kNvfp4, kPhaseDown>::kThreads,
+               : launch_pdl_kernel(pf_routed_kernel<kNvfp4, kPhaseDown>, n_sm, PfRoles<kNvfp4, kPhaseDown>::kThreads,
                                   kPfSmem, pdl, s, p);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, cudaStream_t s) {
+cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, cudaStream_t s, bool pdl) {
   static bool smem_set = false;
   if (!smem_set) {
     cudaError_t e;
@@ -722,16 +709,15 @@ cudaError_t launch_prefill_shared(const PrefillParams& p, int phase, int n_sm, c
                                        : (p.E + 255) / 256 * kRouterSplit;
   const int tiles = rp * ((p.T + 127) / 128);
   const int grid = tiles < n_sm ? tiles : n_sm;
-  if (phase == kPhaseGateUp) pf_shared_kernel<kPhaseGateUp><<<grid, kShThreads, sh_smem<kPhaseGateUp>(), s>>>(p);
-  else if (phase == kPhaseDown) pf_shared_kernel<kPhaseDown><<<grid, kShThreads, sh_smem<kPhaseDown>(), s>>>(p);
-  else pf_shared_kernel<kPhaseRouter><<<grid, kShThreads, sh_smem<kPhaseRouter>(), s>>>(p);
-  return cudaGetLastError();
+  if (phase == kPhaseGateUp) return launch_pdl_kernel(pf_shared_kernel<kPhaseGateUp>, grid, kShThreads, sh_smem<kPhaseGateUp>(), pdl, s, p);
+  if (phase == kPhaseDown) return launch_pdl_kernel(pf_shared_kernel<kPhaseDown>, grid, kShThreads, sh_smem<kPhaseDown>(), pdl, s, p);
+  return launch_pdl_kernel(pf_shared_kernel<kPhaseRouter>, grid, kShThreads, sh_smem<kPhaseRouter>(), pdl, s, p);
 }
 
 cudaError_t launch_prefill_combine(const __half* o, const float* ys, const float* w, const int* inv, int T, int K,
                                    float routed_scale, uint16_t* y, bool pdl, cudaStream_t s) {
   static_assert(kH == 256 * 8, "one CTA of 256 threads x 8 columns per token");
-  return launch_maybe_pdl(pf_combine_kernel<kMaxTopK>, T, 256, 0, pdl, s, o, ys, w, inv, K, routed_scale, y);
+  return launch_pdl_kernel(pf_combine_kernel<kMaxTopK>, T, 256, 0, pdl, s, o, ys, w, inv, K, routed_scale, y);
 }
 
 }  // namespace flint

@@ -80,6 +80,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
                                                    float* __restrict__ logits_out, int T, int E, int K,
                                                    float floor_, int* __restrict__ ids, float* __restrict__ wts,
                                                    unsigned flags, unsigned* __restrict__ err) {
+  pdl_wait();                                      // the logits are the previous kernel's output
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
   if (t >= T) return;
@@ -190,6 +192,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __rest
                                                                int* __restrict__ chunk_base, unsigned flags,
                                                                unsigned* __restrict__ err) {
   __shared__ int h_total[kMaxE], h_before[kMaxE], first[kMaxE];
+  pdl_wait();                                      // the ids are the previous kernel's output
+  pdl_trigger();
   __shared__ int wcnt[kPermWarps * kMaxE];        // [warp][expert]: pairs of the expert in the warp
   __shared__ int scan_w[kMaxE / 32], scan_c[kMaxE / 32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -305,6 +309,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __rest
 // 0,4,1,5,2,6,3,7 to match the fp16 pairs the int4 decoder produces.
 __global__ void __launch_bounds__(256) xg_kernel(const uint16_t* __restrict__ x, int T, int K,
                                                  const int* __restrict__ inv, int rotate, __half* __restrict__ xg) {
+  pdl_wait();                                      // inv is the previous kernel's output
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gw = blockIdx.x * 8 + warp;
   const int t = gw / (kH / kGroup), seg = gw % (kH / kGroup);
@@ -330,28 +336,28 @@ cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* wr, int T, i
 }
 
 cudaError_t launch_topk(const float* logits, int nsplit, float* logits_out, int T, int E, int K, float floor_, int* ids,
-                        float* wts, unsigned flags, unsigned* err, cudaStream_t s) {
+                        float* wts, unsigned flags, unsigned* err, cudaStream_t s, bool pdl) {
   if (nsplit == kRouterSplit)
-    topk_kernel<kRouterSplit><<<(T + 7) / 8, 256, 0, s>>>(logits, logits_out, T, E, K, floor_, ids, wts, flags, err);
-  else if (nsplit == 1)
-    topk_kernel<1><<<(T + 7) / 8, 256, 0, s>>>(logits, logits_out, T, E, K, floor_, ids, wts, flags, err);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+    return launch_pdl_kernel(topk_kernel<kRouterSplit>, (T + 7) / 8, 256, 0, pdl, s, logits, logits_out, T, E, K,
+                             floor_, ids, wts, flags, err);
+  if (nsplit == 1)
+    return launch_pdl_kernel(topk_kernel<1>, (T + 7) / 8, 256, 0, pdl, s, logits, logits_out, T, E, K, floor_, ids,
+                             wts, flags, err);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_permute(const int* ids, int T, int K, int E, int* counts, int* offsets, int* perm, int* inv,
-                           int* chunk_base, unsigned flags, unsigned* err, cudaStream_t s) {
+                           int* chunk_base, unsigned flags, unsigned* err, cudaStream_t s, bool pdl) {
   const int P = T * K;
   const int grid = P > 0 ? (P + kPermThreads - 1) / kPermThreads : 1;
-  permute_kernel<<<grid, kPermThreads, 0, s>>>(ids, P, E, counts, offsets, perm, inv, chunk_base, flags, err);
-  return cudaGetLastError();
+  return launch_pdl_kernel(permute_kernel, grid, kPermThreads, 0, pdl, s, ids, P, E, counts, offsets, perm, inv, chunk_base,
+                           flags, err);
 }
 
-cudaError_t launch_xg(const uint16_t* x, int T, int K, const int* inv, int rotate, __half* xg, cudaStream_t s) {
+cudaError_t launch_xg(const uint16_t* x, int T, int K, const int* inv, int rotate, __half* xg, cudaStream_t s,
+                      bool pdl) {
   const int warps = T * (kH / kGroup);
-  xg_kernel<<<(warps + 7) / 8, 256, 0, s>>>(x, T, K, inv, rotate, xg);
-  return cudaGetLastError();
+  return launch_pdl_kernel(xg_kernel, (warps + 7) / 8, 256, 0, pdl, s, x, T, K, inv, rotate, xg);
 }
 
 }  // namespace flint

@@ -20,12 +20,6 @@ constexpr int kPfN = 64;                     // tokens per tile (MMA N, padded t
 // ---------------------------------------------------------------------------------------------
 // tcgen05 / TMA primitives
 
-// Programmatic dependent launch: the next kernel of the stream may be scheduled once every CTA of this
-// one has called launch_dependents (or exited); wait blocks until the previous kernel has completed
-// and its writes are visible (a no-op without a programmatic predecessor).
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 

@@ -142,6 +142,8 @@ __global__ void __launch_bounds__(256) act_quant_x_kernel(const uint16_t* __rest
   __shared__ float wmax[8];
   __shared__ int dst_row[kMaxTopK], dst_pos[kMaxTopK];
   const int t = blockIdx.x, i = threadIdx.x, warp = i >> 5, lane = i & 31;
+  pdl_wait();                                      // ids, inv, offsets and chunk_base: the permutation's output
+  pdl_trigger();
   if (warp == 0 && lane < top_k) {
     const int e = min(max(__ldg(ids + t * top_k + lane), 0), E - 1);
     const int p = __ldg(inv + t * top_k + lane);
@@ -528,21 +530,6 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a4_kernel(const __grid_consta
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
 }
 
-template <typename Kern>
-cudaError_t launch_pdl(Kern kernel, int grid, int threads, int smem, bool pdl, cudaStream_t s, const PrefillParams& p) {
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, p);
-}
-
 }  // namespace
 
 size_t w4a4_chunk_capacity(size_t P, int E) { return (P + 63) / 64 + static_cast<size_t>(E); }
@@ -558,26 +545,18 @@ cudaError_t launch_pack_sf_atoms(const uint8_t* scales, int rows, int K, uint8_t
 
 cudaError_t launch_act_quant_x(const uint16_t* x, int T, int K, int E, const int* ids, const int* inv,
                                const int* offsets, const int* chunk_base, uint8_t* codes, uint8_t* scales,
-                               uint8_t* atoms, float* ts, int* rowc, cudaStream_t s) {
+                               uint8_t* atoms, float* ts, int* rowc, cudaStream_t s, bool pdl) {
   if (T <= 0) return cudaSuccess;
-  act_quant_x_kernel<<<T, 256, 0, s>>>(x, K, E, ids, inv, offsets, chunk_base, codes, scales, atoms, ts, rowc);
-  return cudaGetLastError();
+  return launch_pdl_kernel(act_quant_x_kernel, T, 256, 0, pdl, s, x, K, E, ids, inv, offsets, chunk_base, codes, scales,
+                           atoms, ts, rowc);
 }
 
 cudaError_t launch_act_quant_h(const float* h, int P, const int* rowc, uint8_t* codes, uint8_t* scales, uint8_t* atoms,
                                float* ts, bool pdl, cudaStream_t s) {
   if (P <= 0) return cudaSuccess;
   constexpr int kRows = 256 / (kI / 8);
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((P + kRows - 1) / kRows);
-  cfg.blockDim = dim3(256);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, act_quant_h_kernel, h, P, rowc, codes, scales, atoms, ts);
+  return launch_pdl_kernel(act_quant_h_kernel, (P + kRows - 1) / kRows, 256, 0, pdl, s, h, P, rowc, codes, scales, atoms,
+                           ts);
 }
 
 cudaError_t launch_w4a4_routed(const PrefillParams& p, int phase, int n_sm, bool pdl, cudaStream_t s) {
@@ -592,8 +571,8 @@ cudaError_t launch_w4a4_routed(const PrefillParams& p, int phase, int n_sm, bool
       return e;
     smem_set = true;
   }
-  return phase == kPhaseGateUp ? launch_pdl(w4a4_kernel<kPhaseGateUp>, n_sm, kW4Threads, kW4Smem, pdl, s, p)
-                               : launch_pdl(w4a4_kernel<kPhaseDown>, n_sm, kW4Threads, kW4Smem, pdl, s, p);
+  return phase == kPhaseGateUp ? launch_pdl_kernel(w4a4_kernel<kPhaseGateUp>, n_sm, kW4Threads, kW4Smem, pdl, s, p)
+                               : launch_pdl_kernel(w4a4_kernel<kPhaseDown>, n_sm, kW4Threads, kW4Smem, pdl, s, p);
 }
 
 }  // namespace flint
