@@ -178,6 +178,42 @@ def test_w4a4_full_size_workload_sampled():
     dev.close()
 
 
+def test_w4a4_smallest_batch_in_a_larger_handle():
+    # T = 9, the smallest batch of the tensor-core path (mostly one-row chunks), on a handle sized for
+    # 300 tokens (chunk numbering and atom arrays larger than used)
+    L = layer(256)
+    T = 9
+    x = S.make_workload_x(T, 256)
+    dev, y = run(L, x, t_max=300)
+    d = fetch(dev, T)
+    active = np.nonzero(np.diff(d["offsets"]))[0]
+    assert check_stages(L, x, d, active) == T * K
+    ref = R.moe_forward(L, x, top_k=K, w4a4=True)
+    PT.check_routing(dev.routing(T), ref, T, K)
+    st = PT.compare_y(y_to_host_bits(y), ref["y"])
+    assert st["finite"] and st["violations"] == 0, st
+    dev.close()
+
+
+def test_w4a4_skewed_loads_sampled():
+    # skewed router (hot experts with up to ~800 rows: 13 chunks of 64, and idle experts): quantisers on
+    # every row, projections of the hottest and of a few other experts, y on sampled tokens
+    L = layer(256, skew=True)
+    T = 2048
+    x = S.make_workload_x(T, 256, skew=True)
+    dev, y = run(L, x)
+    d = fetch(dev, T)
+    counts = np.diff(d["offsets"])
+    assert counts.max() > 640 and (counts == 0).any()
+    experts = sorted({int(np.argmax(counts))} | {int(e) for e in np.nonzero(counts)[0][::40]})
+    assert check_stages(L, x, d, experts) > counts.max()
+    sample = np.array([0, 5, 1024, 2047])
+    ref = R.moe_forward(L, x[sample], top_k=K, w4a4=True)
+    st = PT.compare_y(y_to_host_bits(y)[sample], ref["y"])
+    assert st["finite"] and st["violations"] == 0, st
+    dev.close()
+
+
 def test_w4a4_is_deterministic():
     # repeated forwards agree bit for bit: y, and the gate|up output h before its quantisation
     L = layer(256)
