@@ -51,3 +51,39 @@ def test_quant_bytes_per_weight(fmt):
     reads = 2 * rows * cols * (1 if fmt == "int4" else 2)        # NVFP4 reads the input twice (amax pass)
     assert bench.quant_bytes_per_weight(fmt) * rows * cols == pytest.approx(reads + codes + scales)
     assert np.isclose(bench.quant_bytes_per_weight("int4"), 2.515625)
+
+
+def test_w4a4_stage_bytes_match_the_arrays():
+    # W4A4: the routed stages read the NVFP4 weight arrays and the NVFP4 activation rows (codes, block
+    # scales, one fp32 tensor scale per row); gate|up writes fp32 h, down reads h's NVFP4 rows and writes fp16 o
+    L = S.make_layer(32, "nvfp4")
+    E, T, K, n = 32, 2048, 6, 5
+    P = T * K
+    gu_w = (L["gu_codes"].nbytes + L["gu_scales"].nbytes + L["gu_tscale"].nbytes) // E
+    dn_w = (L["dn_codes"].nbytes + L["dn_scales"].nbytes + L["dn_tscale"].nbytes) // E
+    xa = P * (bench.H // 2 + bench.H // 16 + 4)
+    ha = P * (bench.I // 2 + bench.I // 16 + 4)
+    assert bench.stage_bytes("gu_routed", E, "nvfp4", T, K, n, w4a4=True) == n * gu_w + xa + P * bench.I * 4
+    assert bench.stage_bytes("dn_routed", E, "nvfp4", T, K, n, w4a4=True) == n * dn_w + ha + P * bench.H * 2
+    assert bench.stage_bytes("hq", E, "nvfp4", T, K, n, w4a4=True) == P * bench.I * 4 + ha
+    # the other stages are those of the 16-bit-activation path
+    for st in ("router_logits", "topk", "permute", "gu_shared", "dn_shared", "combine"):
+        assert bench.stage_bytes(st, E, "nvfp4", T, K, n, w4a4=True) == bench.stage_bytes(st, E, "nvfp4", T, K, n)
+
+
+def test_prefill_roofline_picks_the_slower_roofline():
+    peaks = {"hbm_gbs": 6554.6, "bf16_tflops": 1657.2, "source": "measured"}
+    E, T, n = 256, 2048, 256
+    # W4A4 gate|up at T = 2048: 341 MB at 6.55 TB/s (52 µs) against 51.5 GFLOP at 4 x 1657 TF (7.8 µs): HBM
+    r = bench.prefill_roofline("gu_routed", 0.0663, E, "nvfp4", T, n, peaks, "prefill_nvfp4_w4a4", True)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == peaks["hbm_gbs"]
+    assert r["achieved"] == pytest.approx(bench.stage_bytes("gu_routed", E, "nvfp4", T, 6, n, True) / 66.3e-6 / 1e9, rel=1e-3)
+    assert r["frac"] == pytest.approx(r["achieved"] / peaks["hbm_gbs"], rel=1e-3)
+    # with a hypothetical HBM ten times faster the FP4 tensor time is the larger: tensor, peak = 4 x bf16
+    fast = dict(peaks, hbm_gbs=65546.0)
+    r = bench.prefill_roofline("gu_routed", 0.0663, E, "nvfp4", T, n, fast, "prefill_nvfp4_w4a4", True)
+    assert r["bound"] == "tensor" and r["peak"] == pytest.approx(4 * peaks["bf16_tflops"], rel=1e-3)
+    # W4A16: always the bf16 tensor peak (fp16 MMAs at the bf16 rate)
+    r = bench.prefill_roofline("gu_routed", 0.12, E, "int4", T, n, peaks, "prefill_int4", False)
+    assert r["bound"] == "tensor" and r["peak"] == peaks["bf16_tflops"]
+    assert r["achieved"] == pytest.approx(bench.stage_flops("gu_routed", E, T, 6) / 0.12e-3 / 1e12, rel=1e-3)
