@@ -51,6 +51,27 @@ def test_workspace_size_rules():
         assert (B.flint_moe_workspace_size(cfg) > 0) == ok, bad
 
 
+def test_w4a4_configuration_rules():
+    # W4A4 is an NVFP4 mode: refused for int4 and for expert-cache handles; it adds the NVFP4 activation
+    # rows of x and h, their scale atoms per 64-row chunk, the chunk positions and numbering, and the
+    # weight scales as atoms (all 256-byte aligned pieces of the workspace)
+    W = B.FLINT_FLAG_W4A4
+    assert B.flint_moe_workspace_size(_cfg(fmt=B.FLINT_W_INT4_G128_FWHT128, flags=W)) == 0
+    assert B.flint_moe_workspace_size(_cfg(fmt=B.FLINT_W_NVFP4, flags=W, n_slots=64)) == 0
+    T, K, E, H, I = 2048, 6, 256, 2048, 512
+    plain = B.flint_moe_workspace_size(_cfg(fmt=B.FLINT_W_NVFP4, t_max=T))
+    w4 = B.flint_moe_workspace_size(_cfg(fmt=B.FLINT_W_NVFP4, t_max=T, flags=W))
+    P = T * K
+    chunks = (P + 63) // 64 + E
+    al = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    extra = (al(P * H // 2) + al(P * H // 16) + al(P * 4) + al(P * I // 2) + al(P * I // 16) + al(P * 4)
+             + al(P * 4) + al(E * 4) + al(chunks * (H // 64) * 512) + al(chunks * (I // 64) * 512)
+             + al(E * (2 * I // 128) * (H // 64) * 512) + al(E * (H // 128) * (I // 64) * 512))
+    assert w4 - plain == extra
+    # the debug-check flag changes nothing in the workspace
+    assert B.flint_moe_workspace_size(_cfg(fmt=B.FLINT_W_NVFP4, t_max=T, flags=B.FLINT_FLAG_DEBUG_CHECKS)) == plain
+
+
 def test_create_rejects_bad_pointers_without_a_device():
     cfg = _cfg()
     w = B.flint_moe_weights(*([0x1000] * 9))
