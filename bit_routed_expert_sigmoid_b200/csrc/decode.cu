@@ -6,10 +6,10 @@
 // (an arrival counter and a generation word in global memory, one bounded wait per CTA), not a
 // kernel boundary, and every SM keeps weight copies in flight across it.
 //
-//   phase A  no dependencies. Warps 4-6 compute the router logits (a warp per router row, x staged
-//            by one bulk copy) and the routed experts' activation operand (a warp per 128-segment
-//            of a token); warps 0-3 start streaming the shared expert's gate|up tiles at once; one
-//            thread asks L2 for the shared expert's down rows.
+//   phase A  no dependencies (12 warps per CTA). Warps 4-7 compute the router logits (a K quarter
+//            each, x staged by one bulk copy) and the routed experts' activation operand (a warp per
+//            128-segment of a token); warps 0-3 start streaming the shared expert's gate|up tiles at
+//            once; one thread asks L2 for the shared expert's down rows.
 //   barrier 1
 //   phase B  every CTA selects the top-k of every token from the logits (a warp per token) and
 //            builds the routing tables in its own shared memory; then the routed gate|up tiles of
@@ -53,10 +53,10 @@ namespace {
 constexpr uint64_t kWaitNs = FLINT_WAIT_NS;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
-constexpr int kWarps = 8;                    // warps per CTA
-constexpr int kThreads = kWarps * 32;
-constexpr int kRouteWarp0 = 4;               // warps 4..7: router rows, operand, top-k, tables
-constexpr int kRouteThreads = (kWarps - kRouteWarp0) * 32;
+constexpr int kRouteWarp0 = 4;               // warps 4..7: router rows, operand
+constexpr int kRouteWarps = 4;               // one per K quarter of the router rows
+constexpr int kRouteThreads = kRouteWarps * 32;
+constexpr int kTabWarps = kMaxE / 32;        // the routing tables take one thread per expert
 constexpr int kBarRoute = 1;                 // named barrier of the routing warps
 constexpr int kMaxRowsPerCta = 16;           // phase C rows of y per CTA (one MMA tile)
 constexpr int kShDnSlices = kIs / kGroup;    // shared down K slices of 128 (8)
@@ -362,7 +362,7 @@ struct RouteSmem {
   unsigned mask[kMaxE];                     // table scratch: token bit masks
   int4 etab[kMaxActive][2];                 // active experts: {e, offset, count, tokens}, {ts_g, ts_u, ts_d, 0}
   int na;                                   // number of active experts
-  int wsum[8];                              // table scan: per-warp sums
+  int wsum[kTabWarps];                      // table scan: per-warp sums
   float rpart[4][2][kDecodeMaxT];           // router: partial logits of the CTA's two rows per K quarter
 };
 
@@ -429,7 +429,7 @@ __device__ __forceinline__ void topk_select(const DecodeParams& p, int tok, cons
   }
 }
 
-// Routing tables from the selected ids, by all 256 threads of the CTA (tid; every thread calls it):
+// Routing tables from the selected ids, by the CTA's threads (tid; every thread calls it):
 // the P = T*K pairs count their experts and set their token bits with shared-memory atomics (sums
 // and ORs, so the result does not depend on the order they run in); thread e then holds expert e,
 // and one scan over the experts (two 16-bit sums packed in a word: counts and active flags, neither
@@ -441,8 +441,11 @@ __device__ __forceinline__ void topk_select(const DecodeParams& p, int tok, cons
 __device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& rs, bool publish, int tid) {
   const int lane = tid & 31, w = tid >> 5;
   const int T = p.T, E = p.E, K = p.K, P = T * K;
-  rs.cnt[tid] = 0;
-  rs.mask[tid] = 0u;
+  const bool te = tid < kMaxE;                     // threads past the last expert only join the barriers
+  if (te) {
+    rs.cnt[tid] = 0;
+    rs.mask[tid] = 0u;
+  }
   __syncthreads();
   if (tid < P) {
     const int id = rs.ids[tid];
@@ -451,8 +454,8 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& r
   }
   __syncthreads();
   const int e = tid;
-  const int cnt = e < E ? rs.cnt[e] : 0;
-  const unsigned msk = rs.mask[e];
+  const int cnt = te && e < E ? rs.cnt[e] : 0;
+  const unsigned msk = te ? rs.mask[e] : 0u;
   const unsigned own = static_cast<unsigned>(cnt) | (static_cast<unsigned>(cnt > 0) << 16);
   unsigned inc = own;
 #pragma unroll
@@ -460,23 +463,23 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, RouteSmem& r
     const unsigned o = __shfl_up_sync(kFull, inc, m);
     if (lane >= m) inc += o;
   }
-  if (lane == 31) rs.wsum[w] = static_cast<int>(inc);
+  if (lane == 31 && te) rs.wsum[w] = static_cast<int>(inc);
   __syncthreads();
   unsigned before = 0u, total = 0u;
 #pragma unroll
-  for (int v = 0; v < kWarps; ++v) {
+  for (int v = 0; v < kTabWarps; ++v) {
     const unsigned x = static_cast<unsigned>(rs.wsum[v]);
     if (v < w) before += x;
     total += x;
   }
   const unsigned ex = before + inc - own;          // exclusive prefix (packed)
   const int off = static_cast<int>(ex & 0xFFFF), slot = static_cast<int>(ex >> 16);
-  rs.cnt[e] = off;                                 // every count was read before the barrier above
-  if (e < E && publish) {
+  if (te) rs.cnt[e] = off;                         // every count was read before the barrier above
+  if (te && e < E && publish) {
     p.counts[e] = cnt;
     p.offsets[e] = off;
   }
-  if (e < E && cnt > 0) {
+  if (te && e < E && cnt > 0) {
     unsigned toks = 0u, m = msk;
     for (int n = 0; m; ++n) {
       const int tt = __ffs(m) - 1;
@@ -569,18 +572,22 @@ constexpr int kShGuTiles = kIs / 2;         // shared gate|up tiles: 2 hs column
 constexpr int kGuTilesPerExpert = kI / 8;   // 64 routed gate|up tiles: 8 h columns (8 gate + 8 up rows) each
 constexpr int kTokPitch = 2 * kH + 64;      // bytes per staged token row of x or of the routed operand
 
-// Per-warp ring of weight stages. int4: 4 stages of 4096 B codes (+256 B for phase C's scales);
-// NVFP4: 3 stages of 4096 B codes + 512 B of block scales.
+// Warps per CTA and the per-warp ring of weight stages. 12 warps (three per scheduler) keep more
+// independent MMA chains in flight than 8; the shared memory then holds two stages per warp. int4:
+// 4096 B of codes (+256 B for phase C's scales); NVFP4: 4096 B of codes + 512 B of block scales.
 template <int FMT>
 struct Geom {
-  static constexpr int kDepth = FMT == kInt4 ? 4 : 3;
+  static constexpr int kWarps = 12;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kDepth = 2;
   static constexpr int kStage = FMT == kInt4 ? 4096 + 256 : 4096 + 512;
+  static_assert(kWarps >= kRouteWarp0 + kRouteWarps && kWarps * 32 >= kMaxE, "warp roles");
 };
 
 template <int FMT>
 struct DecShared {
-  alignas(128) uint8_t stage[kWarps][Geom<FMT>::kDepth][Geom<FMT>::kStage];
-  alignas(16) uint8_t gu_sc[FMT == kInt4 ? kWarps : 1][2][16 * (kH / kGroup) * 2];   // int4: tile scales, 2 tiles
+  alignas(128) uint8_t stage[Geom<FMT>::kWarps][Geom<FMT>::kDepth][Geom<FMT>::kStage];
+  alignas(16) uint8_t gu_sc[FMT == kInt4 ? Geom<FMT>::kWarps : 1][2][16 * (kH / kGroup) * 2];   // int4: tile scales
   union {
     struct {                                          // phases A and B
       alignas(128) uint8_t xs[kDecodeMaxT][kTokPitch];  // x, bf16
@@ -595,7 +602,7 @@ struct DecShared {
     } c;
   } u;
   RouteSmem rs;
-  uint64_t full[kWarps][Geom<FMT>::kDepth];
+  uint64_t full[Geom<FMT>::kWarps][Geom<FMT>::kDepth];
   uint64_t xbar, xqbar, hqbar, logits_ready;
   unsigned long long bar_base;                        // the grid barriers' counter at the forward's start
 };
@@ -756,8 +763,9 @@ __device__ void dn_issue(const DecodeParams& p, Ring<FMT>& ring, int item, int r
 }
 
 template <int FMT>
-__global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(Geom<FMT>::kThreads, 1) decode_layer_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int D = Geom<FMT>::kDepth;
+  constexpr int kWarps = Geom<FMT>::kWarps, kThreads = Geom<FMT>::kThreads;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   DecShared<FMT>& sm = *reinterpret_cast<DecShared<FMT>*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -790,14 +798,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
     for (int r = 0; r < p.T; ++r) bulk_g2s(sm.u.ab.xs[r], p.x + static_cast<size_t>(r) * kH, kH * 2, &sm.xbar);
   }
   int k_issue = 0;                                 // next gate|up stage to issue: tile k_issue >> 2, quarter & 3
-  if (warp >= kRouteWarp0) {
+  if (warp >= kRouteWarp0 && warp < kRouteWarp0 + kRouteWarps) {
     // router rows c and c + G on the tensor cores (K quarter rw each), then the operand segments
     const int rw = warp - kRouteWarp0, ri = threadIdx.x - kRouteWarp0 * 32;
     RouterRows rr;
     if (!p.route_in) rr.load(p, rw, c + G * g);
     wait_stage(p, &sm.xbar, 0);
     if (!p.route_in) rr.mma(p, rw, sm.u.ab.xs[0], kTokPitch, sm.rs.rpart);
-    if (rw == kWarps - kRouteWarp0 - 1)
+    if (rw == kRouteWarps - 1)
       for (int sg = c; sg < p.T * (kH / kGroup); sg += G)
         xq_segment(p, sg / (kH / kGroup), sg % (kH / kGroup), sm.u.ab.xs[0], kTokPitch);
     named_bar_sync(kBarRoute, kRouteThreads);
@@ -823,9 +831,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_layer_kernel(const __grid_
       mbar_arrive(&sm.logits_ready);
     }
   } else {
-    // the shared expert needs no routing, but x and the router rows go first: its gate|up stages
-    // (the ring holds the warp's whole shared tile) and the L2 fetch of its down rows start once x
-    // has landed
+    // the shared expert needs no routing (its tiles fall to warps 0-3; warps 8-11 have no phase A
+    // work), but x and the router rows go first: its first gate|up stages (as many as the ring
+    // holds) and the L2 fetch of its down rows start once x has landed
     wait_stage(p, &sm.xbar, 0);
     while (ring.has_room() && tile_of(k_issue >> 2) < kShGuTiles) {
       gu_issue<FMT>(p, sm, ring, warp, k_issue & 3, k_issue >> 2, tile_of(k_issue >> 2), ExpertInfo{});
@@ -1158,8 +1166,10 @@ cudaError_t decode_check_residency(int fmt, int* blocks_per_sm) {
                                : allow_smem(decode_layer_kernel<kNvfp4>, smem);
   if (e != cudaSuccess) return e;
   return fmt == kInt4
-             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, decode_layer_kernel<kInt4>, kThreads, smem)
-             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, decode_layer_kernel<kNvfp4>, kThreads, smem);
+             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, decode_layer_kernel<kInt4>,
+                                                             Geom<kInt4>::kThreads, smem)
+             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, decode_layer_kernel<kNvfp4>,
+                                                             Geom<kNvfp4>::kThreads, smem);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int n_sm, cudaStream_t s) {
@@ -1168,7 +1178,7 @@ cudaError_t launch_decode(const DecodeParams& p, int n_sm, cudaStream_t s) {
   const size_t smem = decode_smem_bytes(p.fmt);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(n_sm);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(p.fmt == kInt4 ? Geom<kInt4>::kThreads : Geom<kNvfp4>::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
