@@ -251,8 +251,9 @@ const char* flint_moe_stage_name(flint_moe_t h, int T, int i);
  * (a multiple of 32); larger sizes return FLINT_ERR_INVALID_ARG without launching anything. Calls no
  * cudaMalloc or cudaFree. The first call in a CUDA context looks up the array's device address (once
  * per device and context, with that device current); a context destroyed and re-created
- * (cudaDeviceReset) is noticed and the address looked up again. All calls share the one array: calls whose kernels may overlap on the GPU (different streams
- * without ordering) race on it and must be serialised by the caller. */
+ * (cudaDeviceReset) is noticed and the address looked up again. All calls share the one array:
+ * calls whose kernels may overlap on the GPU (different streams without ordering) race on it and
+ * must be serialised by the caller. */
 flint_status flint_moe_route_noalloc(const void* x, const void* router_w, int T, int n_experts, int top_k,
                                      float norm_floor, int* ids, float* w, void* stream);
 
