@@ -82,9 +82,9 @@ def test_fixed_points_and_bounds():
 
 
 def test_w4a4_layer_structure():
-    # with W4A4 the routed experts see quantised inputs: a layer whose activations are exactly NVFP4
-    # values (x built on the grid with ts = 2^-8) gives the same first projection as W4A16; and the
-    # option is refused for the rotated int4 format
+    # with W4A4 the routed experts see quantised inputs: each permuted row's input is its token's
+    # quantised x, the routing is that of W4A16, y differs from W4A16; the option is refused for the
+    # rotated int4 format
     L = S.make_layer(32, "nvfp4", H=256, I=128, Is=64)
     x = S.make_x(5, H=256)
     a = R.moe_forward(L, x, w4a4=True, keep=True)
