@@ -95,3 +95,29 @@ def test_w4a4_layer_structure():
     assert not np.allclose(a["y"], b["y"])
     with pytest.raises(ValueError):
         R.moe_forward(S.make_layer(32, "int4", H=256, I=128, Is=64), x, w4a4=True)
+
+
+def test_w4a4_on_grid_inputs_matches_w4a16_up_to_the_down_input():
+    # token rows that already lie on the per-row NVFP4 grid are quantised to themselves: each row is
+    # E2M1 code x E4M3 block scale x 2^-8 with a +-6 in every block and one block at scale 448, so the
+    # row's tensor scale is exactly 2^-8 and every block scale and code comes back (and such values are
+    # exact in bf16). The W4A4 layer's routed inputs, gate|up and SwiGLU outputs are then those of the
+    # 16-bit-activation layer bit for bit; only the down input differs (h is quantised, x was not)
+    # (kekzle/Flint-NVFP4, evaluation table: W4A4 quantises the activations of the same NVFP4 weights)
+    L = S.make_layer(32, "nvfp4", H=256, I=128, Is=64)
+    rng = np.random.default_rng(7)
+    T, H = 7, 256
+    sb = rng.integers(0x20, 0x7E, size=(T, H // 16))
+    sb[:, 0] = 0x7E
+    codes = rng.integers(0, 16, size=(T, H))
+    codes[:, ::16] = 7
+    v = R.e2m1_to_f64(codes) * np.repeat(R.e4m3fn_to_f64(sb), 16, axis=1) * 2.0 ** -8
+    x_bits = S.f32_to_bf16_bits(v.astype(np.float32))
+    np.testing.assert_array_equal(R.bf16_to_f64(x_bits), v)
+    a = R.moe_forward(L, x_bits, w4a4=True, keep=True)
+    b = R.moe_forward(L, x_bits, keep=True)
+    np.testing.assert_array_equal(a["ids"], b["ids"])
+    np.testing.assert_array_equal(a["x_in"], b["x_in"])
+    np.testing.assert_array_equal(a["h"], b["h"])
+    assert not np.array_equal(a["h_in"], b["h_in"])
+    np.testing.assert_array_equal(a["ys"], b["ys"])
