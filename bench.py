@@ -544,8 +544,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                       "w4a16: tcgen05 kind::f16 MMA (weights dequantised to exact fp16 in tensor memory, fp16 "
                       "activations), fp32 accumulators in tensor memory; shared expert and router bf16"),
             "data": "synthetic (seeded; random-init weights of the Flint MoE layer shape)",
-            "config": {"workload": f"{args.workload}: E={E} top-6, H=2048, I=512, shared 1024, {fmt}, T={T} "
-                                   "tokens per GPU", "E": E, "T": T, "fmt": fmt, "distinct_experts": n_active,
+            "config": {"workload": layer_workload(args.workload, E, fmt, T), "E": E, "T": T, "fmt": fmt,
+                       "distinct_experts": n_active,
                        "l2": "flushed between timed steps (256 MiB write, outside the timed events)",
                        "parallelism": f"replicas x{world} (token-parallel, no collective)"},
             "hbm": {"algorithmic_bytes": ab, "GB_per_s": round(ab / (ms_per_step * 1e-3) / 1e9, 1),
@@ -590,6 +590,19 @@ def cpu_baseline(args, L, x_bits, E) -> dict:
             "sample": f"fp64 oracle forward of {what}, repeated {reps}x in {el:.1f} s"}
 
 
+def layer_workload(name: str, E: int, fmt: str, T: int) -> str:
+    """config.workload of a one-layer workload: the same string on both arms."""
+    return f"{name}: E={E} top-6, H=2048, I=512, shared 1024, {fmt}, T={T} tokens per GPU"
+
+
+def stack_workload(name: str, n: int, E: int, fmt: str, T: int) -> str:
+    return f"{name}: {n} layers x (E={E} top-6, H=2048, I=512, shared 1024, {fmt}), T={T}, x <- x + moe(rmsnorm(x))"
+
+
+def quant_workload(name: str, E: int, fmt: str) -> str:
+    return f"{name}: E={E} experts x (gate|up {2 * I}x{H}, down {H}x{I}) bf16 -> {fmt}"
+
+
 def run_reference(args) -> dict:
     from bit_routed_expert_sigmoid_b200 import synthetic as S
     from oracle import flint_moe_ref as R
@@ -601,7 +614,7 @@ def run_reference(args) -> dict:
                 "and down banks)", "value": v, "unit": "GB/s", "n_gpus": 1, "steps": 1, "warmup": 0,
                 "ms_per_step": round(nbytes / bps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32 decisions", "data": "synthetic",
-                "config": {"workload": f"{args.workload}: E={E} experts bf16 -> {fmt}", "E": E, "fmt": fmt},
+                "config": {"workload": quant_workload(args.workload, E, fmt), "E": E, "fmt": fmt},
                 "cpu_baseline": {"value": v, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
                                  "sample": f"oracle quantiser on 64 rows x {H}, {nbytes / 1e6:.1f} MB"},
                 "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -622,7 +635,7 @@ def run_reference(args) -> dict:
         return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": 1,
                 "steps": len(times), "warmup": 0, "ms_per_step": round(per_layer * n * 1e3, 3),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": f"{args.workload}: {n} layers, E={E} top-6, H=2048, {fmt}, T={T}", "E": E,
+                "config": {"workload": stack_workload(args.workload, n, E, fmt, T), "E": E,
                            "T": T, "fmt": fmt, "layers": n},
                 "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": blas_threads(),
                                  "kind": "oracle", "sample": sample},
@@ -645,7 +658,7 @@ def run_reference(args) -> dict:
     return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": 1,
             "steps": steps, "warmup": args.warmup, "ms_per_step": round(el / steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{args.workload}: E={E} top-6, H=2048, {fmt}, T={T}", "E": E, "T": T,
+            "config": {"workload": layer_workload(args.workload, E, fmt, T), "E": E, "T": T,
                        "fmt": fmt},
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
@@ -782,7 +795,7 @@ def run_quant(args) -> dict:
         "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32 decisions (IEEE, fixed order) from bf16 input" + (", 128-wide Hadamard rotation" if fmt == "int4" else ""),
         "data": "synthetic (seeded normal bf16 weights, std 0.02, drawn on the device)",
-        "config": {"workload": f"{args.workload}: E={E} experts x (gate|up {2 * I}x{H}, down {H}x{I}) bf16 -> {fmt}",
+        "config": {"workload": quant_workload(args.workload, E, fmt),
                    "E": E, "fmt": fmt, "weights": int(n_w),
                    "l2": f"not flushed: {in_bytes / 1e9:.2f} GB of input per step, larger than the 126 MB L2",
                    "parallelism": "single GPU"},
@@ -908,8 +921,7 @@ def run_stack(args) -> dict:
         "dtype": "w4a16: int4 codes as exact int8 on the integer tensor cores against 16-bit fixed-point "
                  "activations (int32 sums), fp32 accumulate; fp32 residual stream",
         "data": "synthetic (seeded; random-init weights of the Flint MoE layer shape, layer l seed 1000+l)",
-        "config": {"workload": f"{args.workload}: {n} layers x (E={E} top-6, H=2048, I=512, shared 1024, {fmt}), "
-                               f"T={T}, x <- x + moe(rmsnorm(x))", "E": E, "T": T, "fmt": fmt, "layers": n,
+        "config": {"workload": stack_workload(args.workload, n, E, fmt, T), "E": E, "T": T, "fmt": fmt, "layers": n,
                    "distinct_experts_per_layer": round(float(np.mean(n_active)), 2),
                    "l2": f"not flushed: {stack.weight_bytes() / 1e9:.1f} GB of weights stream through the 126 MB L2",
                    "parallelism": "single GPU"},
