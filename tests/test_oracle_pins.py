@@ -396,3 +396,24 @@ def test_combine_pairs_each_weight_with_its_own_expert(top_k):
     np.testing.assert_allclose(out["y"], routed + shared, rtol=1e-11, atol=1e-13)
     # the experts differ enough that pairing a weight with a neighbouring slot is visible
     assert np.abs(O[0] - O[1]).max() > 1e-3
+
+
+def test_stack_step_residual_identities():
+    """x_next = x + layer(bf16(rmsnorm(x))): a layer whose weights are all zero leaves the residual exactly
+    as it was; with eps = 0 the normalised input, and so the layer output, is the same for x and for any
+    positive multiple of x (closed forms of the residual + RMSNorm glue between stacked layers)."""
+    L = _small_layer(E=8)
+    Lz = dict(L)
+    for k in ("gu_codes", "dn_codes", "sh_gu", "sh_dn"):
+        Lz[k] = np.zeros_like(L[k])
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((5, 256)) * 1.26
+    st = R.stack_step(Lz, x)
+    np.testing.assert_array_equal(st["y"], 0.0)
+    np.testing.assert_array_equal(st["x_next"], x)
+    a = R.stack_step(L, x, eps=0.0)
+    b = R.stack_step(L, 8.0 * x, eps=0.0)     # a power of two keeps rmsnorm's fp64 result bit-identical
+    np.testing.assert_array_equal(a["z"], b["z"])
+    np.testing.assert_array_equal(a["y"], b["y"])
+    np.testing.assert_array_equal(b["x_next"], 8.0 * x + a["y"])
+    assert np.abs(a["y"]).max() > 0
