@@ -417,3 +417,17 @@ def test_stack_step_residual_identities():
     np.testing.assert_array_equal(a["y"], b["y"])
     np.testing.assert_array_equal(b["x_next"], 8.0 * x + a["y"])
     assert np.abs(a["y"]).max() > 0
+
+
+def test_routed_scale_scales_only_the_routed_sum():
+    """y = routed_scale * sum_k w_k o_k + shared: scale 0 leaves the shared expert alone, and the routed
+    part is linear in the scale while the routing is untouched."""
+    L = _small_layer(E=8)
+    x = S.make_x(6, H=256)
+    one = R.moe_forward(L, x)
+    zero = R.moe_forward(L, x, routed_scale=0.0)
+    half = R.moe_forward(L, x, routed_scale=0.5)
+    np.testing.assert_array_equal(zero["y"], one["ys"])
+    np.testing.assert_array_equal(half["ids"], one["ids"])
+    np.testing.assert_allclose(half["y"] - half["ys"], 0.5 * (one["y"] - one["ys"]), rtol=1e-12, atol=1e-15)
+    assert np.abs(one["y"] - one["ys"]).max() > 1e-3
